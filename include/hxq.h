@@ -1,0 +1,153 @@
+/*
+ * hxq.h -- C ABI of libhxq: the HXQ / HelixCode HelixLinear forward
+ *          y = x . W^T on NVIDIA B200 (sm_100a), W never stored dense.
+ *
+ * What is computed (sources are the pages this library follows):
+ *  - Scalar mode: W[n][k] = codebook[indices[n*K + k]], a 256-entry fp32
+ *    codebook addressed by one uint8 per weight (Zamba2-1.2B-HXQ model card,
+ *    "What is HelixCode?").
+ *  - 2D mode: weights (k, k+1), k even, of row n are one entry of a
+ *    4096-entry codebook of fp32 pairs, addressed by a 12-bit index; the
+ *    indices are packed two per 3 bytes (HXQ whitepaper, method section:
+ *    2D VQ paragraph and the "12-bit index packing" pipeline step).
+ *  - Sidecar: each (flat position p = n*K + k, fp32 value v) replaces W[n][k]
+ *    by v (HXQ whitepaper, method section, "Sidecar outlier correction").
+ *  - Forward: y[m][n] = sum_k x[m][k] * W[n][k] for bf16 x and fp32 y, the
+ *    product that the pages' HelixLinear runs in place of nn.Linear
+ *    (HXQ whitepaper, method section, buffered forward path paragraph).
+ *
+ * Layouts (all row-major, no padding, no strides):
+ *  codebook   scalar: float[256];  2D: float[4096][2] (component 0 -> even k)
+ *  indices    scalar: uint8[N][K]; 2D: uint8[3*N*K/4], a flat stream of 3-byte
+ *             groups over the pairs in row-major order g = n*K/2 + k/2; the
+ *             group's 24-bit little-endian word b0 | b1<<8 | b2<<16 holds the
+ *             even pair's index in bits 0..11 and the odd pair's in 12..23
+ *  sidecar    int64 positions (unique, in [0, N*K)) and float values
+ *  x          bf16 [M][K] (raw bits, 2 bytes per element)
+ *  y          float [M][N]
+ *
+ * Numerics: M <= 32 computes with the fp32 codebook values (error within
+ * 1e-5 * sum_k |x||w| per output); M > 32 runs the tensor-core prefill on the
+ * weights rounded to bf16 (round to nearest even) with fp32 accumulation
+ * (within 8e-3 * sum_k |x||w|). Results are bitwise repeatable run to run.
+ *
+ * Errors: every entry point validates its arguments on the host and returns
+ * a negative status without launching anything when they are wrong. Device
+ * faults surface on the stream, as usual for CUDA.
+ */
+#ifndef HXQ_H
+#define HXQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct hxq_linear* hxq_linear_t;
+
+enum {
+    HXQ_MODE_SCALAR8 = 0, /* 256 x fp32 codebook, one uint8 index per weight */
+    HXQ_MODE_VQ2D12 = 1   /* 4096 x fp32-pair codebook, 12-bit index per pair */
+};
+
+enum {
+    HXQ_OK = 0,
+    HXQ_EINVAL = -1,       /* a bad argument; nothing was launched           */
+    HXQ_ENOMEM = -2,       /* a device allocation failed                     */
+    HXQ_ECUDA = -3,        /* a CUDA runtime or driver call failed           */
+    HXQ_EUNSUPPORTED = -4, /* the current device is not an sm_100 GPU       */
+    HXQ_ETIMEOUT = -5      /* a device-side wait gave up; see hxq_linear_check */
+};
+
+/* Kernel choice for hxq_linear_forward_ex. */
+enum {
+    HXQ_KERNEL_AUTO = 0,   /* CUDA-core GEMV for M <= 4, tensor cores above  */
+    HXQ_KERNEL_GEMV = 1,   /* CUDA-core fused-decode GEMV, fp32 weights; M <= 32 */
+    HXQ_KERNEL_TC = 2      /* tcgen05 fused-decode GEMM; fp32-exact split
+                              weights (hi+mid bf16) for M <= 32, bf16 weights
+                              above                                          */
+};
+
+/*
+ * Build a HelixLinear handle on the current CUDA device.
+ *
+ *  codebook     scalar: 256 floats; 2D: 8192 floats (4096 pairs)
+ *  indices      scalar: N*K bytes; 2D: 3*N*K/4 bytes (layout above)
+ *  mode         HXQ_MODE_SCALAR8 or HXQ_MODE_VQ2D12
+ *  sidecar_pos  n_sidecar int64 flat positions n*K + k (may be NULL if 0)
+ *  sidecar_val  n_sidecar float replacement values (may be NULL if 0)
+ *  N, K         output and input features, N >= 1, K >= 8, K % 8 == 0;
+ *               2D mode additionally needs K % 4 == 0 (implied)
+ *  out          receives the handle
+ *
+ * Pointers may be device or host memory (copies use cudaMemcpyDefault).
+ * The call copies everything it needs into memory it owns, re-lays the
+ * indices out into 128-row tiles for coalesced loads (same information, rows
+ * padded to whole 16- or 64-weight chunks), sorts the sidecar into per-row
+ * patch lists, and synchronises the device before returning: the caller may
+ * free its buffers afterwards. The handle is immutable and owns a split-K
+ * workspace, so forwards on ONE handle must not overlap in time on the GPU
+ * (different streams racing on it give wrong results); different handles are
+ * independent.
+ *
+ * Returns HXQ_EINVAL for: NULL codebook/indices/out, NULL sidecar arrays with
+ * n_sidecar > 0, n_sidecar < 0 or > N*K, N < 1, K < 8, K % 8 != 0, unknown
+ * mode, a sidecar position outside [0, N*K) or repeated. HXQ_EUNSUPPORTED if
+ * the current device is not compute capability 10.0. HXQ_ENOMEM / HXQ_ECUDA
+ * on allocation / copy failures (nothing is leaked).
+ */
+int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode,
+                      const int64_t* sidecar_pos, const float* sidecar_val,
+                      int64_t n_sidecar, int N, int K, hxq_linear_t* out);
+
+/*
+ * y[M][N] = x[M][K] . W^T on `stream` (a cudaStream_t; NULL = legacy default
+ * stream). x (bf16 bits) and y (float) are device pointers; x must be 16-byte
+ * aligned. Asynchronous: returns after the launch. M >= 1.
+ * Returns HXQ_EINVAL for a NULL handle/x/y, M < 1 or a misaligned x;
+ * HXQ_ECUDA if a launch fails.
+ */
+int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M,
+                       void* stream);
+
+/*
+ * hxq_linear_forward with an explicit kernel choice (HXQ_KERNEL_*) and split
+ * count along K (0 = automatic, else 1..64), for tests and benchmarks. The
+ * numerics of each kernel are those stated above for its M range.
+ * HXQ_EINVAL additionally for an unknown kernel, split_k outside 0..64, or
+ * HXQ_KERNEL_GEMV with M > 32.
+ */
+int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M,
+                          int kernel, int split_k, void* stream);
+
+/*
+ * Test helper: write the decoded fp32 weights W[N][K] (sidecar applied) to
+ * the device buffer W_out on `stream`. Bit-exact with the definition above.
+ * Returns HXQ_EINVAL for a NULL handle or W_out, HXQ_ECUDA on launch failure.
+ */
+int hxq_decode(hxq_linear_t h, float* W_out, void* stream);
+
+/*
+ * Synchronise the device and report whether any kernel of this handle gave up
+ * a bounded device-side wait since the last check (HXQ_ETIMEOUT, then the
+ * flag is cleared) -- the tensor-core kernel bounds every pipeline wait at 2 s
+ * and returns early instead of hanging. HXQ_OK otherwise, HXQ_EINVAL for a
+ * NULL handle, HXQ_ECUDA if the device reports an error.
+ */
+int hxq_linear_check(hxq_linear_t h);
+
+/* Shape of a handle: any output pointer may be NULL. HXQ_EINVAL if h is NULL. */
+int hxq_linear_info(hxq_linear_t h, int* mode, int* N, int* K, int64_t* n_sidecar);
+
+/* Free a handle (NULL is ignored). Synchronises the device first. */
+void hxq_linear_destroy(hxq_linear_t h);
+
+/* Static description of a status code. */
+const char* hxq_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HXQ_H */

@@ -1,0 +1,102 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/hxq.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "hxq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hxq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("hxq_linear_create", "hxq_linear_forward", "hxq_decode", "hxq_linear_destroy",
+                     "hxq_strerror"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    import vq_compressed_linear_b200 as m
+    for name in declared_functions():
+        assert hasattr(m.lib, name), name          # ctypes resolves the symbol or raises
+        assert name in m.EXPORTED
+        assert callable(getattr(m, name))
+
+
+def test_no_cpu_fallback_in_binding():
+    """The binding only marshals: it must not import the oracle or numpy math."""
+    src = open(os.path.join(ROOT, "vq_compressed_linear_b200", "__init__.py")).read()
+    assert "oracle" not in src.replace("no Python or CPU fallback", "")
+    assert "import numpy" not in src
+
+
+def test_strerror():
+    import vq_compressed_linear_b200 as m
+    for code in (0, -1, -2, -3, -4, -5):
+        assert m.hxq_strerror(code)
+    assert m.hxq_strerror(-99) == "unknown status"
+
+
+def _create(m, cb, idx, mode, pos, val, ns, N, K, out=True):
+    h = ctypes.c_void_p()
+    return m.lib.hxq_linear_create(m._ptr(cb), m._ptr(idx), mode, m._ptr(pos), m._ptr(val), ns, N, K,
+                                   ctypes.byref(h) if out else None)
+
+
+@pytest.mark.parametrize("case", ["null_out", "null_cb", "null_idx", "bad_mode", "N0", "K0", "Kneg",
+                                  "K_not_mult8", "neg_sidecar", "too_many_sidecar", "null_sidecar"])
+def test_create_rejects_bad_arguments(case):
+    import vq_compressed_linear_b200 as m
+    N, K = 16, 32
+    cb = np.zeros(256, np.float32)
+    idx = np.zeros(N * K, np.uint8)
+    pos = np.array([1], np.int64)
+    val = np.array([1.0], np.float32)
+    args = dict(cb=cb, idx=idx, mode=0, pos=pos, val=val, ns=1, N=N, K=K, out=True)
+    if case == "null_out": args["out"] = False
+    if case == "null_cb": args["cb"] = None
+    if case == "null_idx": args["idx"] = None
+    if case == "bad_mode": args["mode"] = 2
+    if case == "N0": args["N"] = 0
+    if case == "K0": args["K"] = 0
+    if case == "Kneg": args["K"] = -8
+    if case == "K_not_mult8": args["K"] = 36
+    if case == "neg_sidecar": args["ns"] = -1
+    if case == "too_many_sidecar": args["ns"] = N * K + 1
+    if case == "null_sidecar": args["pos"] = None
+    assert _create(m, **args) == m.HXQ_EINVAL
+
+
+def test_forward_and_decode_reject_null_handle():
+    import vq_compressed_linear_b200 as m
+    x = np.zeros(64, np.uint16)
+    y = np.zeros(64, np.float32)
+    assert m.lib.hxq_linear_forward(None, m._ptr(x), m._ptr(y), 1, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_linear_forward_ex(None, m._ptr(x), m._ptr(y), 1, 0, 0, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_decode(None, m._ptr(y), None) == m.HXQ_EINVAL
+    assert m.lib.hxq_linear_check(None) == m.HXQ_EINVAL
+    assert m.lib.hxq_linear_info(None, None, None, None, None) == m.HXQ_EINVAL
+    m.lib.hxq_linear_destroy(None)  # ignored
+
+
+def test_create_without_device_reports_unsupported():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    import vq_compressed_linear_b200 as m
+    N, K = 16, 32
+    rc = _create(m, np.zeros(256, np.float32), np.zeros(N * K, np.uint8), 0, None, None, 0, N, K)
+    assert rc == m.HXQ_EUNSUPPORTED
+
+
+def test_build_flags_target_sm100a():
+    from vq_compressed_linear_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -1,0 +1,195 @@
+"""Python binding of libhxq, the B200 (sm_100a) HelixLinear forward.
+
+The C ABI (include/hxq.h) is the product: this module only marshals
+arguments. Every step of the forward runs in the library's CUDA kernels;
+there is no Python or CPU fallback, and importing fails loudly when the
+library has not been built (python -m vq_compressed_linear_b200.build).
+
+PyTorch is used for device memory and streams only: tensors are passed by
+data pointer, the current torch stream is passed as the cudaStream_t.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhxq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libhxq.so is missing at {LIB_PATH}: build it with "
+        "`python -m vq_compressed_linear_b200.build` (nvcc, sm_100a)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+HXQ_MODE_SCALAR8 = 0
+HXQ_MODE_VQ2D12 = 1
+HXQ_OK = 0
+HXQ_EINVAL = -1
+HXQ_ENOMEM = -2
+HXQ_ECUDA = -3
+HXQ_EUNSUPPORTED = -4
+HXQ_ETIMEOUT = -5
+HXQ_KERNEL_AUTO = 0
+HXQ_KERNEL_GEMV = 1
+HXQ_KERNEL_TC = 2
+
+_vp, _i, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+lib.hxq_linear_create.argtypes = [_vp, _vp, _i, _vp, _vp, _i64, _i, _i, ctypes.POINTER(_vp)]
+lib.hxq_linear_create.restype = _i
+lib.hxq_linear_forward.argtypes = [_vp, _vp, _vp, _i, _vp]
+lib.hxq_linear_forward.restype = _i
+lib.hxq_linear_forward_ex.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp]
+lib.hxq_linear_forward_ex.restype = _i
+lib.hxq_decode.argtypes = [_vp, _vp, _vp]
+lib.hxq_decode.restype = _i
+lib.hxq_linear_check.argtypes = [_vp]
+lib.hxq_linear_check.restype = _i
+lib.hxq_linear_info.argtypes = [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i),
+                                ctypes.POINTER(_i64)]
+lib.hxq_linear_info.restype = _i
+lib.hxq_linear_destroy.argtypes = [_vp]
+lib.hxq_linear_destroy.restype = None
+lib.hxq_strerror.argtypes = [_i]
+lib.hxq_strerror.restype = ctypes.c_char_p
+
+EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_decode",
+            "hxq_linear_check", "hxq_linear_info", "hxq_linear_destroy", "hxq_strerror")
+
+
+class HXQError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {hxq_strerror(code)} ({code})")
+
+
+def _check(code: int, what: str) -> None:
+    if code != HXQ_OK:
+        raise HXQError(code, what)
+
+
+def _ptr(t) -> int | None:
+    """Data pointer of a tensor / ndarray, or None."""
+    if t is None:
+        return None
+    if hasattr(t, "data_ptr"):
+        return t.data_ptr()
+    return t.ctypes.data
+
+
+def _stream(stream) -> int | None:
+    if stream is not None:
+        return int(getattr(stream, "cuda_stream", stream))
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+# ---- same names as the C ABI -------------------------------------------------
+
+def hxq_strerror(code: int) -> str:
+    return lib.hxq_strerror(int(code)).decode()
+
+
+def hxq_linear_create(codebook, indices, mode, sidecar_pos, sidecar_val, n_sidecar, N, K) -> int:
+    """Returns the handle (an integer); raises HXQError on failure."""
+    h = _vp()
+    _check(lib.hxq_linear_create(_ptr(codebook), _ptr(indices), int(mode), _ptr(sidecar_pos),
+                                 _ptr(sidecar_val), int(n_sidecar), int(N), int(K), ctypes.byref(h)),
+           "hxq_linear_create")
+    return h.value
+
+
+def hxq_linear_forward(h, x, y, M, stream=None) -> None:
+    _check(lib.hxq_linear_forward(h, _ptr(x), _ptr(y), int(M), _stream(stream)), "hxq_linear_forward")
+
+
+def hxq_linear_forward_ex(h, x, y, M, kernel, split_k, stream=None) -> None:
+    _check(lib.hxq_linear_forward_ex(h, _ptr(x), _ptr(y), int(M), int(kernel), int(split_k),
+                                     _stream(stream)), "hxq_linear_forward_ex")
+
+
+def hxq_decode(h, W_out, stream=None) -> None:
+    _check(lib.hxq_decode(h, _ptr(W_out), _stream(stream)), "hxq_decode")
+
+
+def hxq_linear_check(h) -> None:
+    _check(lib.hxq_linear_check(h), "hxq_linear_check")
+
+
+def hxq_linear_info(h) -> tuple[int, int, int, int]:
+    m, n, k, s = _i(), _i(), _i(), _i64()
+    _check(lib.hxq_linear_info(h, ctypes.byref(m), ctypes.byref(n), ctypes.byref(k), ctypes.byref(s)),
+           "hxq_linear_info")
+    return m.value, n.value, k.value, s.value
+
+
+def hxq_linear_destroy(h) -> None:
+    lib.hxq_linear_destroy(h)
+
+
+# ---- convenience wrapper -----------------------------------------------------
+
+class HelixLinear:
+    """A compressed nn.Linear-shaped layer owned by libhxq.
+
+    Arguments are tensors or arrays in the C ABI's layouts (host or device);
+    the handle copies them. forward() takes x as a CUDA bf16 (or raw uint16 /
+    int16 bit pattern) tensor [M, K] and returns float32 y [M, N].
+    """
+
+    def __init__(self, codebook, indices, mode, sidecar_pos, sidecar_val, N, K):
+        n_sidecar = 0 if sidecar_pos is None else int(len(sidecar_pos))
+        if n_sidecar == 0:
+            sidecar_pos = sidecar_val = None
+        self.mode, self.N, self.K = int(mode), int(N), int(K)
+        self.handle = hxq_linear_create(codebook, indices, mode, sidecar_pos, sidecar_val,
+                                        n_sidecar, N, K)
+
+    @classmethod
+    def from_layer(cls, layer: dict) -> "HelixLinear":
+        return cls(layer["codebook"], layer["indices"], layer["mode"], layer["sidecar_pos"],
+                   layer["sidecar_val"], layer["N"], layer["K"])
+
+    def forward(self, x, y=None, kernel=HXQ_KERNEL_AUTO, split_k=0, stream=None):
+        import torch
+        M = int(x.shape[0])
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.float32, device=x.device)
+        hxq_linear_forward_ex(self.handle, x, y, M, kernel, split_k, stream)
+        return y
+
+    __call__ = forward
+
+    def forward_host(self, x_host, y_host, x_dev, y_dev, stream=None):
+        """End-to-end call on host buffers: copy x (pinned) in, run, copy y out.
+        The caller owns the four buffers; the copies and the kernel share the
+        stream, which is synchronised before returning."""
+        import torch
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            x_dev.copy_(x_host, non_blocking=True)
+            hxq_linear_forward_ex(self.handle, x_dev, y_dev, int(x_dev.shape[0]), HXQ_KERNEL_AUTO, 0, s)
+            y_host.copy_(y_dev, non_blocking=True)
+        s.synchronize()
+        return y_host
+
+    def decode(self, stream=None):
+        import torch
+        W = torch.empty((self.N, self.K), dtype=torch.float32, device="cuda")
+        hxq_decode(self.handle, W, stream)
+        return W
+
+    def check(self) -> None:
+        hxq_linear_check(self.handle)
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            hxq_linear_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

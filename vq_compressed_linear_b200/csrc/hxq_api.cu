@@ -1,0 +1,279 @@
+// C ABI of libhxq: argument checks, the handle's device buffers, the tiled
+// index re-layout, the per-row sidecar patch lists and kernel dispatch.
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <numeric>
+#include <vector>
+
+#include "hxq_internal.cuh"
+
+using hxq::Layer;
+
+namespace {
+
+// One thread per 16-byte piece of the tiled layout (see hxq_internal.cuh).
+// Source bytes beyond the end of a row are index 0.
+__global__ void relayout_kernel(Layer L, const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
+                                int64_t n_pieces) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= n_pieces) return;
+  // pieces are enumerated row-fastest inside (tile, chunk, plane)
+  const int64_t per_row_pieces = (int64_t)L.KC * L.P;
+  const int64_t n = i / per_row_pieces;            // output row
+  const int64_t q = i % per_row_pieces;            // (chunk, plane) of this row
+  const int c = (int)(q / L.P), p = (int)(q % L.P);
+  const int t = (int)(n / hxq::kTileRows), r = (int)(n % hxq::kTileRows);
+  const int64_t row_bytes = (L.mode == HXQ_MODE_SCALAR8) ? L.K : 3LL * L.K / 4;
+  const int64_t first = (int64_t)c * 16 * L.P + (int64_t)p * 16;   // byte within the row stream
+  uint32_t w[4];
+  for (int j = 0; j < 4; ++j) {
+    uint32_t v = 0;
+    for (int b = 0; b < 4; ++b) {
+      const int64_t col = first + 4 * j + b;
+      const uint32_t byte = col < row_bytes ? src[n * row_bytes + col] : 0u;
+      v |= byte << (8 * b);
+    }
+    w[j] = v;
+  }
+  *reinterpret_cast<uint4*>(dst + hxq::piece_offset(L, t, c, p, r)) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return HXQ_OK;
+  if (e == cudaErrorMemoryAllocation) return HXQ_ENOMEM;
+  return HXQ_ECUDA;
+}
+
+void free_handle(hxq_linear* h) {
+  if (!h) return;
+  cudaFree(h->d_codebook);
+  cudaFree(h->d_idx);
+  cudaFree(h->d_row_ptr);
+  cudaFree(h->d_patch_k);
+  cudaFree(h->d_patch_v);
+  cudaFree(h->d_work);
+  cudaFree(h->d_counters);
+  cudaFree(h->d_status);
+  delete h;
+}
+
+template <class T>
+cudaError_t dalloc(T** p, size_t count) {
+  *p = nullptr;
+  if (count == 0) count = 1;
+  return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hxq_strerror(int code) {
+  switch (code) {
+    case HXQ_OK: return "ok";
+    case HXQ_EINVAL: return "invalid argument";
+    case HXQ_ENOMEM: return "device allocation failed";
+    case HXQ_ECUDA: return "CUDA runtime or driver error";
+    case HXQ_EUNSUPPORTED: return "device is not an sm_100 (B200-class) GPU";
+    case HXQ_ETIMEOUT: return "a device-side wait gave up (kernel aborted)";
+    default: return "unknown status";
+  }
+}
+
+int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, const int64_t* sidecar_pos,
+                      const float* sidecar_val, int64_t n_sidecar, int N, int K, hxq_linear_t* out) {
+  // ---- pure argument checks: no CUDA call before these pass
+  if (!out) return HXQ_EINVAL;
+  *out = nullptr;
+  if (!codebook || !indices) return HXQ_EINVAL;
+  if (mode != HXQ_MODE_SCALAR8 && mode != HXQ_MODE_VQ2D12) return HXQ_EINVAL;
+  if (N < 1 || K < 8 || (K % 8) != 0) return HXQ_EINVAL;
+  if (n_sidecar < 0 || n_sidecar > (int64_t)N * K) return HXQ_EINVAL;
+  if (n_sidecar > 0 && (!sidecar_pos || !sidecar_val)) return HXQ_EINVAL;
+  if (n_sidecar >= (int64_t)1 << 31) return HXQ_EINVAL;  // patch offsets are int32
+
+  // ---- device check
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_EUNSUPPORTED;
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return HXQ_ECUDA;
+  if (prop.major != 10 || prop.minor != 0) return HXQ_EUNSUPPORTED;
+
+  // ---- sidecar: copy to the host, check, sort into per-row patch lists
+  std::vector<int64_t> pos((size_t)n_sidecar);
+  std::vector<float> val((size_t)n_sidecar);
+  if (n_sidecar > 0) {
+    if (cudaMemcpy(pos.data(), sidecar_pos, n_sidecar * sizeof(int64_t), cudaMemcpyDefault) != cudaSuccess ||
+        cudaMemcpy(val.data(), sidecar_val, n_sidecar * sizeof(float), cudaMemcpyDefault) != cudaSuccess) {
+      cudaGetLastError();
+      return HXQ_ECUDA;
+    }
+  }
+  const int64_t NK = (int64_t)N * K;
+  std::vector<int> order((size_t)n_sidecar);
+  std::iota(order.begin(), order.end(), 0);
+  for (int64_t i = 0; i < n_sidecar; ++i)
+    if (pos[i] < 0 || pos[i] >= NK) return HXQ_EINVAL;
+  std::sort(order.begin(), order.end(), [&](int a, int b) { return pos[a] < pos[b]; });
+  for (int64_t i = 1; i < n_sidecar; ++i)
+    if (pos[order[i]] == pos[order[i - 1]]) return HXQ_EINVAL;
+  std::vector<int> row_ptr((size_t)N + 1, 0), patch_k((size_t)n_sidecar);
+  std::vector<float> patch_v((size_t)n_sidecar);
+  for (int64_t i = 0; i < n_sidecar; ++i) {
+    const int64_t p = pos[order[i]];
+    row_ptr[(size_t)(p / K) + 1]++;
+    patch_k[i] = (int)(p % K);
+    patch_v[i] = val[order[i]];
+  }
+  for (int n = 0; n < N; ++n) row_ptr[n + 1] += row_ptr[n];
+
+  // ---- handle and device buffers
+  hxq_linear* h = new hxq_linear();
+  std::memset(h, 0, sizeof(*h));
+  Layer& L = h->L;
+  L.mode = mode;
+  L.N = N;
+  L.K = K;
+  L.Kp = (K + hxq::kStageK - 1) / hxq::kStageK * hxq::kStageK;
+  L.P = mode == HXQ_MODE_SCALAR8 ? 1 : 3;
+  L.KC = mode == HXQ_MODE_SCALAR8 ? L.Kp / 16 : L.Kp / 64;
+  L.n_tiles = (N + hxq::kTileRows - 1) / hxq::kTileRows;
+  h->n_sidecar = n_sidecar;
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+
+  const size_t cb_floats = mode == HXQ_MODE_SCALAR8 ? 256 : 8192;
+  const size_t idx_bytes = (size_t)N * L.KC * 16 * L.P;
+  const size_t src_bytes = mode == HXQ_MODE_SCALAR8 ? (size_t)NK : (size_t)(3 * NK / 4);
+  // split-K workspace: up to 16 partials of a 32-token GEMV, at least 32 MiB
+  h->work_floats = std::max<size_t>((size_t)16 * 32 * N, (size_t)8 << 20);
+  h->n_counters = L.n_tiles * 64;
+
+  cudaError_t e = cudaSuccess;
+  uint8_t* d_src = nullptr;
+  if ((e = dalloc(&h->d_codebook, cb_floats)) != cudaSuccess ||
+      (e = dalloc(&h->d_idx, idx_bytes)) != cudaSuccess ||
+      (e = dalloc(&h->d_row_ptr, (size_t)N + 1)) != cudaSuccess ||
+      (e = dalloc(&h->d_patch_k, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&h->d_patch_v, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&h->d_work, h->work_floats)) != cudaSuccess ||
+      (e = dalloc(&h->d_counters, (size_t)h->n_counters)) != cudaSuccess ||
+      (e = dalloc(&h->d_status, 1)) != cudaSuccess ||
+      (e = dalloc(&d_src, src_bytes)) != cudaSuccess) {
+    cudaFree(d_src);
+    free_handle(h);
+    cudaGetLastError();
+    return cuda_status(e);
+  }
+  L.codebook = h->d_codebook;
+  L.idx = h->d_idx;
+  L.row_ptr = h->d_row_ptr;
+  L.patch_k = h->d_patch_k;
+  L.patch_v = h->d_patch_v;
+
+  if ((e = cudaMemcpy(h->d_codebook, codebook, cb_floats * sizeof(float), cudaMemcpyDefault)) != cudaSuccess ||
+      (e = cudaMemcpy(d_src, indices, src_bytes, cudaMemcpyDefault)) != cudaSuccess ||
+      (e = cudaMemcpy(h->d_row_ptr, row_ptr.data(), row_ptr.size() * sizeof(int), cudaMemcpyHostToDevice)) !=
+          cudaSuccess ||
+      (n_sidecar > 0 &&
+       ((e = cudaMemcpy(h->d_patch_k, patch_k.data(), n_sidecar * sizeof(int), cudaMemcpyHostToDevice)) !=
+            cudaSuccess ||
+        (e = cudaMemcpy(h->d_patch_v, patch_v.data(), n_sidecar * sizeof(float), cudaMemcpyHostToDevice)) !=
+            cudaSuccess)) ||
+      (e = cudaMemset(h->d_counters, 0, h->n_counters * sizeof(int))) != cudaSuccess ||
+      (e = cudaMemset(h->d_status, 0, sizeof(int))) != cudaSuccess) {
+    cudaFree(d_src);
+    free_handle(h);
+    cudaGetLastError();
+    return cuda_status(e);
+  }
+  const int64_t n_pieces = (int64_t)N * L.KC * L.P;
+  relayout_kernel<<<(unsigned)((n_pieces + 255) / 256), 256>>>(L, d_src, h->d_idx, n_pieces);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  cudaFree(d_src);
+  if (e != cudaSuccess) {
+    free_handle(h);
+    cudaGetLastError();
+    return cuda_status(e);
+  }
+  *out = h;
+  return HXQ_OK;
+}
+
+int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M, int kernel, int split_k,
+                          void* stream) {
+  if (!h || !x_bf16 || !y || M < 1) return HXQ_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) != 0) return HXQ_EINVAL;
+  if (kernel < HXQ_KERNEL_AUTO || kernel > HXQ_KERNEL_TC) return HXQ_EINVAL;
+  if (split_k < 0 || split_k > hxq::kMaxSplitK) return HXQ_EINVAL;
+  if (kernel == HXQ_KERNEL_AUTO) kernel = M <= 4 ? HXQ_KERNEL_GEMV : HXQ_KERNEL_TC;
+  if (kernel == HXQ_KERNEL_GEMV && M > 32) return HXQ_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  cudaError_t e;
+  if (kernel == HXQ_KERNEL_GEMV) {
+    const int split = split_k ? split_k : hxq::choose_split_gemv(*h, M);
+    e = hxq::launch_gemv(*h, x, y, M, split, s);
+  } else {
+    const int split = split_k ? split_k : hxq::choose_split_tc(*h, M);
+    e = hxq::launch_tc(*h, x, y, M, split, s);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e == cudaErrorInvalidValue ? HXQ_EINVAL : HXQ_ECUDA;
+  }
+  return HXQ_OK;
+}
+
+int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M, void* stream) {
+  return hxq_linear_forward_ex(h, x_bf16, y, M, HXQ_KERNEL_AUTO, 0, stream);
+}
+
+int hxq_decode(hxq_linear_t h, float* W_out, void* stream) {
+  if (!h || !W_out) return HXQ_EINVAL;
+  cudaError_t e = hxq::launch_decode(*h, W_out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_ECUDA;
+  }
+  return HXQ_OK;
+}
+
+int hxq_linear_info(hxq_linear_t h, int* mode, int* N, int* K, int64_t* n_sidecar) {
+  if (!h) return HXQ_EINVAL;
+  if (mode) *mode = h->L.mode;
+  if (N) *N = h->L.N;
+  if (K) *K = h->L.K;
+  if (n_sidecar) *n_sidecar = h->n_sidecar;
+  return HXQ_OK;
+}
+
+int hxq_linear_check(hxq_linear_t h) {
+  if (!h) return HXQ_EINVAL;
+  int status = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpy(&status, h->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_ECUDA;
+  }
+  if (status != 0) {
+    cudaMemset(h->d_status, 0, sizeof(int));
+    cudaDeviceSynchronize();
+    return HXQ_ETIMEOUT;
+  }
+  return HXQ_OK;
+}
+
+void hxq_linear_destroy(hxq_linear_t h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  free_handle(h);
+}
+
+}  // extern "C"

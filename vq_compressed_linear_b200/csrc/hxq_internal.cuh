@@ -1,0 +1,247 @@
+// Internal definitions shared by the libhxq translation units: the handle,
+// the tiled index layout, the per-row sidecar patch lists and thin inline-PTX
+// wrappers for mbarriers, TMA and tcgen05 (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hxq.h"
+
+namespace hxq {
+
+// ----------------------------------------------------------------------------
+// Index layout owned by a handle.
+//
+// Rows are grouped in tiles of kTileRows = 128 output features (one per TMEM
+// lane / one per thread of a 128-thread group). Within a row the weights are
+// cut into chunks: 16 weights = 16 bytes in scalar mode, 64 weights = 32
+// pairs = 48 bytes = 3 planes of 16 bytes in 2D mode. The tile stores, for
+// every chunk and plane, the 16-byte pieces of all its rows back to back, so
+// that 32 consecutive rows read 512 consecutive bytes:
+//
+//   piece(tile t, chunk c, plane p, row r) at byte
+//     t*128*KC*CB + (c*P + p)*R_t*16 + r*16
+//
+// with KC chunks per row, P planes per chunk, CB = 16*P bytes per chunk and
+// R_t = min(128, N - 128 t) rows in tile t. K is padded to a multiple of 64
+// (kStageK) with index 0; the kernels pair padded weights only with zero
+// activations, so a finite codebook entry 0 contributes nothing.
+// ----------------------------------------------------------------------------
+constexpr int kTileRows = 128;
+constexpr int kStageK = 64;           // weights per row per pipeline stage
+constexpr int kMaxSplitK = 64;
+
+struct Layer {
+  int mode;          // HXQ_MODE_*
+  int N, K;
+  int Kp;            // K rounded up to kStageK
+  int KC;            // chunks per row: Kp/16 (scalar) or Kp/64 (2D)
+  int P;             // planes per chunk: 1 (scalar) or 3 (2D)
+  int n_tiles;       // ceil(N / 128)
+  const float* codebook;     // 256 or 4096*2 floats
+  const uint8_t* idx;        // tiled layout above
+  const int* row_ptr;        // [N+1] offsets into the patch lists
+  const int* patch_k;        // per row, ascending k
+  const float* patch_v;      // replacement values
+};
+
+__host__ __device__ inline size_t piece_offset(const Layer& L, int t, int c, int p, int r) {
+  const int rows = min(kTileRows, L.N - t * kTileRows);
+  return (size_t)t * kTileRows * L.KC * (16 * L.P) + ((size_t)c * L.P + p) * rows * 16 + (size_t)r * 16;
+}
+
+}  // namespace hxq
+
+struct hxq_linear {
+  hxq::Layer L;
+  int64_t n_sidecar;
+  int device;
+  int num_sms;
+  float* d_codebook;
+  uint8_t* d_idx;
+  int* d_row_ptr;
+  int* d_patch_k;
+  float* d_patch_v;
+  float* d_work;        // split-K partial sums
+  size_t work_floats;
+  int* d_counters;      // per output tile: arrivals of split-K partials
+  int n_counters;
+  int* d_status;        // device-side error word (bounded waits that gave up)
+};
+
+namespace hxq {
+
+// Launchers (each returns a cudaError_t from the launch).
+cudaError_t launch_decode(const hxq_linear& h, float* W, cudaStream_t s);
+cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M, int split,
+                        cudaStream_t s);
+cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, float* y, int M, int split,
+                      cudaStream_t s);
+int choose_split_gemv(const hxq_linear& h, int M);
+int choose_split_tc(const hxq_linear& h, int M);
+
+// Device status bits.
+constexpr int kStatusWaitTimeout = 1;
+
+// ----------------------------------------------------------------------------
+// Inline PTX helpers (sm_100a).
+// ----------------------------------------------------------------------------
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete. Gives up after
+// kWaitLimitNs of wall time or as soon as another thread of the CTA has set
+// *abort; on giving up it sets *abort and returns false. A normal launch never
+// comes near the limit (kernels here run for microseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if ((i & 255) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// 2D tiled TMA load global -> shared, completion counted on `bar` in bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(tmap), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// ---- tcgen05 ---------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (bf16 inputs, fp32 accumulate).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on `bar` when all previously issued tcgen05.mma of this thread finish.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+                 "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// (a == b) ? x : y as one predicated select; written in PTX so that an
+// unrolled chain of these over a register array stays in registers instead
+// of being turned into a dynamically indexed local-memory store.
+__device__ __forceinline__ uint32_t sel_eq(int a, int b, uint32_t x, uint32_t y) {
+  uint32_t r;
+  asm("{\n\t.reg .pred p;\n\tsetp.eq.s32 p, %1, %2;\n\tselp.b32 %0, %3, %4, p;\n\t}"
+      : "=r"(r) : "r"(a), "r"(b), "r"(x), "r"(y));
+  return r;
+}
+__device__ __forceinline__ float sel_eq(int a, int b, float x, float y) {
+  return __uint_as_float(sel_eq(a, b, __float_as_uint(x), __float_as_uint(y)));
+}
+
+// Byte permute: result byte i = byte sel_i of the 8-byte value {b:a}.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+#endif  // __CUDACC__
+
+}  // namespace hxq
