@@ -1,0 +1,505 @@
+"""Benchmark of the HelixLinear forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hxq|reference]
+                    [--workload mamba2|qwen25_3b|vq2d|prefill|tiny] [--no-secondary]
+
+A step is one forward of every layer of the workload (default: the
+Mamba2-1.3B-shaped decode pair in_proj 8512x2048 + out_proj 2048x4096, scalar
+8-bit codebook, M = 1 token) on seeded synthetic inputs.
+
+value: achieved HBM throughput on algorithmic bytes, GB/s = (indices +
+8 B per sidecar entry + codebook + x + y) per step x K / device time of the
+K steps. Inputs are resident in HBM when timing starts; each step uses its
+own replica of the layers, with enough replicas that their total exceeds 4x
+the L2 cache, so every step reads its weights cold from HBM. The K steps are
+one CUDA-graph replay timed with CUDA events on the launching stream.
+
+e2e: the same metric through the public call with host buffers: each step
+copies x from pinned host memory, runs the forwards and copies y back.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on the host cores over a bounded sample of the same workload.
+
+Multi-GPU: every rank runs its own replica of the workload (the layer does
+not shard across GPUs in this build): value = all ranks' bytes / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def layer_bytes(layer, M):
+    N, K, mode = layer["N"], layer["K"], layer["mode"]
+    idx = N * K if mode == synthetic.MODE_SCALAR8 else 3 * N * K // 4
+    cb = 256 * 4 if mode == synthetic.MODE_SCALAR8 else 4096 * 8
+    return idx + 8 * layer["sidecar_pos"].size + cb + 2 * M * K + 4 * M * N
+
+
+def layer_flops(layer, M):
+    return 2.0 * M * layer["N"] * layer["K"]
+
+
+def workload(name, seed=0, M_override=None):
+    """[(label, layer, M)] for one named workload, at the M its bench line uses."""
+    out = []
+    for lname, layer, Ms in synthetic.config_layers(name, seed):
+        Ms_run = Ms if M_override is None else (M_override,)
+        for M in Ms_run:
+            out.append((f"{lname}/M={M}", layer, M))
+    return out
+
+
+DEFAULT_M = {"mamba2": None, "tiny": 1, "qwen25_3b": 1, "vq2d": 1, "prefill": 2048}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"hxq_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            self.proc.wait()
+            self.f.close()
+
+    def summary(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = sorted(r[0] for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("hxq_gemv.cu", "hxq_tc.cu", "hxq_internal.cuh"):
+        h.update(open(os.path.join(ROOT, "vq_compressed_linear_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key):
+    """dram bytes per launch recorded from an ncu capture in profiles/, if the
+    kernel sources are unchanged since (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(kernel_key)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_sha") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def dominant_kernel(layer, M):
+    if M <= 4:
+        return "gemv_scalar" if layer["mode"] == synthetic.MODE_SCALAR8 else "gemv_vq2d"
+    return ("tc_skinny_" if M <= 32 else "tc_prefill_") + \
+        ("scalar" if layer["mode"] == synthetic.MODE_SCALAR8 else "vq2d")
+
+
+def time_workload(hxq, torch, items, steps, warmup, l2_bytes, stream, soak_s=0.0, max_replica_bytes=48 << 30):
+    """Device time of `steps` steps (CUDA graph, rotating replicas).
+    Returns (ms total, bytes per step, flops per step, launches per step, replicas)."""
+    step_bytes = sum(layer_bytes(l, M) for _, l, M in items)
+    step_flops = sum(layer_flops(l, M) for _, l, M in items)
+    dev_bytes_step = sum(l["indices"].size + 8 * l["sidecar_pos"].size for _, l, _ in items)
+    R = max(1, math.ceil(4 * l2_bytes / max(1, dev_bytes_step)))
+    R = min(R, max(1, max_replica_bytes // max(1, dev_bytes_step)), steps + warmup)
+    reps = []
+    for _ in range(R):
+        reps.append([hxq.HelixLinear.from_layer(l) for _, l, _ in items])
+    xs = [torch.from_numpy(synthetic.activations(M, l["K"], 1).view(np.int16)).cuda() for _, l, M in items]
+    ys = [torch.empty((M, l["N"]), dtype=torch.float32, device="cuda") for _, l, M in items]
+
+    def step(i):
+        for j, lin in enumerate(reps[i % R]):
+            lin.forward(xs[j], ys[j], stream=stream)
+
+    with torch.cuda.stream(stream):
+        step(0)  # first launches set kernel attributes outside capture
+    torch.cuda.synchronize()
+    g_warm, g_run = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm, stream=stream):
+        for i in range(warmup):
+            step(i)
+    with torch.cuda.graph(g_run, stream=stream):
+        for i in range(steps):
+            step(warmup + i)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        g_warm.replay()
+        t_end = time.time() + soak_s
+        while time.time() < t_end:
+            g_run.replay()
+            stream.synchronize()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):          # replay() launches on the current stream
+        e0.record(stream)
+        g_run.replay()
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    for lin in reps[0]:
+        lin.check()
+    del g_warm, g_run
+    for rep in reps:
+        for lin in rep:
+            lin.close()
+    return ms, step_bytes, step_flops, len(items), R
+
+
+def e2e_workload(hxq, torch, items, steps, warmup, stream):
+    """Same metric through HelixLinear.forward_host semantics: pinned host x
+    in, y out, every step. Returns (ms, h2d bytes/step, d2h bytes/step)."""
+    lins = [hxq.HelixLinear.from_layer(l) for _, l, _ in items]
+    xh = [torch.from_numpy(synthetic.activations(M, l["K"], 2).view(np.int16)).pin_memory() for _, l, M in items]
+    yh = [torch.empty((M, l["N"]), dtype=torch.float32).pin_memory() for _, l, M in items]
+    xd = [torch.empty_like(x, device="cuda") for x in xh]
+    yd = [torch.empty_like(y, device="cuda") for y in yh]
+
+    def step():
+        for j, lin in enumerate(lins):
+            xd[j].copy_(xh[j], non_blocking=True)
+            lin.forward(xd[j], yd[j], stream=stream)
+            yh[j].copy_(yd[j], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    for lin in lins:
+        lin.close()
+    h2d = sum(x.numel() * 2 for x in xh)
+    d2h = sum(y.numel() * 4 for y in yh)
+    return ms, h2d, d2h
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+_X_CACHE = {}
+
+
+def _x_for(layer, M):
+    key = (M, layer["K"])
+    if key not in _X_CACHE:
+        _X_CACHE[key] = synthetic.activations(M, layer["K"], 1)
+    return _X_CACHE[key]
+
+
+def _oracle_pass(items, frac, offset=0):
+    """One pass of the fp64 oracle over the workload, on `frac` of each
+    layer's output rows (a contiguous, rotating slice). Returns (bytes, flops)
+    credited, scaled by the fraction of rows done."""
+    import oracle
+    b = f = 0.0
+    for _, layer, M in items:
+        x = _x_for(layer, M)
+        N = layer["N"]
+        nr = max(1, int(round(frac * N)))
+        if nr >= N:
+            oracle.forward_layer(layer, x)
+            nr = N
+        else:
+            rows = (offset * nr + np.arange(nr)) % N
+            oracle.forward_rows(layer, x, rows)
+        b += layer_bytes(layer, M) * nr / N
+        f += layer_flops(layer, M) * nr / N
+    return b, f
+
+
+def oracle_sample(items, budget_s=12.0):
+    """cpu_baseline: repeat oracle passes over the workload until about
+    budget_s of CPU time is spent (a row slice per pass when a whole pass would
+    take longer). Returns (GB/s, TFLOP/s, description, threads, seconds)."""
+    for _, layer, M in items:
+        _x_for(layer, M)
+    t0 = time.perf_counter()
+    b, f = _oracle_pass(items, 1.0 if _est_pass_s(items) < budget_s / 4 else 0.05)
+    first = time.perf_counter() - t0
+    frac = 1.0 if first < budget_s / 4 and _est_pass_s(items) < budget_s / 4 else 0.05
+    passes, tb, tf, tt = 1, b, f, first
+    while tt < budget_s:
+        t1 = time.perf_counter()
+        b, f = _oracle_pass(items, frac, passes)
+        tt += time.perf_counter() - t1
+        tb += b
+        tf += f
+        passes += 1
+    desc = f"{passes} oracle passes over " + ", ".join(lbl for lbl, _, _ in items) + \
+        ("" if frac == 1.0 else f" ({frac:.0%} of output rows per pass after the first)")
+    return tb / tt / 1e9, tf / tt / 1e12, desc, _oracle_threads(), tt
+
+
+def _est_pass_s(items):
+    # fp64 oracle: decode ~ 20 ns per weight, product ~ 1 ns per multiply-add
+    return sum(20e-9 * l["N"] * l["K"] + 1e-9 * M * l["N"] * l["K"] for _, l, M in items)
+
+
+def oracle_reference_arm(items, steps, warmup, budget_s=60.0):
+    """--impl reference: W warm-up passes, then K timed passes, each on a row
+    slice sized so that the K passes take about budget_s in total."""
+    frac = min(1.0, budget_s / max(1, steps) / max(1e-6, _est_pass_s(items)))
+    for _, layer, M in items:
+        _x_for(layer, M)
+    for i in range(warmup):
+        _oracle_pass(items, frac, i)
+    t0 = time.perf_counter()
+    tb = tf = 0.0
+    for i in range(steps):
+        b, f = _oracle_pass(items, frac, warmup + i)
+        tb += b
+        tf += f
+    tt = time.perf_counter() - t0
+    desc = f"{steps} oracle passes over " + ", ".join(lbl for lbl, _, _ in items) + \
+        f", {min(frac, 1.0):.2%} of output rows per pass"
+    return tb / tt / 1e9, tf / tt / 1e12, desc, _oracle_threads(), tt
+
+
+def profile_run(hxq, torch, items, steps, warmup):
+    """Small, eager run for ncu: replicas just past 1.25x L2, W + K steps."""
+    props = torch.cuda.get_device_properties(0)
+    l2 = getattr(props, "L2_cache_size", 126 << 20)
+    dev_bytes = sum(l["indices"].size for _, l, _ in items)
+    R = max(1, math.ceil(1.25 * l2 / dev_bytes))
+    reps = [[hxq.HelixLinear.from_layer(l) for _, l, _ in items] for _ in range(R)]
+    xs = [torch.from_numpy(synthetic.activations(M, l["K"], 1).view(np.int16)).cuda() for _, l, M in items]
+    ys = [torch.empty((M, l["N"]), dtype=torch.float32, device="cuda") for _, l, M in items]
+    for i in range(warmup + steps):
+        for j, lin in enumerate(reps[i % R]):
+            lin.forward(xs[j], ys[j])
+    torch.cuda.synchronize()
+    for rep in reps:
+        for lin in rep:
+            lin.check()
+            lin.close()
+    return 0
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hxq", choices=["hxq", "reference"])
+    ap.add_argument("--workload", default="mamba2", choices=list(synthetic.CONFIGS))
+    ap.add_argument("--M", type=int, default=None, help="token count (default: the workload's bench M)")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu", action="store_true",
+                    help="minimal run for profilers: enough layer replicas to exceed L2, then "
+                         "W + K eager steps; prints nothing")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    items = workload(args.workload, 0, args.M if args.M else DEFAULT_M[args.workload])
+    is_prefill = all(M > 32 for _, _, M in items)
+    metric = ("HelixLinear prefill GEMM TFLOP/s" if is_prefill else "HelixLinear GEMV achieved HBM GB/s")
+    unit = "TFLOP/s" if is_prefill else "GB/s"
+    wl_name = {"mamba2": "mamba2_1.3b_decode_scalar8_M1 (in_proj 8512x2048 + out_proj 2048x4096)"}.get(
+        args.workload, args.workload + ":" + ",".join(lbl for lbl, _, _ in items))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        gbs, tfs, sample, threads, secs = oracle_reference_arm(items, args.steps, args.warmup)
+        v = tfs if is_prefill else gbs
+        line = {"impl": "reference", "metric": metric, "value": v, "unit": unit, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl_name},
+                "cpu_baseline": {"value": v, "unit": unit, "cores": threads, "kind": "oracle",
+                                 "sample": sample + f" ({secs:.1f} s)"},
+                "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    import vq_compressed_linear_b200 as hxq
+
+    if args.ncu:
+        return profile_run(hxq, torch, items, args.steps, args.warmup)
+
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    props = torch.cuda.get_device_properties(local_rank)
+    l2 = getattr(props, "L2_cache_size", 126 << 20)
+    stream = torch.cuda.Stream()
+    pk, pk_kind = peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        ms, step_bytes, step_flops, launches, R = time_workload(
+            hxq, torch, items, args.steps, args.warmup, l2, stream, soak_s=1.5)
+        barrier()
+    clocks = clk.summary()
+    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    total_bytes = step_bytes * args.steps * world
+    total_flops = step_flops * args.steps * world
+    gbs = total_bytes / (ms_max * 1e-3) / 1e9
+    tfs = total_flops / (ms_max * 1e-3) / 1e12
+    value = tfs if is_prefill else gbs
+
+    # e2e through the public call, host buffers
+    e_ms, h2d, d2h = e2e_workload(hxq, torch, items, args.steps, args.warmup, stream)
+    te = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e_ms = float(te.item())
+    e_val = (total_flops / (e_ms * 1e-3) / 1e12) if is_prefill else (total_bytes / (e_ms * 1e-3) / 1e9)
+
+    # roofline of the dominant kernel (all launches of this workload are one kernel)
+    _, l0, M0 = items[0]
+    kkey = dominant_kernel(l0, M0)
+    per_launch_ms = ms / (args.steps * launches)
+    if is_prefill:
+        peak = float(pk["bf16_tflops"])
+        achieved = step_flops / launches / (per_launch_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(kkey), "kernel": kkey,
+                "peak_kind": f"{pk_kind} bf16 burst"}
+    else:
+        peak = float(pk["hbm_gbs"])
+        achieved = step_bytes / launches / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(kkey), "kernel": kkey,
+                "peak_kind": f"{pk_kind} copy"}
+
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if is_prefill else "f32", "data": "synthetic",
+            "config": {"workload": wl_name, "tokens_M": sorted({M for _, _, M in items}),
+                       "bytes_per_step": step_bytes, "flops_per_step": step_flops,
+                       "l2": f"{R} rotating layer replicas per rank ({R * sum(l['indices'].size for _, l, _ in items) / 2**20:.0f} MiB of indices) > 4x L2",
+                       "timing": "one CUDA-graph replay of K steps, CUDA events on the launch stream",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof,
+            "e2e": {"value": e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * launches,
+            "clocks": clocks}
+
+    if not args.no_secondary and world == 1:
+        sec = []
+        for wl in ("qwen25_3b", "vq2d", "prefill"):
+            for M in synthetic.CONFIGS[wl][0][4]:
+                its = workload(wl, 0, M)
+                s_ms, sb, sf, sl, sR = time_workload(hxq, torch, its, 20, 3, l2, stream)
+                pre = M > 32
+                v = (sf * 20 / (s_ms * 1e-3) / 1e12) if pre else (sb * 20 / (s_ms * 1e-3) / 1e9)
+                pkv = float(pk["bf16_tflops"]) if pre else float(pk["hbm_gbs"])
+                # roofline time: slower of bytes at HBM peak and flops at tensor peak
+                t_roof = max(sb / (float(pk["hbm_gbs"]) * 1e9), sf / (float(pk["bf16_tflops"]) * 1e12))
+                sec.append({"workload": f"{wl} M={M}", "value": round(v, 1), "unit": "TFLOP/s" if pre else "GB/s",
+                            "frac_of_peak": round(v / pkv, 3),
+                            "frac_of_roofline": round(t_roof / (s_ms * 1e-3 / 20), 3),
+                            "us_per_step": round(s_ms * 1e3 / 20, 2), "launches_per_step": sl})
+        line["secondary"] = sec
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs_c, tfs_c, sample, threads, secs = oracle_sample(items)
+        line["cpu_baseline"] = {"value": tfs_c if is_prefill else gbs_c, "unit": unit, "cores": threads,
+                                "kind": "oracle", "sample": sample + f" ({secs:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

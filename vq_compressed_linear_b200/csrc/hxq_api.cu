@@ -40,6 +40,29 @@ __global__ void relayout_kernel(Layer L, const uint8_t* __restrict__ src, uint8_
   *reinterpret_cast<uint4*>(dst + hxq::piece_offset(L, t, c, p, r)) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// delta[i] = v_i - (the codebook value the sidecar entry replaces), fp32.
+// `pos` holds the flat positions in bucket order.
+__global__ void sidecar_delta_kernel(Layer L, const int64_t* __restrict__ pos, int64_t n,
+                                     float* __restrict__ delta) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int64_t p = pos[i];
+  const int row = (int)(p / L.K), k = (int)(p % L.K);
+  const int t = row / hxq::kTileRows, r = row % hxq::kTileRows;
+  float c;
+  if (L.mode == HXQ_MODE_SCALAR8) {
+    c = L.codebook[L.idx[hxq::piece_offset(L, t, k / 16, 0, r) + k % 16]];
+  } else {
+    const int st = k / hxq::kStageK, bit = 12 * ((k % hxq::kStageK) / 2);
+    const int b0 = bit / 8, b1 = b0 + 1;
+    const uint32_t lo = L.idx[hxq::piece_offset(L, t, st, b0 / 16, r) + b0 % 16];
+    const uint32_t hi = L.idx[hxq::piece_offset(L, t, st, b1 / 16, r) + b1 % 16];
+    const uint32_t e = ((lo | (hi << 8)) >> (bit & 7)) & 0xFFF;
+    c = L.codebook[2 * e + (k & 1)];
+  }
+  delta[i] = L.pval[i] - c;
+}
+
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return HXQ_OK;
   if (e == cudaErrorMemoryAllocation) return HXQ_ENOMEM;
@@ -50,9 +73,10 @@ void free_handle(hxq_linear* h) {
   if (!h) return;
   cudaFree(h->d_codebook);
   cudaFree(h->d_idx);
-  cudaFree(h->d_row_ptr);
-  cudaFree(h->d_patch_k);
-  cudaFree(h->d_patch_v);
+  cudaFree(h->d_bptr);
+  cudaFree(h->d_pkey);
+  cudaFree(h->d_pval);
+  cudaFree(h->d_pdelta);
   cudaFree(h->d_work);
   cudaFree(h->d_counters);
   cudaFree(h->d_status);
@@ -104,7 +128,7 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return HXQ_ECUDA;
   if (prop.major != 10 || prop.minor != 0) return HXQ_EUNSUPPORTED;
 
-  // ---- sidecar: copy to the host, check, sort into per-row patch lists
+  // ---- sidecar: copy to the host, check it, bucket it by (tile, stage, quadrant)
   std::vector<int64_t> pos((size_t)n_sidecar);
   std::vector<float> val((size_t)n_sidecar);
   if (n_sidecar > 0) {
@@ -115,22 +139,13 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
     }
   }
   const int64_t NK = (int64_t)N * K;
-  std::vector<int> order((size_t)n_sidecar);
-  std::iota(order.begin(), order.end(), 0);
   for (int64_t i = 0; i < n_sidecar; ++i)
     if (pos[i] < 0 || pos[i] >= NK) return HXQ_EINVAL;
+  std::vector<int> order((size_t)n_sidecar);
+  std::iota(order.begin(), order.end(), 0);
   std::sort(order.begin(), order.end(), [&](int a, int b) { return pos[a] < pos[b]; });
   for (int64_t i = 1; i < n_sidecar; ++i)
     if (pos[order[i]] == pos[order[i - 1]]) return HXQ_EINVAL;
-  std::vector<int> row_ptr((size_t)N + 1, 0), patch_k((size_t)n_sidecar);
-  std::vector<float> patch_v((size_t)n_sidecar);
-  for (int64_t i = 0; i < n_sidecar; ++i) {
-    const int64_t p = pos[order[i]];
-    row_ptr[(size_t)(p / K) + 1]++;
-    patch_k[i] = (int)(p % K);
-    patch_v[i] = val[order[i]];
-  }
-  for (int n = 0; n < N; ++n) row_ptr[n + 1] += row_ptr[n];
 
   // ---- handle and device buffers
   hxq_linear* h = new hxq_linear();
@@ -147,47 +162,80 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
 
+  const int nst = hxq::n_stages(L);
+  const int64_t n_buckets = (int64_t)L.n_tiles * nst * hxq::kQuads;
+  std::vector<int> bptr((size_t)n_buckets + 1, 0);
+  std::vector<int> bucket((size_t)n_sidecar);
+  for (int64_t i = 0; i < n_sidecar; ++i) {
+    const int64_t p = pos[order[i]];
+    const int row = (int)(p / K), k = (int)(p % K);
+    bucket[i] = hxq::bucket_of(L, row / hxq::kTileRows, k / hxq::kStageK, (row % hxq::kTileRows) / 32);
+    bptr[(size_t)bucket[i] + 1]++;
+  }
+  for (int64_t b = 0; b < n_buckets; ++b) bptr[b + 1] += bptr[b];
+  std::vector<int> fill(bptr.begin(), bptr.end() - 1);
+  std::vector<uint32_t> pkey((size_t)n_sidecar);
+  std::vector<float> pval((size_t)n_sidecar);
+  std::vector<int64_t> bpos((size_t)n_sidecar);
+  for (int64_t i = 0; i < n_sidecar; ++i) {   // stable: position order inside a bucket
+    const int64_t p = pos[order[i]];
+    const int row = (int)(p / K), k = (int)(p % K);
+    const int j = fill[bucket[i]]++;
+    pkey[j] = hxq::patch_key(row % 32, k % hxq::kStageK);
+    pval[j] = val[order[i]];
+    bpos[j] = p;
+  }
+
   const size_t cb_floats = mode == HXQ_MODE_SCALAR8 ? 256 : 8192;
   const size_t idx_bytes = (size_t)N * L.KC * 16 * L.P;
   const size_t src_bytes = mode == HXQ_MODE_SCALAR8 ? (size_t)NK : (size_t)(3 * NK / 4);
-  // split-K workspace: up to 16 partials of a 32-token GEMV, at least 32 MiB
-  h->work_floats = std::max<size_t>((size_t)16 * 32 * N, (size_t)8 << 20);
-  h->n_counters = L.n_tiles * 64;
+  // stream-K workspace: two partial tiles per CTA (GEMV: per 128-thread
+  // virtual CTA, up to 32 tokens; tensor-core kernel: per CTA, up to 256 tokens)
+  h->work_floats = std::max<size_t>((size_t)h->num_sms * 4 * 2 * 32 * hxq::kTileRows,
+                                    hxq::tc_workspace_floats(h->num_sms));
+  h->n_counters = L.n_tiles * 64 * hxq::kQuads;  // (token block, tile, quadrant)
 
   cudaError_t e = cudaSuccess;
   uint8_t* d_src = nullptr;
+  int64_t* d_bpos = nullptr;
   if ((e = dalloc(&h->d_codebook, cb_floats)) != cudaSuccess ||
       (e = dalloc(&h->d_idx, idx_bytes)) != cudaSuccess ||
-      (e = dalloc(&h->d_row_ptr, (size_t)N + 1)) != cudaSuccess ||
-      (e = dalloc(&h->d_patch_k, (size_t)n_sidecar)) != cudaSuccess ||
-      (e = dalloc(&h->d_patch_v, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&h->d_bptr, (size_t)n_buckets + 1)) != cudaSuccess ||
+      (e = dalloc(&h->d_pkey, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&h->d_pval, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&h->d_pdelta, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&d_bpos, (size_t)n_sidecar)) != cudaSuccess ||
       (e = dalloc(&h->d_work, h->work_floats)) != cudaSuccess ||
       (e = dalloc(&h->d_counters, (size_t)h->n_counters)) != cudaSuccess ||
       (e = dalloc(&h->d_status, 1)) != cudaSuccess ||
       (e = dalloc(&d_src, src_bytes)) != cudaSuccess) {
     cudaFree(d_src);
+    cudaFree(d_bpos);
     free_handle(h);
     cudaGetLastError();
     return cuda_status(e);
   }
   L.codebook = h->d_codebook;
   L.idx = h->d_idx;
-  L.row_ptr = h->d_row_ptr;
-  L.patch_k = h->d_patch_k;
-  L.patch_v = h->d_patch_v;
+  L.bptr = h->d_bptr;
+  L.pkey = h->d_pkey;
+  L.pval = h->d_pval;
+  L.pdelta = h->d_pdelta;
 
   if ((e = cudaMemcpy(h->d_codebook, codebook, cb_floats * sizeof(float), cudaMemcpyDefault)) != cudaSuccess ||
       (e = cudaMemcpy(d_src, indices, src_bytes, cudaMemcpyDefault)) != cudaSuccess ||
-      (e = cudaMemcpy(h->d_row_ptr, row_ptr.data(), row_ptr.size() * sizeof(int), cudaMemcpyHostToDevice)) !=
-          cudaSuccess ||
+      (e = cudaMemcpy(h->d_bptr, bptr.data(), bptr.size() * sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess ||
       (n_sidecar > 0 &&
-       ((e = cudaMemcpy(h->d_patch_k, patch_k.data(), n_sidecar * sizeof(int), cudaMemcpyHostToDevice)) !=
+       ((e = cudaMemcpy(h->d_pkey, pkey.data(), n_sidecar * sizeof(uint32_t), cudaMemcpyHostToDevice)) !=
             cudaSuccess ||
-        (e = cudaMemcpy(h->d_patch_v, patch_v.data(), n_sidecar * sizeof(float), cudaMemcpyHostToDevice)) !=
+        (e = cudaMemcpy(h->d_pval, pval.data(), n_sidecar * sizeof(float), cudaMemcpyHostToDevice)) !=
+            cudaSuccess ||
+        (e = cudaMemcpy(d_bpos, bpos.data(), n_sidecar * sizeof(int64_t), cudaMemcpyHostToDevice)) !=
             cudaSuccess)) ||
       (e = cudaMemset(h->d_counters, 0, h->n_counters * sizeof(int))) != cudaSuccess ||
       (e = cudaMemset(h->d_status, 0, sizeof(int))) != cudaSuccess) {
     cudaFree(d_src);
+    cudaFree(d_bpos);
     free_handle(h);
     cudaGetLastError();
     return cuda_status(e);
@@ -195,8 +243,13 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   const int64_t n_pieces = (int64_t)N * L.KC * L.P;
   relayout_kernel<<<(unsigned)((n_pieces + 255) / 256), 256>>>(L, d_src, h->d_idx, n_pieces);
   e = cudaGetLastError();
+  if (e == cudaSuccess && n_sidecar > 0) {
+    sidecar_delta_kernel<<<(unsigned)((n_sidecar + 255) / 256), 256>>>(L, d_bpos, n_sidecar, h->d_pdelta);
+    e = cudaGetLastError();
+  }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   cudaFree(d_src);
+  cudaFree(d_bpos);
   if (e != cudaSuccess) {
     free_handle(h);
     cudaGetLastError();
@@ -212,17 +265,15 @@ int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M, i
   if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) != 0) return HXQ_EINVAL;
   if (kernel < HXQ_KERNEL_AUTO || kernel > HXQ_KERNEL_TC) return HXQ_EINVAL;
   if (split_k < 0 || split_k > hxq::kMaxSplitK) return HXQ_EINVAL;
-  if (kernel == HXQ_KERNEL_AUTO) kernel = M <= 4 ? HXQ_KERNEL_GEMV : HXQ_KERNEL_TC;
-  if (kernel == HXQ_KERNEL_GEMV && M > 32) return HXQ_EINVAL;
+  if (kernel == HXQ_KERNEL_AUTO) kernel = (M <= 4 && hxq::gemv_supports(*h, M)) ? HXQ_KERNEL_GEMV : HXQ_KERNEL_TC;
+  if (kernel == HXQ_KERNEL_GEMV && !hxq::gemv_supports(*h, M)) return HXQ_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   cudaError_t e;
   if (kernel == HXQ_KERNEL_GEMV) {
-    const int split = split_k ? split_k : hxq::choose_split_gemv(*h, M);
-    e = hxq::launch_gemv(*h, x, y, M, split, s);
+    e = hxq::launch_gemv(*h, x, y, M, split_k, s);
   } else {
-    const int split = split_k ? split_k : hxq::choose_split_tc(*h, M);
-    e = hxq::launch_tc(*h, x, y, M, split, s);
+    e = hxq::launch_tc(*h, x, y, M, split_k, s);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();

@@ -14,16 +14,6 @@
 namespace hxq {
 namespace {
 
-// First patch of row n with column >= k0 (patch lists are sorted by column).
-__device__ __forceinline__ int first_patch(const Layer& L, int n, int k0) {
-  int lo = L.row_ptr[n], hi = L.row_ptr[n + 1];
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (L.patch_k[mid] < k0) lo = mid + 1; else hi = mid;
-  }
-  return lo;
-}
-
 // One thread per (row, chunk); consecutive threads walk along a row so the
 // fp32 stores are contiguous.
 __global__ void __launch_bounds__(256) decode_scalar_kernel(Layer L, float* __restrict__ W) {
@@ -37,10 +27,16 @@ __global__ void __launch_bounds__(256) decode_scalar_kernel(Layer L, float* __re
 #pragma unroll
   for (int j = 0; j < 16; ++j) v[j] = __ldg(L.codebook + ((w[j >> 2] >> (8 * (j & 3))) & 0xFF));
   const int k0 = c * 16;
-  for (int p = first_patch(L, n, k0); p < L.row_ptr[n + 1] && L.patch_k[p] < k0 + 16; ++p) {
-    const int j = L.patch_k[p] - k0;
+  {  // sidecar entries of this row in this chunk, from the (tile, stage, quadrant) bucket
+    const int b = bucket_of(L, t, k0 / kStageK, r / 32);
+    for (int p = L.bptr[b]; p < L.bptr[b + 1]; ++p) {
+      const uint32_t key = L.pkey[p];
+      const int j = (int)(key >> 5) - (k0 % kStageK);
+      if ((int)(key & 31) == (r & 31) && j >= 0 && j < 16) {
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) v[jj] = sel_eq(jj, j, L.patch_v[p], v[jj]);
+        for (int jj = 0; jj < 16; ++jj) v[jj] = sel_eq(jj, j, L.pval[p], v[jj]);
+      }
+    }
   }
   float* out = W + (int64_t)n * L.K + k0;
   const int cnt = min(16, L.K - k0);
@@ -70,16 +66,18 @@ __global__ void __launch_bounds__(256) decode_vq2d_kernel(Layer L, float* __rest
   const int k0 = c * 64;
   float* out = W + (int64_t)n * L.K + k0;
   const int cnt = min(64, L.K - k0);
-  int p = first_patch(L, n, k0);
-  const int pend = L.row_ptr[n + 1];
+  const int b = bucket_of(L, t, c, r / 32);
+  const int pb = L.bptr[b], pe = L.bptr[b + 1];
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const int bit = 12 * j;
     const uint32_t e = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & 0xFFF;
     float2 v = __ldg(cb2 + e);
-    while (p < pend && L.patch_k[p] < k0 + 2 * j + 2) {
-      if (L.patch_k[p] == k0 + 2 * j) v.x = L.patch_v[p]; else v.y = L.patch_v[p];
-      ++p;
+    for (int p = pb; p < pe; ++p) {
+      const uint32_t key = L.pkey[p];
+      if ((int)(key & 31) != (r & 31)) continue;
+      if ((int)(key >> 5) == 2 * j) v.x = L.pval[p];
+      if ((int)(key >> 5) == 2 * j + 1) v.y = L.pval[p];
     }
     if (2 * j + 1 < cnt) {
       *reinterpret_cast<float2*>(out + 2 * j) = v;

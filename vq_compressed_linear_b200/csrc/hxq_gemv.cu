@@ -1,33 +1,41 @@
-// Fused decode + GEMV on CUDA cores for few tokens (M <= 32, used by default
-// for M <= 4): y[m][n] = sum_k x[m][k] * W[n][k] with W decoded on the fly
-// from the codebook and never written anywhere (the pages' buffered path
+// Fused decode + GEMV on CUDA cores for few tokens (M <= 4 by default; up to
+// M = 32 on request): y[m][n] = sum_k x[m][k] * W[n][k] with W decoded on the
+// fly from the codebook and never written anywhere (the pages' buffered path
 // instead materialises W and calls cuBLAS: HXQ whitepaper, method section,
 // buffered forward path paragraph).
 //
-// Work decomposition. A unit is one 128-row tile times one contiguous range
-// of 64-weight stages along K (split-K). Each CTA is persistent: it builds
-// its shared-memory codebook once, then takes units blockIdx.x,
-// blockIdx.x + gridDim.x, ... Inside a unit the CTA's G = 4 groups of 128
-// threads take the stages round-robin; thread r of a group owns row r of
-// the tile and reads its 16-byte index pieces, so a warp reads 512
-// contiguous bytes per load.
+// Work decomposition (stream-K). The work items are the tile-stages of the
+// layer, (tile of 128 rows) x (64 weights along K), numbered tile-major. A
+// persistent grid of one 512-thread CTA per SM takes contiguous item ranges
+// of equal size, so every CTA streams the same number of index bytes
+// whatever the layer shape. Inside a CTA the 4 groups of 128 threads take
+// the items round-robin; thread r of a group owns row r of the item's tile
+// (a warp reads 512 contiguous bytes per 16-byte load) and keeps the next
+// items' loads in flight in a register ring while it decodes the current
+// one. At each tile boundary of the CTA's range the groups' sums meet in
+// shared memory; a tile covered by one CTA goes straight to y, a tile split
+// between CTAs leaves one fp32 partial per CTA in the workspace and the last
+// CTA to arrive (integer atomic per tile) adds them in CTA order: results
+// are bitwise repeatable.
 //
 // Scalar codebook in shared memory: replicated once per lane with entry e of
 // lane l at byte e*256 + l*4, so the 32 lanes of a lookup always hit 32
 // different banks. The byte address is one PRMT away from the index word:
 // {0, 0, index byte, l*4}.
 //
-// 2D codebook: the 4096 fp32 pairs (32 KB) are kept once; lookups of random
-// pairs can conflict on banks (the pair table is too large to replicate).
+// 2D codebook: the 4096 fp32 pairs (32 KB) are kept once; random pair
+// lookups can conflict on banks (a per-lane replica would need 1 MB).
 //
-// Sidecar: each row keeps a pointer into its column-sorted patch list and
-// substitutes the stored value for the decoded one at the patched columns,
-// before the multiply (replacement, HXQ whitepaper, method section,
-// "Sidecar outlier correction").
+// Activations are staged once per CTA in shared memory (fp32, or bf16 when
+// fp32 would not fit), zero-padded to whole 64-weight stages.
 //
-// Split-K: units of one tile write fp32 partials to the workspace; the last
-// unit to arrive (counted with an integer atomic per tile) sums them in split
-// order s = 0, 1, ..., so results are bitwise repeatable.
+// Sidecar (replacement of single weights, HXQ whitepaper, method section,
+// "Sidecar outlier correction"): replacing w = c by v adds (v - c) x to the
+// dot product, so each entry carries delta = v - c (fp32, computed once when
+// the handle is built) and is applied as one extra multiply-add at the end of
+// its stage. A warp's entries for a stage (bucket of its 32 rows x 64
+// columns) are loaded one stage ahead, one entry per lane, and handed to the
+// owning lane with shuffles: no dependent memory access on the hot path.
 #include <algorithm>
 #include <climits>
 
@@ -37,304 +45,341 @@ namespace hxq {
 namespace {
 
 constexpr int kGemvThreads = 512;
-constexpr int kGroups = kGemvThreads / kTileRows;  // 4
+constexpr int kGroups = kGemvThreads / kTileRows;  // virtual CTAs per CTA
+constexpr size_t kSmemLimit = 227 * 1024;          // dynamic shared memory per CTA
 
-template <int MT>
-struct GemvSmem {
-  static constexpr size_t table_bytes(int mode) { return mode == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8; }
-  static constexpr size_t red_bytes() { return (size_t)kGroups * MT * kTileRows * sizeof(float); }
-};
+// Dynamic shared memory of one CTA: codebook table, activations (fp32 or
+// bf16) and the groups' partial sums.
+inline size_t gemv_smem(int mode, int MT, int Kp, bool xf32) {
+  return (size_t)(mode == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8) + (size_t)MT * Kp * (xf32 ? 4 : 2) +
+         (size_t)kGroups * MT * kTileRows * sizeof(float);
+}
+
+template <int MODE>
+constexpr int table_bytes() { return MODE == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8; }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Load 8 activations x[m][k0 .. k0+8) as fp32 (0 beyond row end or m >= M).
-__device__ __forceinline__ void load_x8(const uint16_t* __restrict__ x, int K, int M, int m, int k0, float (&f)[8]) {
-  uint4 q = make_uint4(0, 0, 0, 0);
-  if (m < M && k0 < K) q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)m * K + k0));
-  f[0] = bf16lo(q.x); f[1] = bf16hi(q.x); f[2] = bf16lo(q.y); f[3] = bf16hi(q.y);
-  f[4] = bf16lo(q.z); f[5] = bf16hi(q.z); f[6] = bf16lo(q.w); f[7] = bf16hi(q.w);
+// CTA whose item range [b W / G, (b+1) W / G) contains item w (W * G < 2^31).
+__device__ __forceinline__ int cta_of(int w, int W, int G) {
+  int b = (w * G) / W;
+  while (b + 1 < G && ((b + 1) * W) / G <= w) ++b;
+  while (b > 0 && (b * W) / G > w) --b;
+  return b;
 }
 
-struct Unit {
-  int t, s, st0, st1;  // tile, split, stage range [st0, st1)
-};
-
-__device__ __forceinline__ Unit unit_of(int u, int S, int n_stages) {
-  Unit U;
-  U.t = u / S;
-  U.s = u % S;
-  U.st0 = (int)((int64_t)U.s * n_stages / S);
-  U.st1 = (int)((int64_t)(U.s + 1) * n_stages / S);
-  return U;
-}
-
-// Sum the groups' partials of this unit and publish: straight to y when the
-// unit covers all of K, else through the workspace with the last-arriver sum.
-template <int MT>
-__device__ void finish_unit(const Layer& L, const Unit& U, int M, int S, float* red, float* __restrict__ y,
-                            float* __restrict__ work, int* __restrict__ counters, int* flag) {
-  const int rows = min(kTileRows, L.N - U.t * kTileRows);
-  for (int i = threadIdx.x; i < MT * kTileRows; i += blockDim.x) {
-    const int m = i / kTileRows, r = i % kTileRows;
-    if (m >= M || r >= rows) continue;
-    float v = 0.f;
+// Load the NP 16-byte index pieces of stage `st` of row r in tile t, and the
+// bounds of the sidecar bucket of this warp's 32 rows for that stage.
+template <int NP>
+__device__ __forceinline__ void load_stage(const Layer& L, int t, int st, int r, uint4 (&q)[NP], int& bs,
+                                           int& bc) {
+  const int rows = min(kTileRows, L.N - t * kTileRows);
+  if (r < rows) {
+    const uint8_t* p = L.idx + (size_t)t * kTileRows * L.KC * 16 * L.P + ((size_t)st * NP) * rows * 16 + r * 16;
 #pragma unroll
-    for (int g = 0; g < kGroups; ++g) v += red[(g * MT + m) * kTileRows + r];
-    const size_t n = (size_t)U.t * kTileRows + r;
-    if (S == 1) y[(size_t)m * L.N + n] = v;
-    else work[((size_t)U.s * M + m) * L.N + n] = v;
+    for (int j = 0; j < NP; ++j) q[j] = ldg_stream16(p + (size_t)j * rows * 16);
+  } else {
+#pragma unroll
+    for (int j = 0; j < NP; ++j) q[j] = make_uint4(0, 0, 0, 0);
   }
-  if (S == 1) return;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) *flag = atomicAdd(counters + U.t * 64, 1) == S - 1;
-  __syncthreads();
-  if (!*flag) return;
-  __threadfence();
-  for (int i = threadIdx.x; i < M * kTileRows; i += blockDim.x) {
-    const int m = i / kTileRows, r = i % kTileRows;
-    if (r >= rows) continue;
-    const size_t n = (size_t)U.t * kTileRows + r;
-    float v = 0.f;
-    for (int s = 0; s < S; ++s) v += __ldcg(work + ((size_t)s * M + m) * L.N + n);
-    y[(size_t)m * L.N + n] = v;
-  }
-  if (threadIdx.x == 0) counters[U.t * 64] = 0;
+  const int b = bucket_of(L, t, st, r >> 5);
+  bs = __ldg(L.bptr + b);
+  bc = __ldg(L.bptr + b + 1) - bs;
 }
 
-template <int MT>
-__global__ void __launch_bounds__(kGemvThreads, 1)
-gemv_scalar_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int S,
-                   float* __restrict__ work, int* __restrict__ counters) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  float* table = reinterpret_cast<float*>(smem);                       // 64 KB
-  float* red = reinterpret_cast<float*>(smem + 256 * 256);             // G*MT*128 floats
-  __shared__ int flag;
-  const int lane = threadIdx.x & 31;
-  const int g = threadIdx.x / kTileRows, r = threadIdx.x % kTileRows;
+// 16 activations x[m][k0 .. k0+16) from shared memory as fp32.
+template <bool XF32>
+__device__ __forceinline__ void x16(const uint8_t* xs, int Kp, int m, int k0, float (&f)[16]) {
+  if (XF32) {
+    const float4* p = reinterpret_cast<const float4*>(xs + ((size_t)m * Kp + k0) * 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = p[i];
+      f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(xs + ((size_t)m * Kp + k0) * 2);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 v = p[i];
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        f[8 * i + 2 * j] = bf16lo(u[j]);
+        f[8 * i + 2 * j + 1] = bf16hi(u[j]);
+      }
+    }
+  }
+}
 
-  for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x)
-    table[(i >> 5) * 64 + (i & 31)] = __ldg(L.codebook + (i >> 5));
+template <int MT, bool XF32>
+__device__ __forceinline__ void accumulate16(float2 (&acc)[MT], const float (&w)[16], const uint8_t* xs, int Kp,
+                                             int k0) {
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    float xv[16];
+    x16<XF32>(xs, Kp, m, k0, xv);
+#pragma unroll
+    for (int j = 0; j < 16; j += 2)
+      acc[m] = __ffma2_rn(make_float2(w[j], w[j + 1]), make_float2(xv[j], xv[j + 1]), acc[m]);
+  }
+}
+
+template <int MT, bool XF32>
+__device__ __forceinline__ void add_patch(float2 (&acc)[MT], float d, const uint8_t* xs, int Kp, int k) {
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const float xv = XF32 ? *reinterpret_cast<const float*>(xs + ((size_t)m * Kp + k) * 4)
+                          : bf16lo(*reinterpret_cast<const uint16_t*>(xs + ((size_t)m * Kp + k) * 2));
+    acc[m].x = fmaf(d, xv, acc[m].x);
+  }
+}
+
+// Byte offset of the first index piece of item w (tile-major order, NP
+// pieces per row and stage); the items of any contiguous range occupy one
+// contiguous byte range. Item W (one past the last) maps to the end.
+template <int NP>
+__device__ __forceinline__ size_t item_offset(const Layer& L, int w, int n_st) {
+  const int t = w / n_st, st = w % n_st;
+  if (t >= L.n_tiles) return (size_t)L.N * L.KC * 16 * L.P;
+  const int rows = min(kTileRows, L.N - t * kTileRows);
+  return (size_t)t * kTileRows * L.KC * 16 * L.P + (size_t)st * NP * rows * 16;
+}
+
+template <int MT, bool XF32, int MODE>
+__global__ void __launch_bounds__(kGemvThreads, 1)
+gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int W,
+            float* __restrict__ work, int* __restrict__ counters) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int TB = table_bytes<MODE>();
+  constexpr int NP = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per stage
+  uint8_t* xs = smem + TB;
+  // per-group partial sums [kGroups][MT][kTileRows], after the activations
+  float* red = reinterpret_cast<float*>(xs + (size_t)MT * L.Kp * (XF32 ? 4 : 2));
+  __shared__ int last_flag;
+
+  const int g = threadIdx.x >> 7, r = threadIdx.x & (kTileRows - 1), lane = threadIdx.x & 31;
+  const int n_st = n_stages(L);
+  const int G = gridDim.x;
+  const int w0 = (blockIdx.x * W) / G, w1 = ((blockIdx.x + 1) * W) / G;
+
+  // 0. the next kernel in the stream may start its own prologue
+  pdl_launch_dependents();
+  // 1. stream this CTA's whole index range into L2 (TMA bulk prefetch), then
+  //    issue this thread's first item load; items of this thread are
+  //    w0 + g, w0 + g + 4, ...
+  if (threadIdx.x == 0 && w1 > w0) {
+    const size_t a = item_offset<NP>(L, w0, n_st), b = item_offset<NP>(L, w1, n_st);
+    for (size_t o = a; o < b; o += 65536) prefetch_l2_bulk(L.idx + o, (uint32_t)min((size_t)65536, b - o));
+  }
+  uint4 cur[NP];
+  int cbs = 0, cbc = 0;
+  int nt = (w0 + g) / n_st, nst = (w0 + g) % n_st;  // next item to load
+  if (w0 + g < w1) load_stage<NP>(L, nt, nst, r, cur, cbs, cbc);
+
+  // 2. shared-memory codebook; activations once the previous kernel is done
+  if (MODE == HXQ_MODE_SCALAR8) {
+    float* tw = reinterpret_cast<float*>(smem);
+    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) tw[(i >> 5) * 64 + (i & 31)] = __ldg(L.codebook + (i >> 5));
+  } else {
+    const float4* cb = reinterpret_cast<const float4*>(L.codebook);
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) reinterpret_cast<float4*>(smem)[i] = __ldg(cb + i);
+  }
+  uint32_t ek = 0;  // sidecar entries (key, delta) of the current item, one per lane
+  float ed = 0.f;
+  if (lane < cbc) {
+    ek = __ldg(L.pkey + cbs + lane);
+    ed = __ldg(L.pdelta + cbs + lane);
+  }
+  pdl_wait();
+  for (int i = threadIdx.x; i < MT * (L.Kp / 8); i += blockDim.x) {
+    const int m = i / (L.Kp / 8), k = (i % (L.Kp / 8)) * 8;
+    uint4 q = make_uint4(0, 0, 0, 0);
+    if (m < M && k < L.K) q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)m * L.K + k));
+    if (XF32) {
+      float4* d = reinterpret_cast<float4*>(xs + ((size_t)m * L.Kp + k) * 4);
+      d[0] = make_float4(bf16lo(q.x), bf16hi(q.x), bf16lo(q.y), bf16hi(q.y));
+      d[1] = make_float4(bf16lo(q.z), bf16hi(q.z), bf16lo(q.w), bf16hi(q.w));
+    } else {
+      *reinterpret_cast<uint4*>(xs + ((size_t)m * L.Kp + k) * 2) = q;
+    }
+  }
   __syncthreads();
 
   const uint32_t lane4 = (uint32_t)lane * 4u;
-  const char* tb = reinterpret_cast<const char*>(table);
-  const int n_stages = L.Kp / kStageK;
-  const int units = L.n_tiles * S;
+  nst += kGroups;  // (nt, nst): item after the current one
+  while (nst >= n_st) { nst -= n_st; ++nt; }
 
-  for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const Unit U = unit_of(u, S, n_stages);
-    const int rows = min(kTileRows, L.N - U.t * kTileRows);
-    const int n = U.t * kTileRows + r;
-    float acc[MT];
+  for (int seg0 = w0; seg0 < w1;) {  // segments: the CTA's items of one tile
+    const int t = seg0 / n_st;
+    const int seg1 = min(w1, (t + 1) * n_st);
+    float2 acc[MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0.f;
-    if (r < rows) {
-      int p = 0, pend = 0, pk = INT_MAX;
-      {
-        // first patch at or after the unit's first column
-        int lo = L.row_ptr[n], hi = L.row_ptr[n + 1];
-        pend = hi;
-        const int k0 = U.st0 * kStageK;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (L.patch_k[mid] < k0) lo = mid + 1; else hi = mid;
-        }
-        p = lo;
-        pk = p < pend ? L.patch_k[p] : INT_MAX;
-      }
-      for (int st = U.st0 + g; st < U.st1; st += kGroups) {
-        uint4 q[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) q[c] = ldg_stream16(L.idx + piece_offset(L, U.t, st * 4 + c, 0, r));
+    for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.f, 0.f);
+
+    // this thread's items of the segment: w == w0 + g (mod 4)
+    for (int w = seg0 + ((w0 + g - seg0) % kGroups + kGroups) % kGroups; w < seg1; w += kGroups) {
+      // next item's loads go out first; they land while this item computes
+      uint4 nxt[NP];
+      int nbs = 0, nbc = 0;
+      if (w + kGroups < w1) load_stage<NP>(L, nt, nst, r, nxt, nbs, nbc);
+      nst += kGroups;
+      while (nst >= n_st) { nst -= n_st; ++nt; }
+
+      const int kst = (w - t * n_st) * kStageK;
+      if (MODE == HXQ_MODE_SCALAR8) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int k0 = st * kStageK + c * 16;
-          const uint32_t wd[4] = {q[c].x, q[c].y, q[c].z, q[c].w};
+          const uint32_t wd[4] = {cur[c].x, cur[c].y, cur[c].z, cur[c].w};
           float wv[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
-            const uint32_t a = prmt(wd[j >> 2], lane4, sel);
-            wv[j] = *reinterpret_cast<const float*>(tb + a);
+            const uint32_t a = prmt(wd[j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
+            wv[j] = *reinterpret_cast<const float*>(smem + a);
           }
-          while (pk < k0 + 16) {                       // rare: sidecar patches
-            if (pk >= k0) {
-              const float v = L.patch_v[p];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) wv[j] = sel_eq(pk - k0, j, v, wv[j]);
-            }
-            ++p;
-            pk = p < pend ? L.patch_k[p] : INT_MAX;
-          }
-#pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            float xa[8], xb[8];
-            load_x8(x, L.K, M, m, k0, xa);
-            load_x8(x, L.K, M, m, k0 + 8, xb);
-            float a = acc[m];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) a = fmaf(wv[j], xa[j], a);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) a = fmaf(wv[8 + j], xb[j], a);
-            acc[m] = a;
-          }
+          accumulate16<MT, XF32>(acc, wv, xs, L.Kp, kst + c * 16);
         }
-      }
-    }
+      } else {
+        uint32_t wd[13];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) red[(g * MT + m) * kTileRows + r] = acc[m];
-    __syncthreads();
-    finish_unit<MT>(L, U, M, S, red, y, work, counters, &flag);
-    __syncthreads();
-  }
-}
-
-template <int MT>
-__global__ void __launch_bounds__(kGemvThreads, 1)
-gemv_vq2d_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int S,
-                 float* __restrict__ work, int* __restrict__ counters) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  float2* table = reinterpret_cast<float2*>(smem);                     // 32 KB
-  float* red = reinterpret_cast<float*>(smem + 4096 * 8);
-  __shared__ int flag;
-  const int g = threadIdx.x / kTileRows, r = threadIdx.x % kTileRows;
-
-  const float2* cb2 = reinterpret_cast<const float2*>(L.codebook);
-  for (int i = threadIdx.x; i < 4096; i += blockDim.x) table[i] = __ldg(cb2 + i);
-  __syncthreads();
-
-  const int n_stages = L.Kp / kStageK;
-  const int units = L.n_tiles * S;
-
-  for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const Unit U = unit_of(u, S, n_stages);
-    const int rows = min(kTileRows, L.N - U.t * kTileRows);
-    const int n = U.t * kTileRows + r;
-    float acc[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0.f;
-    if (r < rows) {
-      int p, pend, pk;
-      {
-        int lo = L.row_ptr[n], hi = L.row_ptr[n + 1];
-        pend = hi;
-        const int k0 = U.st0 * kStageK;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (L.patch_k[mid] < k0) lo = mid + 1; else hi = mid;
+        for (int c = 0; c < 3; ++c) {
+          wd[4 * c] = cur[c].x; wd[4 * c + 1] = cur[c].y; wd[4 * c + 2] = cur[c].z; wd[4 * c + 3] = cur[c].w;
         }
-        p = lo;
-        pk = p < pend ? L.patch_k[p] : INT_MAX;
-      }
-      for (int st = U.st0 + g; st < U.st1; st += kGroups) {
-        uint32_t w[13];
+        wd[12] = 0;
 #pragma unroll
-        for (int pl = 0; pl < 3; ++pl) {
-          const uint4 q = ldg_stream16(L.idx + piece_offset(L, U.t, st, pl, r));
-          w[4 * pl] = q.x; w[4 * pl + 1] = q.y; w[4 * pl + 2] = q.z; w[4 * pl + 3] = q.w;
-        }
-        w[12] = 0;
-        const int kbase = st * kStageK;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {                 // 4 x 16 weights
+        for (int h = 0; h < 4; ++h) {
           float wv[16];
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
             const int j = h * 8 + jj, bit = 12 * j;
-            const uint32_t e = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & 0xFFF;
-            const float2 v = table[e];
-            wv[2 * jj] = v.x;
-            wv[2 * jj + 1] = v.y;
+            const uint32_t e8 = (bit & 31) >= 3
+                ? (__funnelshift_r(wd[bit >> 5], wd[(bit >> 5) + 1], (bit & 31) - 3) & 0x7FF8u)
+                : ((wd[bit >> 5] << (3 - (bit & 31))) & 0x7FF8u);
+            const float2 pr = *reinterpret_cast<const float2*>(smem + e8);
+            wv[2 * jj] = pr.x;
+            wv[2 * jj + 1] = pr.y;
           }
-          const int k0 = kbase + h * 16;
-          while (pk < k0 + 16) {
-            if (pk >= k0) {
-              const float v = L.patch_v[p];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) wv[j] = sel_eq(pk - k0, j, v, wv[j]);
-            }
-            ++p;
-            pk = p < pend ? L.patch_k[p] : INT_MAX;
-          }
-#pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            float xa[8], xb[8];
-            load_x8(x, L.K, M, m, k0, xa);
-            load_x8(x, L.K, M, m, k0 + 8, xb);
-            float a = acc[m];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) a = fmaf(wv[j], xa[j], a);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) a = fmaf(wv[8 + j], xb[j], a);
-            acc[m] = a;
-          }
+          accumulate16<MT, XF32>(acc, wv, xs, L.Kp, kst + h * 16);
         }
       }
-    }
+      // sidecar corrections of this item: acc += delta * x[k]
+      const int nb = min(cbc, 32);
+      for (int j = 0; j < nb; ++j) {
+        const uint32_t key = __shfl_sync(0xffffffffu, ek, j);
+        const float dv = __shfl_sync(0xffffffffu, ed, j);
+        if ((int)(key & 31) == lane) add_patch<MT, XF32>(acc, dv, xs, L.Kp, kst + (int)(key >> 5));
+      }
+      for (int j = 32; j < cbc; ++j) {  // more than 32 entries in one bucket: direct loads
+        const uint32_t key = __ldg(L.pkey + cbs + j);
+        if ((int)(key & 31) == lane)
+          add_patch<MT, XF32>(acc, __ldg(L.pdelta + cbs + j), xs, L.Kp, kst + (int)(key >> 5));
+      }
+      // advance: next item's sidecar entries, then its index pieces
+      ek = 0;
+      ed = 0.f;
+      if (lane < nbc) {
+        ek = __ldg(L.pkey + nbs + lane);
+        ed = __ldg(L.pdelta + nbs + lane);
+      }
 #pragma unroll
-    for (int m = 0; m < MT; ++m) red[(g * MT + m) * kTileRows + r] = acc[m];
+      for (int j = 0; j < NP; ++j) cur[j] = nxt[j];
+      cbs = nbs;
+      cbc = nbc;
+    }
+
+    // segment end: the 4 groups' sums meet in shared memory
+#pragma unroll
+    for (int m = 0; m < MT; ++m) red[(g * MT + m) * kTileRows + r] = acc[m].x + acc[m].y;
     __syncthreads();
-    finish_unit<MT>(L, U, M, S, red, y, work, counters, &flag);
+    const int rows = min(kTileRows, L.N - t * kTileRows);
+    const bool full = seg0 == t * n_st && seg1 == (t + 1) * n_st;
+    const int slot = (t == w0 / n_st) ? 0 : 1;
+    float* part = work + (size_t)(blockIdx.x * 2 + slot) * MT * kTileRows;
+    for (int i = threadIdx.x; i < MT * kTileRows; i += blockDim.x) {
+      const int m = i / kTileRows, rr = i % kTileRows;
+      const float v = red[(0 * MT + m) * kTileRows + rr] + red[(1 * MT + m) * kTileRows + rr] +
+                      red[(2 * MT + m) * kTileRows + rr] + red[(3 * MT + m) * kTileRows + rr];
+      if (full) {
+        if (m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
+      } else {
+        part[i] = v;
+      }
+    }
+    if (!full) {
+      __threadfence();
+      __syncthreads();
+      const int c_first = cta_of(t * n_st, W, G), c_last = cta_of((t + 1) * n_st - 1, W, G);
+      if (threadIdx.x == 0) last_flag = atomicAdd(counters + t, 1) == c_last - c_first;
+      __syncthreads();
+      if (last_flag) {
+        __threadfence();
+        for (int i = threadIdx.x; i < MT * kTileRows; i += blockDim.x) {
+          const int m = i / kTileRows, rr = i % kTileRows;
+          if (m >= M || rr >= rows) continue;
+          float v = 0.f;
+#pragma unroll 4
+          for (int c = c_first; c <= c_last; ++c) {
+            const int cs = (t == ((c * W) / G) / n_st) ? 0 : 1;
+            v += __ldcg(work + (size_t)(c * 2 + cs) * MT * kTileRows + i);
+          }
+          y[(size_t)m * L.N + t * kTileRows + rr] = v;
+        }
+        if (threadIdx.x == 0) counters[t] = 0;
+      }
+    }
     __syncthreads();
+    seg0 = seg1;
   }
 }
 
-template <int MT>
-cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, float* y, int M, int S, cudaStream_t s) {
-  const bool scalar = h.L.mode == HXQ_MODE_SCALAR8;
-  const size_t smem = GemvSmem<MT>::table_bytes(h.L.mode) + GemvSmem<MT>::red_bytes();
-  auto kern = scalar ? gemv_scalar_kernel<MT> : gemv_vq2d_kernel<MT>;
+template <int MT, bool XF32, int MODE>
+cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t s) {
+  const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32);
+  auto kern = gemv_kernel<MT, XF32, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) per_sm = 1;
-  const int units = h.L.n_tiles * S;
-  const int grid = std::min(units, h.num_sms * per_sm);
-  kern<<<grid, kGemvThreads, smem, s>>>(h.L, x, y, M, S, h.d_work, h.d_counters);
-  return cudaGetLastError();
+  const int W = h.L.n_tiles * (h.L.Kp / kStageK);
+  return launch_pdl(kern, grid, kGemvThreads, smem, s, h.L, x, y, M, W, h.d_work, h.d_counters);
 }
+
+template <int MT, int MODE>
+cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t s) {
+  if (gemv_smem(MODE, MT, h.L.Kp, true) <= kSmemLimit) return launch_cfg<MT, true, MODE>(h, x, y, M, grid, s);
+  return launch_cfg<MT, false, MODE>(h, x, y, M, grid, s);
+}
+
+template <int MODE>
+cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t s) {
+  if (M <= 1) return launch_mt<1, MODE>(h, x, y, M, grid, s);
+  if (M <= 2) return launch_mt<2, MODE>(h, x, y, M, grid, s);
+  if (M <= 4) return launch_mt<4, MODE>(h, x, y, M, grid, s);
+  if (M <= 8) return launch_mt<8, MODE>(h, x, y, M, grid, s);
+  if (M <= 16) return launch_mt<16, MODE>(h, x, y, M, grid, s);
+  return launch_mt<32, MODE>(h, x, y, M, grid, s);
+}
+
+int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : M <= 16 ? 16 : 32; }
 
 }  // namespace
 
-// Split count along K: balance units over the persistent CTAs (whole waves),
-// keep every group busy (at least kGroups stages per unit) and stay within
-// the workspace.
-int choose_split_gemv(const hxq_linear& h, int M) {
-  const int n_stages = h.L.Kp / kStageK;
-  const int slots = h.num_sms;
-  int best = 1;
-  double best_score = -1.0;
-  for (int S = 1; S <= std::min(n_stages, kMaxSplitK); ++S) {
-    if (S > 1 && (size_t)S * M * h.L.N > h.work_floats) break;
-    const int units = h.L.n_tiles * S;
-    const int waves = (units + slots - 1) / slots;
-    const double wave_eff = (double)units / ((double)waves * slots);
-    const double per_unit = (double)n_stages / S;
-    const double group_eff = std::min(1.0, per_unit / kGroups);
-    const double score = wave_eff * group_eff / (1.0 + 0.002 * S);
-    if (score > best_score + 1e-9) {
-      best_score = score;
-      best = S;
-    }
-  }
-  return best;
+bool gemv_supports(const hxq_linear& h, int M) {
+  return M >= 1 && M <= 32 && gemv_smem(h.L.mode, mt_of(M), h.L.Kp, false) <= kSmemLimit;
 }
 
+// Persistent grid: one CTA per SM, fewer when the layer has fewer work items.
+// `split` (when non-zero) sets the grid so that each tile's K is shared by
+// about `split` CTAs.
 cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M, int split, cudaStream_t s) {
-  const int n_stages = h.L.Kp / kStageK;
-  int S = std::max(1, std::min(split, n_stages));
-  if (S > 1 && (size_t)S * M * h.L.N > h.work_floats) return cudaErrorInvalidValue;
-  if (M <= 1) return launch_mt<1>(h, x, y, M, S, s);
-  if (M <= 2) return launch_mt<2>(h, x, y, M, S, s);
-  if (M <= 4) return launch_mt<4>(h, x, y, M, S, s);
-  if (M <= 8) return launch_mt<8>(h, x, y, M, S, s);
-  if (M <= 16) return launch_mt<16>(h, x, y, M, S, s);
-  if (M <= 32) return launch_mt<32>(h, x, y, M, S, s);
-  return cudaErrorInvalidValue;
+  if (!gemv_supports(h, M)) return cudaErrorInvalidValue;
+  const int64_t W = (int64_t)h.L.n_tiles * (h.L.Kp / kStageK);
+  int64_t grid = split > 0 ? (int64_t)h.L.n_tiles * split : h.num_sms;
+  grid = std::max<int64_t>(1, std::min<int64_t>({grid, (int64_t)h.num_sms, W}));
+  if (W * grid >= INT_MAX) return cudaErrorInvalidValue;  // item arithmetic is 32-bit
+  // every CTA writes at most two partial tiles of mt_of(M) x 128 floats
+  if ((size_t)grid * 2 * mt_of(M) * kTileRows > h.work_floats) return cudaErrorInvalidValue;
+  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, (int)grid, s);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, (int)grid, s);
 }
 
 }  // namespace hxq

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/hxq.h"
+#include "hxq.h"  // include/ (on the include path)
 
 namespace hxq {
 
@@ -41,10 +41,25 @@ struct Layer {
   int n_tiles;       // ceil(N / 128)
   const float* codebook;     // 256 or 4096*2 floats
   const uint8_t* idx;        // tiled layout above
-  const int* row_ptr;        // [N+1] offsets into the patch lists
-  const int* patch_k;        // per row, ascending k
-  const float* patch_v;      // replacement values
+  // Sidecar, bucketed by (tile t, stage st, warp quadrant q = row / 32):
+  // bucket b = (t * n_stages + st) * 4 + q holds entries [bptr[b], bptr[b+1])
+  // of the position-sorted sidecar that fall in rows 32q .. 32q+31 of tile t
+  // and columns 64 st .. 64 st + 63. A warp loads its bucket for the next
+  // stage together with that stage's indices, so applying the sidecar costs
+  // no dependent memory round trip.
+  const int* bptr;           // [n_tiles * n_stages * 4 + 1]
+  const uint32_t* pkey;      // lane (bits 0-4) | column within the stage (bits 5-10)
+  const float* pval;         // the replacement value v
+  const float* pdelta;       // v - (codebook value it replaces), rounded to fp32
 };
+
+constexpr int kQuads = kTileRows / 32;
+
+__host__ __device__ inline int n_stages(const Layer& L) { return L.Kp / kStageK; }
+__host__ __device__ inline int bucket_of(const Layer& L, int t, int st, int q) {
+  return (t * n_stages(L) + st) * kQuads + q;
+}
+__host__ __device__ inline uint32_t patch_key(int lane, int kk) { return (uint32_t)lane | ((uint32_t)kk << 5); }
 
 __host__ __device__ inline size_t piece_offset(const Layer& L, int t, int c, int p, int r) {
   const int rows = min(kTileRows, L.N - t * kTileRows);
@@ -60,9 +75,10 @@ struct hxq_linear {
   int num_sms;
   float* d_codebook;
   uint8_t* d_idx;
-  int* d_row_ptr;
-  int* d_patch_k;
-  float* d_patch_v;
+  int* d_bptr;
+  uint32_t* d_pkey;
+  float* d_pval;
+  float* d_pdelta;
   float* d_work;        // split-K partial sums
   size_t work_floats;
   int* d_counters;      // per output tile: arrivals of split-K partials
@@ -78,8 +94,27 @@ cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M,
                         cudaStream_t s);
 cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, float* y, int M, int split,
                       cudaStream_t s);
-int choose_split_gemv(const hxq_linear& h, int M);
-int choose_split_tc(const hxq_linear& h, int M);
+bool gemv_supports(const hxq_linear& h, int M);
+size_t tc_workspace_floats(int num_sms);
+
+// Launch `kern` with programmatic stream serialization: it may start while
+// the previous kernel in the stream drains, and waits for it (griddepcontrol
+// .wait) only where it reads that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 // Device status bits.
 constexpr int kStatusWaitTimeout = 1;
@@ -140,7 +175,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if ((i & 255) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort = 1;
       return false;
     }
@@ -233,6 +268,17 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
   return r;
 }
+
+// Asynchronous bulk prefetch of [p, p + bytes) from global memory into L2
+// (TMA engine; no registers, completes on its own). p and bytes: multiples of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue now / wait until the previous kernel's results are visible.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint4 ldg_stream16(const void* p) {
   uint4 v;

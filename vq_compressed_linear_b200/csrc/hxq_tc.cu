@@ -10,15 +10,22 @@
 //    decoded weights never touch shared or global memory. Thread r of a
 //    decoding warp group owns TMEM lane r = row r of the tile; it reads its
 //    16-byte index pieces (a warp reads 512 contiguous bytes), looks the
-//    indices up in a shared-memory table, patches sidecar columns, packs two
-//    bf16 per 32-bit TMEM cell and stores 64 weights (one pipeline stage) at
-//    a time.
-//  * B (x) arrives by TMA into 128-byte-swizzled shared memory, 64 tokens'
-//    worth of K per stage; rows past M and columns past K read as zero.
+//    indices up in a shared-memory table, substitutes sidecar values, packs
+//    two bf16 per 32-bit TMEM cell and stores 64 weights (one stage) at a time.
+//  * B (x) arrives by TMA into 128-byte-swizzled shared memory, 64 columns of
+//    K per stage; rows past M and columns past K read as zero.
 //  * One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32 in TMEM)
-//    and signals stage release and completion with tcgen05.commit.
-//  * The decoding warps then read D back with tcgen05.ld and store y (or a
-//    split-K partial; the last of the S partials of a tile sums them in order).
+//    and signals stage release and segment completion with tcgen05.commit.
+//  * Four epilogue warps read D back with tcgen05.ld and store y.
+//
+// Work decomposition (stream-K): the items are (token block, tile, stage)
+// triples numbered stage-fastest; a persistent grid of one CTA per SM takes
+// contiguous item ranges of equal size. A run of items of one (token block,
+// tile) is a segment; a segment that covers all of K is written to y
+// directly, the others leave fp32 partials in the workspace and the last
+// contributor to arrive sums them in CTA order (bitwise repeatable). With
+// BN <= 128 the accumulator is double-buffered so the next segment's MMAs
+// overlap the previous segment's epilogue.
 //
 // Weight precision (TERMS):
 //  * TERMS = 1 (M > 32, the prefill): each weight is rounded to bf16 (round
@@ -29,10 +36,13 @@
 //    significand bits: |w - hi - mid| <= 2^-17 |w|, inside the fp32-codebook
 //    tolerance 1e-5 * sum |x||w| that applies to the decode GEMV.
 //
-// Pipeline: kStages slots, each with an x buffer (TMA) and an A region in
-// TMEM; mbarriers full_x / full_a / empty per slot and one for the
-// accumulator. Every wait is bounded (2 s): on timeout the CTA sets a status
-// bit, drains what it issued, frees TMEM and returns.
+// Sidecar (HXQ whitepaper, method section, "Sidecar outlier correction"):
+// the decoding warp loads its (tile, stage, 32-row) bucket one item ahead,
+// one entry per lane; shuffles hand each entry to its row's lane, which
+// substitutes the value (as bf16, or as its hi+mid split) before the store.
+//
+// Every mbarrier wait is bounded (2 s): on timeout the CTA sets a status bit,
+// drains what it issued, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -45,11 +55,24 @@
 namespace hxq {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kDecodeGroups = 4;                       // groups of 4 warps (128 rows)
-constexpr int kTcThreads = 128 + kDecodeGroups * 128;  // warps 0..3 control, 4.. decode
-constexpr int kAColBase = 256;                         // A regions live in TMEM columns 256..511
+constexpr int kEpiWarp0 = 4;                            // warps 4..7: epilogue
+constexpr int kDecWarp0 = 8;                            // warps 8..: decoders
 constexpr int kTmemCols = 512;
+constexpr int kMaxTokBlocks = 64;                       // token blocks per launch (counter space)
+constexpr int kMaxContrib = 4;                          // CTAs sharing one tile's K at most
+constexpr int kPrefetchItems = 16;                      // index bytes streamed into L2 this far ahead
+
+// Decoding groups of 4 warps (128 rows each): 4 for bf16 weights, 3 for the
+// hi+mid split, whose decoders need more registers.
+template <int TERMS>
+constexpr int dec_groups() { return TERMS == 1 ? 4 : 3; }
+template <int TERMS>
+constexpr int tc_threads() { return 32 * (kDecWarp0 + 4 * dec_groups<TERMS>()); }
+// Pipeline stages in flight: a multiple of the decoding groups (each slot
+// belongs to one group), as many as shared memory (x slots next to the
+// table) and TMEM (A slots next to the accumulators) allow.
+template <int BN, int TERMS>
+constexpr int num_slots() { return TERMS == 2 ? 6 : (BN >= 256 ? 4 : 8); }
 
 __device__ __forceinline__ uint32_t bf16_bits(float f) {
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
@@ -80,58 +103,77 @@ constexpr size_t table_bytes() {
   return MODE == HXQ_MODE_SCALAR8 ? 256 * 256 : (TERMS == 1 ? 4096 * 4 : 4096 * 8);
 }
 
+template <int BN>
+constexpr int num_acc() { return BN <= 128 ? 2 : 1; }
+
 template <int BN, int TERMS, int MODE>
 constexpr size_t tc_smem_bytes() {
-  return 1024 /* alignment slack */ + (size_t)kStages * BN * 128 + table_bytes<MODE, TERMS>();
+  return table_bytes<MODE, TERMS>() + 1024 /* alignment slack */ + (size_t)num_slots<BN, TERMS>() * BN * 128;
 }
 
-// Replace the weight at column offset j (0..15) of a 16-weight chunk by the
-// word `pw` (scalar tables: one word per weight).
+// Replace the word at offset j (0..15) of a 16-weight chunk by pw.
 __device__ __forceinline__ void patch16(uint32_t (&v)[16], int j, uint32_t pw) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = sel_eq(i, j, pw, v[i]);
 }
-// Replace half `h` of pair word j (0..7) by the 16-bit value hv.
+// Replace half h of pair word j (0..7) by the 16-bit value hv.
 __device__ __forceinline__ void patch8_half(uint32_t (&v)[8], int j, int h, uint32_t hv) {
 #pragma unroll
   for (int i = 0; i < 8; ++i)
     v[i] = sel_eq(i, j, h ? ((v[i] & 0xFFFFu) | (hv << 16)) : ((v[i] & 0xFFFF0000u) | hv), v[i]);
 }
 
+// CTA whose item range [b W / G, (b+1) W / G) contains item w.
+// (W * G < 2^31, checked at launch)
+__device__ __forceinline__ int cta_of(int w, int W, int G) {
+  int b = (w * G) / W;
+  while (b + 1 < G && ((b + 1) * W) / G <= w) ++b;
+  while (b > 0 && (b * W) / G > w) --b;
+  return b;
+}
+
 template <int BN, int TERMS, int MODE>
-__global__ void __launch_bounds__(kTcThreads, 1)
-tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ y, int M, int S,
+__global__ void __launch_bounds__(tc_threads<TERMS>(), 1)
+tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ y, int M, int tok0, int n_tb,
           float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
   constexpr int XSLOT = BN * 128;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* xs = smem;
-  uint8_t* table = smem + kStages * XSLOT;
-  __shared__ uint64_t bar_x[kStages], bar_a[kStages], bar_empty[kStages], bar_acc;
+  constexpr int kSlots = num_slots<BN, TERMS>();
+  constexpr int kDecGroups = dec_groups<TERMS>();
+  static_assert(kSlots % kDecGroups == 0, "each slot belongs to one decoding group");
+  constexpr int TB = (int)table_bytes<MODE, TERMS>();
+  constexpr int NACC = num_acc<BN>();
+  constexpr int ACOL0 = NACC * BN < 64 ? 64 : NACC * BN;  // first TMEM column of the A slots
+  static_assert(ACOL0 + kSlots * 32 * TERMS <= kTmemCols, "TMEM budget");
+  // The decode table sits at the start of dynamic shared memory so lookups
+  // address it from the array symbol (plain LDS); the x slots follow,
+  // aligned to 1024 bytes for the 128-byte swizzle.
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t xs_pad = (1024u - ((smem_u32(smem) + TB) & 1023u)) & 1023u;
+  uint8_t* xs = smem + TB + xs_pad;
+  __shared__ uint64_t bar_x[kSlots], bar_a[kSlots], bar_empty[kSlots], bar_acc[NACC], bar_dfree[NACC], bar_drain;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_sh, last_sh;
+  __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tb = (M + BN - 1) / BN;
-  int u = blockIdx.x;
-  const int s = u % S;
-  u /= S;
-  const int tb = u % n_tb, t = u / n_tb;
-  const int n_stages_all = L.Kp / kStageK;
-  const int st0 = (int)((int64_t)s * n_stages_all / S);
-  const int st1 = (int)((int64_t)(s + 1) * n_stages_all / S);
-  const int nst = st1 - st0;
-  const int rows = min(kTileRows, L.N - t * kTileRows);
+  const int n_st = n_stages(L);
+  const int W = n_tb * L.n_tiles * n_st;
+  const int G = gridDim.x;
+  const int w0 = (blockIdx.x * W) / G, w1 = ((blockIdx.x + 1) * W) / G;
+  const int n_items = w1 - w0;
 
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(&bar_x[i], 1);
       mbar_init(&bar_a[i], 4);
       mbar_init(&bar_empty[i], 1);
     }
-    mbar_init(&bar_acc, 1);
+    for (int i = 0; i < NACC; ++i) {
+      mbar_init(&bar_acc[i], 1);
+      mbar_init(&bar_dfree[i], 4);
+    }
+    mbar_init(&bar_drain, 1);
     abort_sh = 0;
-    last_sh = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) prefetch_tmap(&tmx);
@@ -141,7 +183,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
   }
   // shared-memory decode table
   if (MODE == HXQ_MODE_SCALAR8) {
-    uint32_t* tw = reinterpret_cast<uint32_t*>(table);
+    uint32_t* tw = reinterpret_cast<uint32_t*>(smem);
     for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
       const float c = __ldg(L.codebook + (i >> 5));
       tw[(i >> 5) * 64 + (i & 31)] = TERMS == 1 ? (bf16_bits(c) << 16) : split_word(c);
@@ -151,10 +193,10 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
     for (int i = threadIdx.x; i < 4096; i += blockDim.x) {
       const float2 c = __ldg(cb2 + i);
       if (TERMS == 1) {
-        reinterpret_cast<uint32_t*>(table)[i] = bf16_bits(c.x) | (bf16_bits(c.y) << 16);
+        reinterpret_cast<uint32_t*>(smem)[i] = bf16_bits(c.x) | (bf16_bits(c.y) << 16);
       } else {
         const uint32_t a = split_word(c.x), b = split_word(c.y);
-        reinterpret_cast<uint2*>(table)[i] = make_uint2(prmt(a, b, 0x7632), prmt(a, b, 0x5410));
+        reinterpret_cast<uint2*>(smem)[i] = make_uint2(prmt(a, b, 0x7632), prmt(a, b, 0x5410));
       }
     }
   }
@@ -167,98 +209,207 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
   if (warp == 0) {
     // ---------------- TMA producer: x tiles
     if (lane == 0) {
+      // the decoders' index bytes: streamed into L2 kPrefetchItems ahead
+      constexpr int NPC = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;
+      auto prefetch_item = [&](int i) {
+        const int w = w0 + i, t = (w / n_st) % L.n_tiles, st = w % n_st;
+        const int rows = min(kTileRows, L.N - t * kTileRows);
+        prefetch_l2_bulk(L.idx + piece_offset(L, t, MODE == HXQ_MODE_SCALAR8 ? st * 4 : st, 0, 0),
+                         (uint32_t)(NPC * rows * 16));
+      };
+      for (int i = 0; i < min(n_items, kPrefetchItems); ++i) prefetch_item(i);
+      pdl_wait();  // x may be the previous kernel's output
       int issued = 0;
-      for (int i = 0; i < nst; ++i) {
-        const int b = i % kStages;
-        if (!mbar_wait(&bar_empty[b], ((i / kStages) & 1) ^ 1, abrt)) break;
+      for (int i = 0; i < n_items; ++i) {
+        const int w = w0 + i, b = i % kSlots;
+        const int T = w / n_st, st = w % n_st;
+        const int tb = T / L.n_tiles;
+        if (i + kPrefetchItems < n_items) prefetch_item(i + kPrefetchItems);
+        if (!mbar_wait(&bar_empty[b], ((i / kSlots) & 1) ^ 1, abrt)) break;
         mbar_arrive_expect_tx(&bar_x[b], XSLOT);
-        tma_load_2d(xs + b * XSLOT, &tmx, &bar_x[b], (st0 + i) * kStageK, tb * BN);
+        tma_load_2d(xs + b * XSLOT, &tmx, &bar_x[b], st * kStageK, tok0 + tb * BN);
         ++issued;
       }
       if (*abrt) {  // drain the loads this thread issued before leaving
-        for (int i = max(0, issued - kStages); i < issued; ++i) {
-          volatile int never = 0;
-          mbar_wait(&bar_x[i % kStages], (i / kStages) & 1, &never);
-        }
+        volatile int never = 0;
+        for (int i = max(0, issued - kSlots); i < issued; ++i)
+          mbar_wait(&bar_x[i % kSlots], (i / kSlots) & 1, &never);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16<BN>();
-      for (int i = 0; i < nst; ++i) {
-        const int b = i % kStages;
-        const uint32_t par = (i / kStages) & 1;
-        if (!mbar_wait(&bar_x[b], par, abrt)) break;
-        if (!mbar_wait(&bar_a[b], par, abrt)) break;
+      int seg = -1;
+      for (int i = 0; i < n_items; ++i) {
+        const int w = w0 + i, b = i % kSlots;
+        const bool first = (i == 0) || (w % n_st == 0);
+        const bool last = (i == n_items - 1) || ((w + 1) % n_st == 0);
+        if (first) {
+          ++seg;
+          const int u = seg / NACC;
+          if (u >= 1 && !mbar_wait(&bar_dfree[seg % NACC], (u - 1) & 1, abrt)) break;
+        }
+        const uint32_t par = (i / kSlots) & 1;
+        if (!mbar_wait(&bar_x[b], par, abrt) || !mbar_wait(&bar_a[b], par, abrt)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(xs + b * XSLOT);
+        const uint32_t dcol = tmem + (seg % NACC) * BN;
 #pragma unroll
         for (int kk = 0; kk < kStageK / 16; ++kk) {
           const uint64_t bdesc = smem_desc_sw128(xaddr + kk * 32);
 #pragma unroll
           for (int term = 0; term < TERMS; ++term) {
-            const uint32_t acol = tmem + kAColBase + b * 32 * TERMS + term * 32 + kk * 8;
-            tc_mma_ts(tmem, acol, bdesc, idesc, (i | kk | term) ? 1u : 0u);
+            const uint32_t acol = tmem + ACOL0 + b * 32 * TERMS + term * 32 + kk * 8;
+            tc_mma_ts(dcol, acol, bdesc, idesc, (!first || kk || term) ? 1u : 0u);
           }
         }
         tc_commit(&bar_empty[b]);
+        if (last) tc_commit(&bar_acc[seg % NACC]);
       }
-      tc_commit(&bar_acc);
       if (*abrt) {  // let issued MMAs finish before TMEM is freed
         volatile int never = 0;
-        mbar_wait(&bar_acc, 0, &never);
+        tc_commit(&bar_drain);
+        mbar_wait(&bar_drain, 0, &never);
       }
     }
-  } else if (warp >= 4) {
-    // ---------------- decoders, then epilogue
-    const int dg = (warp - 4) >> 2;  // decode group
-    const int q = warp & 3;          // TMEM lane quadrant
-    const int r = q * 32 + lane;     // row of the tile
-    const int n = t * kTileRows + r;
-    const bool valid = r < rows;
+  } else if (warp >= kEpiWarp0 && warp < kDecWarp0) {
+    // ---------------- epilogue: D (y^T tile) from TMEM to y / workspace
+    const int q = warp & 3, r = q * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    const uint32_t lane4 = (uint32_t)lane * 4u;
-    const char* tb8 = reinterpret_cast<const char*>(table);
-
-    int p = 0, pend = 0, pk = INT_MAX;
-    if (valid) {
-      int lo = L.row_ptr[n], hi = L.row_ptr[n + 1];
-      pend = hi;
-      const int k0 = st0 * kStageK;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (L.patch_k[mid] < k0) lo = mid + 1; else hi = mid;
-      }
-      p = lo;
-      pk = p < pend ? L.patch_k[p] : INT_MAX;
-    }
-    constexpr int NPC = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per stage
-    uint4 qn[NPC];
-    auto load_stage = [&](int st, uint4 (&dst)[NPC]) {
+    pdl_wait();  // y, the workspace and the counters may be in use by the previous kernel
+    int seg = -1;
+    for (int i = 0; i < n_items; ++i) {
+      const int w = w0 + i;
+      if (!((i == n_items - 1) || ((w + 1) % n_st == 0))) continue;  // not a segment end
+      ++seg;
+      const int T = w / n_st, tb = T / L.n_tiles, t = T % L.n_tiles;
+      const int seg_start = max(w0, T * n_st);
+      const bool full = seg_start == T * n_st && w == T * n_st + n_st - 1;
+      const int rows = min(kTileRows, L.N - t * kTileRows);
+      const int n = t * kTileRows + r;
+      const int tok_b = tok0 + tb * BN;           // first token of this block
+      const int ntok = min(BN, M - tok_b);
+      if (!mbar_wait(&bar_acc[seg % NACC], (seg / NACC) & 1, abrt)) break;
+      tc_fence_after();
+      const int slot = (T == w0 / n_st) ? 0 : 1;
+      float* part = work + ((size_t)(blockIdx.x * 2 + slot) * BN) * kTileRows + r;
+      const uint32_t dcol = lane_base + (seg % NACC) * BN;
+#pragma unroll 1
+      for (int cc = 0; cc < BN; cc += 16) {
+        uint32_t v[16];
+        tmem_ld16(dcol + cc, v);
+        tmem_wait_ld();
+        if (full) {
+          if (r < rows) {
 #pragma unroll
-      for (int c = 0; c < NPC; ++c) {
-        if (valid) {
-          const int chunk = MODE == HXQ_MODE_SCALAR8 ? st * 4 + c : st;
-          const int plane = MODE == HXQ_MODE_SCALAR8 ? 0 : c;
-          dst[c] = ldg_stream16(L.idx + piece_offset(L, t, chunk, plane, r));
+            for (int j = 0; j < 16; ++j)
+              if (cc + j < ntok) y[(size_t)(tok_b + cc + j) * L.N + n] = __uint_as_float(v[j]);
+          }
         } else {
-          dst[c] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) part[(size_t)(cc + j) * kTileRows] = __uint_as_float(v[j]);
         }
       }
-    };
-    if (dg < nst) load_stage(st0 + dg, qn);
-
-    for (int i = dg; i < nst; i += kDecodeGroups) {
-      const int b = i % kStages;
-      uint4 qc[NPC];
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_dfree[seg % NACC]);
+      if (!full) {
+        // Split tile: each epilogue warp counts its own 32 rows, so no
+        // barrier spans warps (a warp that gave up a wait cannot strand the
+        // others). The last contributor's warp sums the partials in CTA order.
+        __threadfence();
+        __syncwarp();
+        const int c_first = cta_of(T * n_st, W, G), c_last = cta_of(T * n_st + n_st - 1, W, G);
+        int last = 0;
+        if (lane == 0) last = atomicAdd(counters + T * kQuads + q, 1) == c_last - c_first;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          if (r < rows) {
+            for (int j0 = 0; j0 < ntok; j0 += 4) {  // 4 tokens' loads in flight per contributor
+              float s4[4] = {0.f, 0.f, 0.f, 0.f};
+              for (int c = c_first; c <= c_last; ++c) {
+                const int cs = (T == ((c * W) / G) / n_st) ? 0 : 1;
+                const float* src = work + ((size_t)(c * 2 + cs) * BN + j0) * kTileRows + r;
 #pragma unroll
-      for (int c = 0; c < NPC; ++c) qc[c] = qn[c];
-      if (i + kDecodeGroups < nst) load_stage(st0 + i + kDecodeGroups, qn);
-      if (!mbar_wait(&bar_empty[b], ((i / kStages) & 1) ^ 1, abrt)) break;
+                for (int u = 0; u < 4; ++u)
+                  if (j0 + u < ntok) s4[u] += __ldcg(src + u * kTileRows);
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if (j0 + u < ntok) y[(size_t)(tok_b + j0 + u) * L.N + n] = s4[u];
+            }
+          }
+          if (lane == 0) counters[T * kQuads + q] = 0;
+        }
+      }
+    }
+  } else if (warp >= kDecWarp0) {
+    // ---------------- decoders
+    const int dg = (warp - kDecWarp0) >> 2;  // decoding group
+    const int q = warp & 3;                  // TMEM lane quadrant
+    const int r = q * 32 + lane;             // row of the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    const uint32_t lane4 = (uint32_t)lane * 4u;
+    constexpr int NPC = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per stage
+
+    // index pieces and sidecar bucket bounds of one item
+    auto load_item = [&](int i, uint4 (&qd)[NPC], int& bs, int& bc) {
+      const int w = w0 + i;
+      const int T = w / n_st, st = w % n_st, t = T % L.n_tiles;
+      const int rows = min(kTileRows, L.N - t * kTileRows);
+#pragma unroll
+      for (int c = 0; c < NPC; ++c) {
+        if (r < rows) {
+          const int chunk = MODE == HXQ_MODE_SCALAR8 ? st * 4 + c : st;
+          const int plane = MODE == HXQ_MODE_SCALAR8 ? 0 : c;
+          qd[c] = ldg_stream16(L.idx + piece_offset(L, t, chunk, plane, r));
+        } else {
+          qd[c] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      const int b = bucket_of(L, t, st, q);
+      bs = __ldg(L.bptr + b);
+      bc = __ldg(L.bptr + b + 1) - bs;
+    };
+    uint4 qc[NPC];
+    int cbs = 0, cbc = 0;
+    if (dg < n_items) load_item(dg, qc, cbs, cbc);
+
+    for (int i = dg; i < n_items; i += kDecGroups) {
+      const int b = i % kSlots;
+      // the group's next item loads first: they land while this one decodes
+      uint4 qn[NPC];
+      int nbs = 0, nbc = 0;
+      if (i + kDecGroups < n_items) load_item(i + kDecGroups, qn, nbs, nbc);
+      const int bs = cbs, bc = cbc;
+      // this item's sidecar entries, one per lane
+      uint32_t ek = 0xFFFFFFFFu;
+      float ev = 0.f;
+      if (lane < bc) {
+        ek = __ldg(L.pkey + bs + lane);
+        ev = __ldg(L.pval + bs + lane);
+      }
+      // entries of this lane's row: up to two kept in registers, more -> rescan
+      int pk0 = -1, pk1 = -1;
+      float pv0 = 0.f, pv1 = 0.f;
+      bool more = bc > 32;
+      {
+        const int nb = min(bc, 32);
+        for (int j = 0; j < nb; ++j) {
+          const uint32_t key = __shfl_sync(0xffffffffu, ek, j);
+          const float v = __shfl_sync(0xffffffffu, ev, j);
+          if ((int)(key & 31) == lane) {
+            if (pk0 < 0) { pk0 = (int)(key >> 5); pv0 = v; }
+            else if (pk1 < 0) { pk1 = (int)(key >> 5); pv1 = v; }
+            else more = true;
+          }
+        }
+      }
+      if (!mbar_wait(&bar_empty[b], ((i / kSlots) & 1) ^ 1, abrt)) break;
       tc_fence_after();
-      const uint32_t acol = lane_base + kAColBase + b * 32 * TERMS;
-      const int kst = (st0 + i) * kStageK;
+      const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS;
       if (MODE == HXQ_MODE_SCALAR8) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -267,14 +418,22 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const uint32_t a = prmt(wd[j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
-            v[j] = *reinterpret_cast<const uint32_t*>(tb8 + a);
+            v[j] = *reinterpret_cast<const uint32_t*>(smem + a);
           }
-          const int k0 = kst + c * 16;
-          while (pk < k0 + 16) {
-            const float pv = L.patch_v[p];
-            patch16(v, pk - k0, TERMS == 1 ? (bf16_bits(pv) << 16) : split_word(pv));
-            ++p;
-            pk = p < pend ? L.patch_k[p] : INT_MAX;
+          const int k0 = c * 16;
+          if ((unsigned)(pk0 - k0) < 16u)
+            patch16(v, pk0 - k0, TERMS == 1 ? (bf16_bits(pv0) << 16) : split_word(pv0));
+          if ((unsigned)(pk1 - k0) < 16u)
+            patch16(v, pk1 - k0, TERMS == 1 ? (bf16_bits(pv1) << 16) : split_word(pv1));
+          if (more) {  // rare: a third entry in this row and stage, or > 32 in the bucket
+            for (int j = 0; j < bc; ++j) {
+              const uint32_t key = __ldg(L.pkey + bs + j);
+              const int o = (int)(key >> 5) - k0;
+              if ((int)(key & 31) == lane && (unsigned)o < 16u) {
+                const float pv = __ldg(L.pval + bs + j);
+                patch16(v, o, TERMS == 1 ? (bf16_bits(pv) << 16) : split_word(pv));
+              }
+            }
           }
           uint32_t hi[8];
 #pragma unroll
@@ -288,30 +447,29 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
           }
         }
       } else {
-        uint32_t w[13];
+        uint32_t wd[13];
 #pragma unroll
         for (int c = 0; c < 3; ++c) {
-          w[4 * c] = qc[c].x; w[4 * c + 1] = qc[c].y; w[4 * c + 2] = qc[c].z; w[4 * c + 3] = qc[c].w;
+          wd[4 * c] = qc[c].x; wd[4 * c + 1] = qc[c].y; wd[4 * c + 2] = qc[c].z; wd[4 * c + 3] = qc[c].w;
         }
-        w[12] = 0;
+        wd[12] = 0;
 #pragma unroll
         for (int h = 0; h < 4; ++h) {  // 8 pairs = 16 weights per step
           uint32_t hi[8], mid[8];
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
             const int j = h * 8 + jj, bit = 12 * j;
-            const uint32_t e = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & 0xFFF;
+            const uint32_t e = __funnelshift_r(wd[bit >> 5], wd[(bit >> 5) + 1], bit & 31) & 0xFFF;
             if (TERMS == 1) {
-              hi[jj] = reinterpret_cast<const uint32_t*>(table)[e];
+              hi[jj] = *reinterpret_cast<const uint32_t*>(smem + e * 4);
             } else {
-              const uint2 hm = reinterpret_cast<const uint2*>(table)[e];
+              const uint2 hm = *reinterpret_cast<const uint2*>(smem + e * 8);
               hi[jj] = hm.x;
               mid[jj] = hm.y;
             }
           }
-          const int k0 = kst + h * 16;
-          while (pk < k0 + 16) {
-            const float pv = L.patch_v[p];
+          const int k0 = h * 16;
+          auto apply = [&](int pk, float pv) {
             const int o = pk - k0;
             if (TERMS == 1) {
               patch8_half(hi, o >> 1, o & 1, bf16_bits(pv));
@@ -320,8 +478,15 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
               patch8_half(hi, o >> 1, o & 1, sw >> 16);
               patch8_half(mid, o >> 1, o & 1, sw & 0xFFFFu);
             }
-            ++p;
-            pk = p < pend ? L.patch_k[p] : INT_MAX;
+          };
+          if ((unsigned)(pk0 - k0) < 16u) apply(pk0, pv0);
+          if ((unsigned)(pk1 - k0) < 16u) apply(pk1, pv1);
+          if (more) {
+            for (int j = 0; j < bc; ++j) {
+              const uint32_t key = __ldg(L.pkey + bs + j);
+              if ((int)(key & 31) == lane && (unsigned)((int)(key >> 5) - k0) < 16u)
+                apply((int)(key >> 5), __ldg(L.pval + bs + j));
+            }
           }
           tmem_st8(acol + h * 8, hi);
           if (TERMS == 2) tmem_st8(acol + 32 + h * 8, mid);
@@ -331,26 +496,10 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_a[b]);
-    }
-
-    // ---------------- epilogue: D (y^T tile) from TMEM to y / workspace
-    if (!*abrt && mbar_wait(&bar_acc, 0, abrt)) {
-      tc_fence_after();
-      for (int cc = dg * 16; cc < BN; cc += kDecodeGroups * 16) {
-        uint32_t v[16];
-        tmem_ld16(lane_base + cc, v);
-        tmem_wait_ld();
-        if (valid) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int tok = tb * BN + cc + j;
-            if (tok < M) {
-              if (S == 1) y[(size_t)tok * L.N + n] = __uint_as_float(v[j]);
-              else work[((size_t)s * M + tok) * L.N + n] = __uint_as_float(v[j]);
-            }
-          }
-        }
-      }
+      for (int c = 0; c < NPC; ++c) qc[c] = qn[c];
+      cbs = nbs;
+      cbc = nbc;
     }
   }
 
@@ -361,28 +510,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (*abrt) {
-    if (threadIdx.x == 0) atomicOr(status, kStatusWaitTimeout);
-    return;
-  }
-  if (S == 1) return;
-  __threadfence();
-  __syncthreads();
-  int* ctr = counters + t * 64 + tb;
-  if (threadIdx.x == 0) last_sh = atomicAdd(ctr, 1) == S - 1;
-  __syncthreads();
-  if (!last_sh) return;
-  __threadfence();
-  const int ntok = min(BN, M - tb * BN);
-  for (int i = threadIdx.x; i < ntok * rows; i += blockDim.x) {
-    const int j = i / rows, rr = i % rows;
-    const int tok = tb * BN + j;
-    const size_t nn = (size_t)t * kTileRows + rr;
-    float v = 0.f;
-    for (int ss = 0; ss < S; ++ss) v += __ldcg(work + ((size_t)ss * M + tok) * L.N + nn);
-    y[(size_t)tok * L.N + nn] = v;
-  }
-  if (threadIdx.x == 0) *ctr = 0;
+  if (*abrt && threadIdx.x == 0) atomicOr(status, kStatusWaitTimeout);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -398,7 +526,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int BN, int TERMS, int MODE>
-cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int S, cudaStream_t st) {
+cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid_req, cudaStream_t st) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tm;
@@ -412,59 +540,54 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
   // at least 116 KB of shared memory keeps one CTA per SM (each CTA takes all
   // 512 TMEM columns)
+  static_assert(tc_smem_bytes<BN, TERMS, MODE>() <= 227 * 1024, "shared memory budget");
   const size_t smem = std::max<size_t>(tc_smem_bytes<BN, TERMS, MODE>(), 116 * 1024);
   auto kern = tc_kernel<BN, TERMS, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int n_tb = (M + BN - 1) / BN;
-  const int64_t units = (int64_t)h.L.n_tiles * n_tb * S;
-  kern<<<(unsigned)units, kTcThreads, smem, st>>>(tm, h.L, y, M, S, h.d_work, h.d_counters, h.d_status);
-  return cudaGetLastError();
+  const int n_tb_all = (M + BN - 1) / BN;
+  const int n_st = n_stages(h.L);
+  for (int tb0 = 0; tb0 < n_tb_all; tb0 += kMaxTokBlocks) {
+    const int n_tb = std::min(kMaxTokBlocks, n_tb_all - tb0);
+    const int64_t U = (int64_t)n_tb * h.L.n_tiles;  // (token block, tile) pairs
+    const int64_t W = U * n_st;
+    // one CTA per SM, but no tile's K shared by more than kMaxContrib CTAs
+    int64_t grid = grid_req > 0 ? grid_req : std::min<int64_t>(h.num_sms, U * kMaxContrib);
+    grid = std::max<int64_t>(1, std::min<int64_t>({grid, (int64_t)h.num_sms, W}));
+    if (W * grid >= INT_MAX) return cudaErrorInvalidValue;  // item arithmetic is 32-bit
+    if ((size_t)grid * 2 * BN * kTileRows > h.work_floats) return cudaErrorInvalidValue;
+    e = launch_pdl(kern, (unsigned)grid, tc_threads<TERMS>(), smem, st, tm, h.L, y, M, tb0 * BN, n_tb, h.d_work,
+                   h.d_counters, h.d_status);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <int MODE>
-cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M, int S, cudaStream_t st) {
-  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, y, M, S, st);
-  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, y, M, S, st);
-  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, y, M, S, st);
-  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, y, M, S, st);
-  return launch_cfg<256, 1, MODE>(h, x, y, M, S, st);
+cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t st) {
+  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, y, M, grid, st);
+  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, y, M, grid, st);
+  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, y, M, grid, st);
+  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, y, M, grid, st);
+  return launch_cfg<256, 1, MODE>(h, x, y, M, grid, st);
 }
-
-int tc_bn(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
 }  // namespace
 
-int choose_split_tc(const hxq_linear& h, int M) {
-  const int n_stages = h.L.Kp / kStageK;
-  const int n_tb = (M + tc_bn(M) - 1) / tc_bn(M);
-  if (n_tb > 64) return 1;  // split-K counters cover 64 token blocks per tile
-  const int slots = h.num_sms;
-  int best = 1;
-  double best_score = -1.0;
-  for (int S = 1; S <= std::min(n_stages, kMaxSplitK); ++S) {
-    if (S > 1 && (size_t)S * M * h.L.N > h.work_floats) break;
-    const int64_t units = (int64_t)h.L.n_tiles * n_tb * S;
-    const int64_t waves = (units + slots - 1) / slots;
-    const double wave_eff = (double)units / ((double)waves * slots);
-    const double per_unit = (double)n_stages / S;
-    const double pipe_eff = std::min(1.0, per_unit / (2.0 * kStages));
-    const double score = wave_eff * pipe_eff / (1.0 + 0.002 * S);
-    if (score > best_score + 1e-9) {
-      best_score = score;
-      best = S;
-    }
-  }
-  return best;
-}
+size_t tc_workspace_floats(int num_sms) { return (size_t)num_sms * 2 * 256 * kTileRows; }
 
+// `split` (when non-zero) sets the persistent grid so that each tile's K is
+// shared by about `split` CTAs; 0 = one CTA per SM.
 cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, float* y, int M, int split, cudaStream_t st) {
-  const int n_stages = h.L.Kp / kStageK;
-  const int S = std::max(1, std::min(split, n_stages));
-  const int n_tb = (M + tc_bn(M) - 1) / tc_bn(M);
-  if (S > 1 && ((size_t)S * M * h.L.N > h.work_floats || n_tb > 64)) return cudaErrorInvalidValue;
-  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, S, st);
-  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, S, st);
+  int grid = 0;
+  if (split > 0) {
+    const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    const int n_tb = std::min(kMaxTokBlocks, (M + bn - 1) / bn);
+    grid = std::max(1, n_tb * h.L.n_tiles * split);
+    grid = std::min(grid, n_tb * h.L.n_tiles * kMaxContrib * 4);
+  }
+  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, grid, st);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, grid, st);
 }
 
 }  // namespace hxq
