@@ -41,7 +41,7 @@ __global__ void relayout_kernel(Layer L, const uint8_t* __restrict__ src, uint8_
 }
 
 // delta[i] = v_i - (the codebook value the sidecar entry replaces), fp32.
-// `pos` holds the flat positions in bucket order.
+// `pos` holds the flat positions in patch-list order.
 __global__ void sidecar_delta_kernel(Layer L, const int64_t* __restrict__ pos, int64_t n,
                                      float* __restrict__ delta) {
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -60,7 +60,7 @@ __global__ void sidecar_delta_kernel(Layer L, const int64_t* __restrict__ pos, i
     const uint32_t e = ((lo | (hi << 8)) >> (bit & 7)) & 0xFFF;
     c = L.codebook[2 * e + (k & 1)];
   }
-  delta[i] = L.pval[i] - c;
+  delta[i] = L.pv[i] - c;
 }
 
 int cuda_status(cudaError_t e) {
@@ -73,10 +73,10 @@ void free_handle(hxq_linear* h) {
   if (!h) return;
   cudaFree(h->d_codebook);
   cudaFree(h->d_idx);
-  cudaFree(h->d_bptr);
-  cudaFree(h->d_pkey);
-  cudaFree(h->d_pval);
-  cudaFree(h->d_pdelta);
+  cudaFree(h->d_row_ptr);
+  cudaFree(h->d_pk);
+  cudaFree(h->d_pv);
+  cudaFree(h->d_pd);
   cudaFree(h->d_work);
   cudaFree(h->d_counters);
   cudaFree(h->d_status);
@@ -128,7 +128,7 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return HXQ_ECUDA;
   if (prop.major != 10 || prop.minor != 0) return HXQ_EUNSUPPORTED;
 
-  // ---- sidecar: copy to the host, check it, bucket it by (tile, stage, quadrant)
+  // ---- sidecar: copy to the host, check it, sort it into per-row patch lists
   std::vector<int64_t> pos((size_t)n_sidecar);
   std::vector<float> val((size_t)n_sidecar);
   if (n_sidecar > 0) {
@@ -162,29 +162,18 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
 
-  const int nst = hxq::n_stages(L);
-  const int64_t n_buckets = (int64_t)L.n_tiles * nst * hxq::kQuads;
-  std::vector<int> bptr((size_t)n_buckets + 1, 0);
-  std::vector<int> bucket((size_t)n_sidecar);
+  // position order = row-major order: rows, then ascending columns
+  std::vector<int> row_ptr((size_t)N + 1, 0), pk((size_t)n_sidecar);
+  std::vector<float> pv((size_t)n_sidecar);
+  std::vector<int64_t> ppos((size_t)n_sidecar);
   for (int64_t i = 0; i < n_sidecar; ++i) {
     const int64_t p = pos[order[i]];
-    const int row = (int)(p / K), k = (int)(p % K);
-    bucket[i] = hxq::bucket_of(L, row / hxq::kTileRows, k / hxq::kStageK, (row % hxq::kTileRows) / 32);
-    bptr[(size_t)bucket[i] + 1]++;
+    row_ptr[(size_t)(p / K) + 1]++;
+    pk[i] = (int)(p % K);
+    pv[i] = val[order[i]];
+    ppos[i] = p;
   }
-  for (int64_t b = 0; b < n_buckets; ++b) bptr[b + 1] += bptr[b];
-  std::vector<int> fill(bptr.begin(), bptr.end() - 1);
-  std::vector<uint32_t> pkey((size_t)n_sidecar);
-  std::vector<float> pval((size_t)n_sidecar);
-  std::vector<int64_t> bpos((size_t)n_sidecar);
-  for (int64_t i = 0; i < n_sidecar; ++i) {   // stable: position order inside a bucket
-    const int64_t p = pos[order[i]];
-    const int row = (int)(p / K), k = (int)(p % K);
-    const int j = fill[bucket[i]]++;
-    pkey[j] = hxq::patch_key(row % 32, k % hxq::kStageK);
-    pval[j] = val[order[i]];
-    bpos[j] = p;
-  }
+  for (int n = 0; n < N; ++n) row_ptr[n + 1] += row_ptr[n];
 
   const size_t cb_floats = mode == HXQ_MODE_SCALAR8 ? 256 : 8192;
   const size_t idx_bytes = (size_t)N * L.KC * 16 * L.P;
@@ -200,10 +189,10 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   int64_t* d_bpos = nullptr;
   if ((e = dalloc(&h->d_codebook, cb_floats)) != cudaSuccess ||
       (e = dalloc(&h->d_idx, idx_bytes)) != cudaSuccess ||
-      (e = dalloc(&h->d_bptr, (size_t)n_buckets + 1)) != cudaSuccess ||
-      (e = dalloc(&h->d_pkey, (size_t)n_sidecar)) != cudaSuccess ||
-      (e = dalloc(&h->d_pval, (size_t)n_sidecar)) != cudaSuccess ||
-      (e = dalloc(&h->d_pdelta, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&h->d_row_ptr, (size_t)N + 1)) != cudaSuccess ||
+      (e = dalloc(&h->d_pk, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&h->d_pv, (size_t)n_sidecar)) != cudaSuccess ||
+      (e = dalloc(&h->d_pd, (size_t)n_sidecar)) != cudaSuccess ||
       (e = dalloc(&d_bpos, (size_t)n_sidecar)) != cudaSuccess ||
       (e = dalloc(&h->d_work, h->work_floats)) != cudaSuccess ||
       (e = dalloc(&h->d_counters, (size_t)h->n_counters)) != cudaSuccess ||
@@ -217,20 +206,19 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   }
   L.codebook = h->d_codebook;
   L.idx = h->d_idx;
-  L.bptr = h->d_bptr;
-  L.pkey = h->d_pkey;
-  L.pval = h->d_pval;
-  L.pdelta = h->d_pdelta;
+  L.row_ptr = h->d_row_ptr;
+  L.pk = h->d_pk;
+  L.pv = h->d_pv;
+  L.pd = h->d_pd;
 
   if ((e = cudaMemcpy(h->d_codebook, codebook, cb_floats * sizeof(float), cudaMemcpyDefault)) != cudaSuccess ||
       (e = cudaMemcpy(d_src, indices, src_bytes, cudaMemcpyDefault)) != cudaSuccess ||
-      (e = cudaMemcpy(h->d_bptr, bptr.data(), bptr.size() * sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess ||
+      (e = cudaMemcpy(h->d_row_ptr, row_ptr.data(), row_ptr.size() * sizeof(int), cudaMemcpyHostToDevice)) !=
+          cudaSuccess ||
       (n_sidecar > 0 &&
-       ((e = cudaMemcpy(h->d_pkey, pkey.data(), n_sidecar * sizeof(uint32_t), cudaMemcpyHostToDevice)) !=
-            cudaSuccess ||
-        (e = cudaMemcpy(h->d_pval, pval.data(), n_sidecar * sizeof(float), cudaMemcpyHostToDevice)) !=
-            cudaSuccess ||
-        (e = cudaMemcpy(d_bpos, bpos.data(), n_sidecar * sizeof(int64_t), cudaMemcpyHostToDevice)) !=
+       ((e = cudaMemcpy(h->d_pk, pk.data(), n_sidecar * sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess ||
+        (e = cudaMemcpy(h->d_pv, pv.data(), n_sidecar * sizeof(float), cudaMemcpyHostToDevice)) != cudaSuccess ||
+        (e = cudaMemcpy(d_bpos, ppos.data(), n_sidecar * sizeof(int64_t), cudaMemcpyHostToDevice)) !=
             cudaSuccess)) ||
       (e = cudaMemset(h->d_counters, 0, h->n_counters * sizeof(int))) != cudaSuccess ||
       (e = cudaMemset(h->d_status, 0, sizeof(int))) != cudaSuccess) {
@@ -244,7 +232,7 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   relayout_kernel<<<(unsigned)((n_pieces + 255) / 256), 256>>>(L, d_src, h->d_idx, n_pieces);
   e = cudaGetLastError();
   if (e == cudaSuccess && n_sidecar > 0) {
-    sidecar_delta_kernel<<<(unsigned)((n_sidecar + 255) / 256), 256>>>(L, d_bpos, n_sidecar, h->d_pdelta);
+    sidecar_delta_kernel<<<(unsigned)((n_sidecar + 255) / 256), 256>>>(L, d_bpos, n_sidecar, h->d_pd);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();

@@ -27,16 +27,10 @@ __global__ void __launch_bounds__(256) decode_scalar_kernel(Layer L, float* __re
 #pragma unroll
   for (int j = 0; j < 16; ++j) v[j] = __ldg(L.codebook + ((w[j >> 2] >> (8 * (j & 3))) & 0xFF));
   const int k0 = c * 16;
-  {  // sidecar entries of this row in this chunk, from the (tile, stage, quadrant) bucket
-    const int b = bucket_of(L, t, k0 / kStageK, r / 32);
-    for (int p = L.bptr[b]; p < L.bptr[b + 1]; ++p) {
-      const uint32_t key = L.pkey[p];
-      const int j = (int)(key >> 5) - (k0 % kStageK);
-      if ((int)(key & 31) == (r & 31) && j >= 0 && j < 16) {
+  // sidecar entries of this row in this chunk (patch list sorted by column)
+  for (int p = row_lower_bound(L, n, k0); p < L.row_ptr[n + 1] && L.pk[p] < k0 + 16; ++p) {
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) v[jj] = sel_eq(jj, j, L.pval[p], v[jj]);
-      }
-    }
+    for (int jj = 0; jj < 16; ++jj) v[jj] = sel_eq(jj, L.pk[p] - k0, L.pv[p], v[jj]);
   }
   float* out = W + (int64_t)n * L.K + k0;
   const int cnt = min(16, L.K - k0);
@@ -66,18 +60,15 @@ __global__ void __launch_bounds__(256) decode_vq2d_kernel(Layer L, float* __rest
   const int k0 = c * 64;
   float* out = W + (int64_t)n * L.K + k0;
   const int cnt = min(64, L.K - k0);
-  const int b = bucket_of(L, t, c, r / 32);
-  const int pb = L.bptr[b], pe = L.bptr[b + 1];
+  int p = row_lower_bound(L, n, k0);
+  const int pe = L.row_ptr[n + 1];
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const int bit = 12 * j;
     const uint32_t e = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & 0xFFF;
     float2 v = __ldg(cb2 + e);
-    for (int p = pb; p < pe; ++p) {
-      const uint32_t key = L.pkey[p];
-      if ((int)(key & 31) != (r & 31)) continue;
-      if ((int)(key >> 5) == 2 * j) v.x = L.pval[p];
-      if ((int)(key >> 5) == 2 * j + 1) v.y = L.pval[p];
+    for (; p < pe && L.pk[p] < k0 + 2 * j + 2; ++p) {
+      if (L.pk[p] == k0 + 2 * j) v.x = L.pv[p]; else v.y = L.pv[p];
     }
     if (2 * j + 1 < cnt) {
       *reinterpret_cast<float2*>(out + 2 * j) = v;

@@ -32,10 +32,9 @@
 // Sidecar (replacement of single weights, HXQ whitepaper, method section,
 // "Sidecar outlier correction"): replacing w = c by v adds (v - c) x to the
 // dot product, so each entry carries delta = v - c (fp32, computed once when
-// the handle is built) and is applied as one extra multiply-add at the end of
-// its stage. A warp's entries for a stage (bucket of its 32 rows x 64
-// columns) are loaded one stage ahead, one entry per lane, and handed to the
-// owning lane with shuffles: no dependent memory access on the hot path.
+// the handle is built). The main loop decodes with the codebook alone; at the
+// end of each tile segment, the row's patch list (bounds loaded when the
+// segment starts) adds delta * x[k] for the entries in the segment's columns.
 #include <algorithm>
 #include <climits>
 
@@ -69,11 +68,9 @@ __device__ __forceinline__ int cta_of(int w, int W, int G) {
   return b;
 }
 
-// Load the NP 16-byte index pieces of stage `st` of row r in tile t, and the
-// bounds of the sidecar bucket of this warp's 32 rows for that stage.
+// Load the NP 16-byte index pieces of stage `st` of row r in tile t.
 template <int NP>
-__device__ __forceinline__ void load_stage(const Layer& L, int t, int st, int r, uint4 (&q)[NP], int& bs,
-                                           int& bc) {
+__device__ __forceinline__ void load_stage(const Layer& L, int t, int st, int r, uint4 (&q)[NP]) {
   const int rows = min(kTileRows, L.N - t * kTileRows);
   if (r < rows) {
     const uint8_t* p = L.idx + (size_t)t * kTileRows * L.KC * 16 * L.P + ((size_t)st * NP) * rows * 16 + r * 16;
@@ -83,9 +80,6 @@ __device__ __forceinline__ void load_stage(const Layer& L, int t, int st, int r,
 #pragma unroll
     for (int j = 0; j < NP; ++j) q[j] = make_uint4(0, 0, 0, 0);
   }
-  const int b = bucket_of(L, t, st, r >> 5);
-  bs = __ldg(L.bptr + b);
-  bc = __ldg(L.bptr + b + 1) - bs;
 }
 
 // 16 activations x[m][k0 .. k0+16) from shared memory as fp32.
@@ -174,35 +168,58 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
     for (size_t o = a; o < b; o += 65536) prefetch_l2_bulk(L.idx + o, (uint32_t)min((size_t)65536, b - o));
   }
   uint4 cur[NP];
-  int cbs = 0, cbc = 0;
   int nt = (w0 + g) / n_st, nst = (w0 + g) % n_st;  // next item to load
-  if (w0 + g < w1) load_stage<NP>(L, nt, nst, r, cur, cbs, cbc);
+  if (w0 + g < w1) load_stage<NP>(L, nt, nst, r, cur);
 
   // 2. shared-memory codebook; activations once the previous kernel is done
+  // (compile-time trip counts: all of a thread's codebook loads are in
+  // flight together)
   if (MODE == HXQ_MODE_SCALAR8) {
+    constexpr int PER = 256 * 32 / kGemvThreads;
+    float cv[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) cv[j] = __ldg(L.codebook + ((threadIdx.x + j * kGemvThreads) >> 5));
     float* tw = reinterpret_cast<float*>(smem);
-    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) tw[(i >> 5) * 64 + (i & 31)] = __ldg(L.codebook + (i >> 5));
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int i = threadIdx.x + j * kGemvThreads;
+      tw[(i >> 5) * 64 + (i & 31)] = cv[j];
+    }
   } else {
+    constexpr int PER = 2048 / kGemvThreads;
     const float4* cb = reinterpret_cast<const float4*>(L.codebook);
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) reinterpret_cast<float4*>(smem)[i] = __ldg(cb + i);
-  }
-  uint32_t ek = 0;  // sidecar entries (key, delta) of the current item, one per lane
-  float ed = 0.f;
-  if (lane < cbc) {
-    ek = __ldg(L.pkey + cbs + lane);
-    ed = __ldg(L.pdelta + cbs + lane);
+    float4 cv[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) cv[j] = __ldg(cb + threadIdx.x + j * kGemvThreads);
+#pragma unroll
+    for (int j = 0; j < PER; ++j) reinterpret_cast<float4*>(smem)[threadIdx.x + j * kGemvThreads] = cv[j];
   }
   pdl_wait();
-  for (int i = threadIdx.x; i < MT * (L.Kp / 8); i += blockDim.x) {
-    const int m = i / (L.Kp / 8), k = (i % (L.Kp / 8)) * 8;
-    uint4 q = make_uint4(0, 0, 0, 0);
-    if (m < M && k < L.K) q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)m * L.K + k));
-    if (XF32) {
-      float4* d = reinterpret_cast<float4*>(xs + ((size_t)m * L.Kp + k) * 4);
-      d[0] = make_float4(bf16lo(q.x), bf16hi(q.x), bf16lo(q.y), bf16hi(q.y));
-      d[1] = make_float4(bf16lo(q.z), bf16hi(q.z), bf16lo(q.w), bf16hi(q.w));
-    } else {
-      *reinterpret_cast<uint4*>(xs + ((size_t)m * L.Kp + k) * 2) = q;
+  {
+    constexpr int XU = 4;  // activation loads in flight per thread
+    const int n8 = MT * (L.Kp / 8);
+    for (int i0 = threadIdx.x; i0 < n8; i0 += XU * kGemvThreads) {
+      uint4 q[XU];
+#pragma unroll
+      for (int u = 0; u < XU; ++u) {
+        const int i = i0 + u * kGemvThreads;
+        const int m = i / (L.Kp / 8), k = (i % (L.Kp / 8)) * 8;
+        q[u] = make_uint4(0, 0, 0, 0);
+        if (i < n8 && m < M && k < L.K) q[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)m * L.K + k));
+      }
+#pragma unroll
+      for (int u = 0; u < XU; ++u) {
+        const int i = i0 + u * kGemvThreads;
+        if (i >= n8) break;
+        const int m = i / (L.Kp / 8), k = (i % (L.Kp / 8)) * 8;
+        if (XF32) {
+          float4* d = reinterpret_cast<float4*>(xs + ((size_t)m * L.Kp + k) * 4);
+          d[0] = make_float4(bf16lo(q[u].x), bf16hi(q[u].x), bf16lo(q[u].y), bf16hi(q[u].y));
+          d[1] = make_float4(bf16lo(q[u].z), bf16hi(q[u].z), bf16lo(q[u].w), bf16hi(q[u].w));
+        } else {
+          *reinterpret_cast<uint4*>(xs + ((size_t)m * L.Kp + k) * 2) = q[u];
+        }
+      }
     }
   }
   __syncthreads();
@@ -214,6 +231,13 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   for (int seg0 = w0; seg0 < w1;) {  // segments: the CTA's items of one tile
     const int t = seg0 / n_st;
     const int seg1 = min(w1, (t + 1) * n_st);
+    // group 0 adds the sidecar corrections of row n; its list bounds load now
+    const int n = t * kTileRows + r;
+    int pr0 = 0, pr1 = 0;
+    if (g == 0 && n < L.N) {
+      pr0 = __ldg(L.row_ptr + n);
+      pr1 = __ldg(L.row_ptr + n + 1);
+    }
     float2 acc[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.f, 0.f);
@@ -222,8 +246,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
     for (int w = seg0 + ((w0 + g - seg0) % kGroups + kGroups) % kGroups; w < seg1; w += kGroups) {
       // next item's loads go out first; they land while this item computes
       uint4 nxt[NP];
-      int nbs = 0, nbc = 0;
-      if (w + kGroups < w1) load_stage<NP>(L, nt, nst, r, nxt, nbs, nbc);
+      if (w + kGroups < w1) load_stage<NP>(L, nt, nst, r, nxt);
       nst += kGroups;
       while (nst >= n_st) { nst -= n_st; ++nt; }
 
@@ -263,29 +286,18 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
           accumulate16<MT, XF32>(acc, wv, xs, L.Kp, kst + h * 16);
         }
       }
-      // sidecar corrections of this item: acc += delta * x[k]
-      const int nb = min(cbc, 32);
-      for (int j = 0; j < nb; ++j) {
-        const uint32_t key = __shfl_sync(0xffffffffu, ek, j);
-        const float dv = __shfl_sync(0xffffffffu, ed, j);
-        if ((int)(key & 31) == lane) add_patch<MT, XF32>(acc, dv, xs, L.Kp, kst + (int)(key >> 5));
-      }
-      for (int j = 32; j < cbc; ++j) {  // more than 32 entries in one bucket: direct loads
-        const uint32_t key = __ldg(L.pkey + cbs + j);
-        if ((int)(key & 31) == lane)
-          add_patch<MT, XF32>(acc, __ldg(L.pdelta + cbs + j), xs, L.Kp, kst + (int)(key >> 5));
-      }
-      // advance: next item's sidecar entries, then its index pieces
-      ek = 0;
-      ed = 0.f;
-      if (lane < nbc) {
-        ek = __ldg(L.pkey + nbs + lane);
-        ed = __ldg(L.pdelta + nbs + lane);
-      }
 #pragma unroll
       for (int j = 0; j < NP; ++j) cur[j] = nxt[j];
-      cbs = nbs;
-      cbc = nbc;
+    }
+
+    // sidecar corrections of this segment's columns: acc += delta * x[k]
+    if (pr1 > pr0) {
+      const int ka = (seg0 - t * n_st) * kStageK, kb = (seg1 - t * n_st) * kStageK;
+#pragma unroll 1
+      for (int p = pr0; p < pr1; ++p) {
+        const int k = __ldg(L.pk + p);
+        if (k >= ka && k < kb) add_patch<MT, XF32>(acc, __ldg(L.pd + p), xs, L.Kp, k);
+      }
     }
 
     // segment end: the 4 groups' sums meet in shared memory

@@ -41,25 +41,17 @@ struct Layer {
   int n_tiles;       // ceil(N / 128)
   const float* codebook;     // 256 or 4096*2 floats
   const uint8_t* idx;        // tiled layout above
-  // Sidecar, bucketed by (tile t, stage st, warp quadrant q = row / 32):
-  // bucket b = (t * n_stages + st) * 4 + q holds entries [bptr[b], bptr[b+1])
-  // of the position-sorted sidecar that fall in rows 32q .. 32q+31 of tile t
-  // and columns 64 st .. 64 st + 63. A warp loads its bucket for the next
-  // stage together with that stage's indices, so applying the sidecar costs
-  // no dependent memory round trip.
-  const int* bptr;           // [n_tiles * n_stages * 4 + 1]
-  const uint32_t* pkey;      // lane (bits 0-4) | column within the stage (bits 5-10)
-  const float* pval;         // the replacement value v
-  const float* pdelta;       // v - (codebook value it replaces), rounded to fp32
+  // Sidecar as per-row patch lists: the entries of row n are
+  // [row_ptr[n], row_ptr[n+1]), in ascending column order.
+  const int* row_ptr;        // [N+1]
+  const int* pk;             // column k
+  const float* pv;           // the replacement value v
+  const float* pd;           // v - (codebook value it replaces), rounded to fp32
 };
 
 constexpr int kQuads = kTileRows / 32;
 
 __host__ __device__ inline int n_stages(const Layer& L) { return L.Kp / kStageK; }
-__host__ __device__ inline int bucket_of(const Layer& L, int t, int st, int q) {
-  return (t * n_stages(L) + st) * kQuads + q;
-}
-__host__ __device__ inline uint32_t patch_key(int lane, int kk) { return (uint32_t)lane | ((uint32_t)kk << 5); }
 
 __host__ __device__ inline size_t piece_offset(const Layer& L, int t, int c, int p, int r) {
   const int rows = min(kTileRows, L.N - t * kTileRows);
@@ -75,10 +67,10 @@ struct hxq_linear {
   int num_sms;
   float* d_codebook;
   uint8_t* d_idx;
-  int* d_bptr;
-  uint32_t* d_pkey;
-  float* d_pval;
-  float* d_pdelta;
+  int* d_row_ptr;
+  int* d_pk;
+  float* d_pv;
+  float* d_pd;
   float* d_work;        // split-K partial sums
   size_t work_floats;
   int* d_counters;      // per output tile: arrivals of split-K partials
@@ -260,6 +252,16 @@ __device__ __forceinline__ uint32_t sel_eq(int a, int b, uint32_t x, uint32_t y)
 }
 __device__ __forceinline__ float sel_eq(int a, int b, float x, float y) {
   return __uint_as_float(sel_eq(a, b, __float_as_uint(x), __float_as_uint(y)));
+}
+
+// First entry of row n's patch list with column >= k0 (binary search).
+__device__ __forceinline__ int row_lower_bound(const Layer& L, int n, int k0) {
+  int lo = L.row_ptr[n], hi = L.row_ptr[n + 1];
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(L.pk + mid) < k0) lo = mid + 1; else hi = mid;
+  }
+  return lo;
 }
 
 // Byte permute: result byte i = byte sel_i of the 8-byte value {b:a}.

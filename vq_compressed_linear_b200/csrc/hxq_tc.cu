@@ -37,9 +37,9 @@
 //    tolerance 1e-5 * sum |x||w| that applies to the decode GEMV.
 //
 // Sidecar (HXQ whitepaper, method section, "Sidecar outlier correction"):
-// the decoding warp loads its (tile, stage, 32-row) bucket one item ahead,
-// one entry per lane; shuffles hand each entry to its row's lane, which
-// substitutes the value (as bf16, or as its hi+mid split) before the store.
+// each decoding thread keeps a cursor into its row's column-sorted patch list
+// with the next entry already in registers, and substitutes the stored value
+// (as bf16, or as its hi+mid split) before the store.
 //
 // Every mbarrier wait is bounded (2 s): on timeout the CTA sets a status bit,
 // drains what it issued, frees TMEM and returns.
@@ -181,21 +181,40 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
     tmem_alloc(&tmem_base_sh, kTmemCols);
     tmem_relinquish();
   }
-  // shared-memory decode table
+  // shared-memory decode table (compile-time trip counts: a thread's
+  // codebook loads are all in flight together)
+  constexpr int NT = tc_threads<TERMS>();
   if (MODE == HXQ_MODE_SCALAR8) {
+    constexpr int PER = (256 * 32 + NT - 1) / NT;
+    float cv[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int i = threadIdx.x + j * NT;
+      cv[j] = i < 256 * 32 ? __ldg(L.codebook + (i >> 5)) : 0.f;
+    }
     uint32_t* tw = reinterpret_cast<uint32_t*>(smem);
-    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-      const float c = __ldg(L.codebook + (i >> 5));
-      tw[(i >> 5) * 64 + (i & 31)] = TERMS == 1 ? (bf16_bits(c) << 16) : split_word(c);
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int i = threadIdx.x + j * NT;
+      if (i < 256 * 32) tw[(i >> 5) * 64 + (i & 31)] = TERMS == 1 ? (bf16_bits(cv[j]) << 16) : split_word(cv[j]);
     }
   } else {
+    constexpr int PER = (4096 + NT - 1) / NT;
     const float2* cb2 = reinterpret_cast<const float2*>(L.codebook);
-    for (int i = threadIdx.x; i < 4096; i += blockDim.x) {
-      const float2 c = __ldg(cb2 + i);
+    float2 cv[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int i = threadIdx.x + j * NT;
+      cv[j] = i < 4096 ? __ldg(cb2 + i) : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int i = threadIdx.x + j * NT;
+      if (i >= 4096) break;
       if (TERMS == 1) {
-        reinterpret_cast<uint32_t*>(smem)[i] = bf16_bits(c.x) | (bf16_bits(c.y) << 16);
+        reinterpret_cast<uint32_t*>(smem)[i] = bf16_bits(cv[j].x) | (bf16_bits(cv[j].y) << 16);
       } else {
-        const uint32_t a = split_word(c.x), b = split_word(c.y);
+        const uint32_t a = split_word(cv[j].x), b = split_word(cv[j].y);
         reinterpret_cast<uint2*>(smem)[i] = make_uint2(prmt(a, b, 0x7632), prmt(a, b, 0x5410));
       }
     }
@@ -354,8 +373,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
     const uint32_t lane4 = (uint32_t)lane * 4u;
     constexpr int NPC = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per stage
 
-    // index pieces and sidecar bucket bounds of one item
-    auto load_item = [&](int i, uint4 (&qd)[NPC], int& bs, int& bc) {
+    // index pieces of one item
+    auto load_item = [&](int i, uint4 (&qd)[NPC]) {
       const int w = w0 + i;
       const int T = w / n_st, st = w % n_st, t = T % L.n_tiles;
       const int rows = min(kTileRows, L.N - t * kTileRows);
@@ -369,43 +388,36 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
           qd[c] = make_uint4(0, 0, 0, 0);
         }
       }
-      const int b = bucket_of(L, t, st, q);
-      bs = __ldg(L.bptr + b);
-      bc = __ldg(L.bptr + b + 1) - bs;
     };
     uint4 qc[NPC];
-    int cbs = 0, cbc = 0;
-    if (dg < n_items) load_item(dg, qc, cbs, cbc);
+    if (dg < n_items) load_item(dg, qc);
+    // Sidecar cursor over this row's patch list (ascending columns): the
+    // next entry's column and value are always already in registers, so an
+    // item without a patch costs one compare per 16 weights.
+    int cur_T = -1, pp = 0, pe = 0, pkn = INT_MAX;
+    float pvn = 0.f;
 
     for (int i = dg; i < n_items; i += kDecGroups) {
       const int b = i % kSlots;
+      const int w = w0 + i, T = w / n_st, st = w % n_st, t = T % L.n_tiles;
       // the group's next item loads first: they land while this one decodes
       uint4 qn[NPC];
-      int nbs = 0, nbc = 0;
-      if (i + kDecGroups < n_items) load_item(i + kDecGroups, qn, nbs, nbc);
-      const int bs = cbs, bc = cbc;
-      // this item's sidecar entries, one per lane
-      uint32_t ek = 0xFFFFFFFFu;
-      float ev = 0.f;
-      if (lane < bc) {
-        ek = __ldg(L.pkey + bs + lane);
-        ev = __ldg(L.pval + bs + lane);
-      }
-      // entries of this lane's row: up to two kept in registers, more -> rescan
-      int pk0 = -1, pk1 = -1;
-      float pv0 = 0.f, pv1 = 0.f;
-      bool more = bc > 32;
-      {
-        const int nb = min(bc, 32);
-        for (int j = 0; j < nb; ++j) {
-          const uint32_t key = __shfl_sync(0xffffffffu, ek, j);
-          const float v = __shfl_sync(0xffffffffu, ev, j);
-          if ((int)(key & 31) == lane) {
-            if (pk0 < 0) { pk0 = (int)(key >> 5); pv0 = v; }
-            else if (pk1 < 0) { pk1 = (int)(key >> 5); pv1 = v; }
-            else more = true;
-          }
+      if (i + kDecGroups < n_items) load_item(i + kDecGroups, qn);
+      const int kst = st * kStageK;
+      if (T != cur_T) {  // new tile: position the cursor at this stage
+        cur_T = T;
+        const int n = t * kTileRows + r;
+        pkn = INT_MAX;
+        if (n < L.N) {
+          pp = row_lower_bound(L, n, kst);
+          pe = L.row_ptr[n + 1];
+          if (pp < pe) { pkn = __ldg(L.pk + pp); pvn = __ldg(L.pv + pp); }
         }
+      }
+      while (pkn < kst) {  // entries in other groups' stages
+        ++pp;
+        pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
+        pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
       }
       if (!mbar_wait(&bar_empty[b], ((i / kSlots) & 1) ^ 1, abrt)) break;
       tc_fence_after();
@@ -420,20 +432,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
             const uint32_t a = prmt(wd[j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
             v[j] = *reinterpret_cast<const uint32_t*>(smem + a);
           }
-          const int k0 = c * 16;
-          if ((unsigned)(pk0 - k0) < 16u)
-            patch16(v, pk0 - k0, TERMS == 1 ? (bf16_bits(pv0) << 16) : split_word(pv0));
-          if ((unsigned)(pk1 - k0) < 16u)
-            patch16(v, pk1 - k0, TERMS == 1 ? (bf16_bits(pv1) << 16) : split_word(pv1));
-          if (more) {  // rare: a third entry in this row and stage, or > 32 in the bucket
-            for (int j = 0; j < bc; ++j) {
-              const uint32_t key = __ldg(L.pkey + bs + j);
-              const int o = (int)(key >> 5) - k0;
-              if ((int)(key & 31) == lane && (unsigned)o < 16u) {
-                const float pv = __ldg(L.pval + bs + j);
-                patch16(v, o, TERMS == 1 ? (bf16_bits(pv) << 16) : split_word(pv));
-              }
-            }
+          const int k0 = kst + c * 16;
+          while (pkn < k0 + 16) {  // sidecar: substitute the stored value
+            patch16(v, pkn - k0, TERMS == 1 ? (bf16_bits(pvn) << 16) : split_word(pvn));
+            ++pp;
+            pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
+            pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
           }
           uint32_t hi[8];
 #pragma unroll
@@ -468,25 +472,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
               mid[jj] = hm.y;
             }
           }
-          const int k0 = h * 16;
-          auto apply = [&](int pk, float pv) {
-            const int o = pk - k0;
+          const int k0 = kst + h * 16;
+          while (pkn < k0 + 16) {  // sidecar: substitute the stored value
+            const int o = pkn - k0;
             if (TERMS == 1) {
-              patch8_half(hi, o >> 1, o & 1, bf16_bits(pv));
+              patch8_half(hi, o >> 1, o & 1, bf16_bits(pvn));
             } else {
-              const uint32_t sw = split_word(pv);
+              const uint32_t sw = split_word(pvn);
               patch8_half(hi, o >> 1, o & 1, sw >> 16);
               patch8_half(mid, o >> 1, o & 1, sw & 0xFFFFu);
             }
-          };
-          if ((unsigned)(pk0 - k0) < 16u) apply(pk0, pv0);
-          if ((unsigned)(pk1 - k0) < 16u) apply(pk1, pv1);
-          if (more) {
-            for (int j = 0; j < bc; ++j) {
-              const uint32_t key = __ldg(L.pkey + bs + j);
-              if ((int)(key & 31) == lane && (unsigned)((int)(key >> 5) - k0) < 16u)
-                apply((int)(key >> 5), __ldg(L.pval + bs + j));
-            }
+            ++pp;
+            pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
+            pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
           }
           tmem_st8(acol + h * 8, hi);
           if (TERMS == 2) tmem_st8(acol + 32 + h * 8, mid);
@@ -498,8 +496,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
       if (lane == 0) mbar_arrive(&bar_a[b]);
 #pragma unroll
       for (int c = 0; c < NPC; ++c) qc[c] = qn[c];
-      cbs = nbs;
-      cbc = nbc;
     }
   }
 
