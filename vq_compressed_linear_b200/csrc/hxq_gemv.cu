@@ -1,22 +1,25 @@
 // Fused decode + GEMV on CUDA cores for few tokens (M <= 4 by default; up to
-// M = 32 on request): y[m][n] = sum_k x[m][k] * W[n][k] with W decoded on the
+// M = 16 on request): y[m][n] = sum_k x[m][k] * W[n][k] with W decoded on the
 // fly from the codebook and never written anywhere (the pages' buffered path
 // instead materialises W and calls cuBLAS: HXQ whitepaper, method section,
 // buffered forward path paragraph).
 //
 // Work decomposition (stream-K). The work items are the tile-stages of the
-// layer, (tile of 128 rows) x (64 weights along K), numbered tile-major. A
-// persistent grid of one 512-thread CTA per SM takes contiguous item ranges
-// of equal size, so every CTA streams the same number of index bytes
-// whatever the layer shape. Inside a CTA the 4 groups of 128 threads take
-// the items round-robin; thread r of a group owns row r of the item's tile
-// (a warp reads 512 contiguous bytes per 16-byte load) and keeps the next
-// items' loads in flight in a register ring while it decodes the current
-// one. At each tile boundary of the CTA's range the groups' sums meet in
-// shared memory; a tile covered by one CTA goes straight to y, a tile split
-// between CTAs leaves one fp32 partial per CTA in the workspace and the last
-// CTA to arrive (integer atomic per tile) adds them in CTA order: results
-// are bitwise repeatable.
+// layer, (tile of 128 rows) x (64 weights along K), numbered tile-major; an
+// item's indices are one contiguous block of the tiled layout. A persistent
+// grid of one CTA per SM takes contiguous item ranges of equal size, so every
+// CTA streams the same number of index bytes whatever the layer shape.
+//
+// Inside a CTA a producer warp streams the items' index blocks with TMA bulk
+// copies into a ring of shared-memory slots (up to 12 x 8 KB in flight per
+// SM; it starts before the previous kernel has finished, since the indices do
+// not depend on it), and 4 groups of 128 consumer threads take the items
+// round-robin: thread r of a group owns row r of the item's tile, reads its
+// 16-byte pieces from the slot, releases the slot and decodes. At each tile
+// boundary of the CTA's range the groups' sums meet in shared memory; a tile
+// covered by one CTA goes straight to y, a tile split between CTAs leaves one
+// fp32 partial per CTA in the workspace and the last CTA to arrive (integer
+// atomic per tile) adds them in CTA order: results are bitwise repeatable.
 //
 // Scalar codebook in shared memory: replicated once per lane with entry e of
 // lane l at byte e*256 + l*4, so the 32 lanes of a lookup always hit 32
@@ -32,9 +35,11 @@
 // Sidecar (replacement of single weights, HXQ whitepaper, method section,
 // "Sidecar outlier correction"): replacing w = c by v adds (v - c) x to the
 // dot product, so each entry carries delta = v - c (fp32, computed once when
-// the handle is built). The main loop decodes with the codebook alone; at the
-// end of each tile segment, the row's patch list (bounds loaded when the
-// segment starts) adds delta * x[k] for the entries in the segment's columns.
+// the handle is built). The main loop decodes with the codebook alone; each
+// group loads its share of the row's patch entries when a tile segment
+// starts (list bounds fetched one segment ahead) and adds delta * x[k] for
+// those in the segment's columns at its end -- no dependent memory access on
+// the critical path.
 #include <algorithm>
 #include <climits>
 
@@ -43,15 +48,28 @@
 namespace hxq {
 namespace {
 
-constexpr int kGemvThreads = 512;
-constexpr int kGroups = kGemvThreads / kTileRows;  // virtual CTAs per CTA
-constexpr size_t kSmemLimit = 227 * 1024;          // dynamic shared memory per CTA
+constexpr int kGemvThreads = 512;                  // consumers; one more warp produces
+constexpr int kGroups = kGemvThreads / kTileRows;  // consumer groups (128 rows each)
+constexpr int kMaxRing = 12;                       // index slots in flight per CTA
+constexpr size_t kSmemLimit = 226 * 1024;          // dynamic shared memory per CTA (static kept apart)
 
 // Dynamic shared memory of one CTA: codebook table, activations (fp32 or
-// bf16) and the groups' partial sums.
-inline size_t gemv_smem(int mode, int MT, int Kp, bool xf32) {
+// bf16) and the groups' partial sums, then the index ring.
+inline size_t gemv_smem_fixed(int mode, int MT, int Kp, bool xf32) {
   return (size_t)(mode == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8) + (size_t)MT * Kp * (xf32 ? 4 : 2) +
          (size_t)kGroups * MT * kTileRows * sizeof(float);
+}
+inline int slot_bytes(int mode) { return (mode == HXQ_MODE_SCALAR8 ? 4 : 3) * kTileRows * 16; }
+// Ring slots that fit next to the fixed part (a multiple of the groups; 0 if
+// fewer than one per group fit).
+inline int ring_slots(int mode, int MT, int Kp, bool xf32) {
+  const size_t fixed = gemv_smem_fixed(mode, MT, Kp, xf32);
+  if (fixed + 128 > kSmemLimit) return 0;
+  const int fit = (int)((kSmemLimit - fixed - 128) / slot_bytes(mode));
+  return std::min(kMaxRing, fit / kGroups * kGroups);
+}
+inline size_t gemv_smem(int mode, int MT, int Kp, bool xf32) {
+  return gemv_smem_fixed(mode, MT, Kp, xf32) + 128 + (size_t)ring_slots(mode, MT, Kp, xf32) * slot_bytes(mode);
 }
 
 template <int MODE>
@@ -66,20 +84,6 @@ __device__ __forceinline__ int cta_of(int w, int W, int G) {
   while (b + 1 < G && ((b + 1) * W) / G <= w) ++b;
   while (b > 0 && (b * W) / G > w) --b;
   return b;
-}
-
-// Load the NP 16-byte index pieces of stage `st` of row r in tile t.
-template <int NP>
-__device__ __forceinline__ void load_stage(const Layer& L, int t, int st, int r, uint4 (&q)[NP]) {
-  const int rows = min(kTileRows, L.N - t * kTileRows);
-  if (r < rows) {
-    const uint8_t* p = L.idx + (size_t)t * kTileRows * L.KC * 16 * L.P + ((size_t)st * NP) * rows * 16 + r * 16;
-#pragma unroll
-    for (int j = 0; j < NP; ++j) q[j] = ldg_stream16(p + (size_t)j * rows * 16);
-  } else {
-#pragma unroll
-    for (int j = 0; j < NP; ++j) q[j] = make_uint4(0, 0, 0, 0);
-  }
 }
 
 // 16 activations x[m][k0 .. k0+16) from shared memory as fp32.
@@ -130,50 +134,72 @@ __device__ __forceinline__ void add_patch(float2 (&acc)[MT], float d, const uint
   }
 }
 
-// Byte offset of the first index piece of item w (tile-major order, NP
-// pieces per row and stage); the items of any contiguous range occupy one
-// contiguous byte range. Item W (one past the last) maps to the end.
-template <int NP>
-__device__ __forceinline__ size_t item_offset(const Layer& L, int w, int n_st) {
-  const int t = w / n_st, st = w % n_st;
-  if (t >= L.n_tiles) return (size_t)L.N * L.KC * 16 * L.P;
-  const int rows = min(kTileRows, L.N - t * kTileRows);
-  return (size_t)t * kTileRows * L.KC * 16 * L.P + (size_t)st * NP * rows * 16;
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kGemvThreads) : "memory");
 }
 
 template <int MT, bool XF32, int MODE>
-__global__ void __launch_bounds__(kGemvThreads, 1)
-gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int W,
-            float* __restrict__ work, int* __restrict__ counters) {
+__global__ void __launch_bounds__(kGemvThreads + 32, 1)
+gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int W, int R,
+            float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int TB = table_bytes<MODE>();
-  constexpr int NP = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per stage
+  constexpr int NP = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per row and stage
   uint8_t* xs = smem + TB;
   // per-group partial sums [kGroups][MT][kTileRows], after the activations
   float* red = reinterpret_cast<float*>(xs + (size_t)MT * L.Kp * (XF32 ? 4 : 2));
-  __shared__ int last_flag;
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(red + kGroups * MT * kTileRows) + 127) & ~(uintptr_t)127);
+  constexpr int SLOT = NP * kTileRows * 16;
+  __shared__ uint64_t bar_full[kMaxRing], bar_empty[kMaxRing];
+  __shared__ int last_flag, abort_sh;
 
-  const int g = threadIdx.x >> 7, r = threadIdx.x & (kTileRows - 1), lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_st = n_stages(L);
   const int G = gridDim.x;
   const int w0 = (blockIdx.x * W) / G, w1 = ((blockIdx.x + 1) * W) / G;
+  volatile int* abrt = &abort_sh;
 
-  // 0. the next kernel in the stream may start its own prologue
-  pdl_launch_dependents();
-  // 1. stream this CTA's whole index range into L2 (TMA bulk prefetch), then
-  //    issue this thread's first item load; items of this thread are
-  //    w0 + g, w0 + g + 4, ...
-  if (threadIdx.x == 0 && w1 > w0) {
-    const size_t a = item_offset<NP>(L, w0, n_st), b = item_offset<NP>(L, w1, n_st);
-    for (size_t o = a; o < b; o += 65536) prefetch_l2_bulk(L.idx + o, (uint32_t)min((size_t)65536, b - o));
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < R; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_empty[i], 4);  // the 4 warps of the consuming group
+    }
+    abort_sh = 0;
+    fence_mbar_init();
   }
-  uint4 cur[NP];
-  int nt = (w0 + g) / n_st, nst = (w0 + g) % n_st;  // next item to load
-  if (w0 + g < w1) load_stage<NP>(L, nt, nst, r, cur);
+  __syncthreads();
+  pdl_launch_dependents();  // the next kernel in the stream may start its prologue
 
-  // 2. shared-memory codebook; activations once the previous kernel is done
-  // (compile-time trip counts: all of a thread's codebook loads are in
-  // flight together)
+  if (warp == kGemvThreads / 32) {
+    // ---------------- producer: index blocks of the CTA's items, in order
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < w1 - w0; ++i) {
+        const int s = i % R;
+        if (!mbar_wait(&bar_empty[s], ((i / R) & 1) ^ 1, abrt)) break;
+        const int w = w0 + i, t = w / n_st, st = w % n_st;
+        const int rows = min(kTileRows, L.N - t * kTileRows);
+        const uint32_t bytes = (uint32_t)(NP * rows * 16);
+        mbar_arrive_expect_tx(&bar_full[s], bytes);
+        bulk_load(ring + (size_t)s * SLOT,
+                  L.idx + (size_t)t * kTileRows * L.KC * 16 * L.P + (size_t)st * NP * rows * 16, bytes,
+                  &bar_full[s]);
+        ++issued;
+      }
+      if (*abrt) {  // let the copies this thread issued land before the CTA ends
+        volatile int never = 0;
+        for (int i = max(0, issued - R); i < issued; ++i) mbar_wait(&bar_full[i % R], (i / R) & 1, &never);
+      }
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---------------- consumers
+  const int g = threadIdx.x >> 7, r = threadIdx.x & (kTileRows - 1);
+  // shared-memory codebook (compile-time trip counts: a thread's codebook
+  // loads are all in flight together)
   if (MODE == HXQ_MODE_SCALAR8) {
     constexpr int PER = 256 * 32 / kGemvThreads;
     float cv[PER];
@@ -194,6 +220,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
 #pragma unroll
     for (int j = 0; j < PER; ++j) reinterpret_cast<float4*>(smem)[threadIdx.x + j * kGemvThreads] = cv[j];
   }
+  // activations (zero-padded to Kp) once the previous kernel is done
   pdl_wait();
   {
     constexpr int XU = 4;  // activation loads in flight per thread
@@ -222,33 +249,60 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       }
     }
   }
-  __syncthreads();
+  consumer_sync();
 
   const uint32_t lane4 = (uint32_t)lane * 4u;
-  nst += kGroups;  // (nt, nst): item after the current one
-  while (nst >= n_st) { nst -= n_st; ++nt; }
+  bool waited_ok = true;  // after a timed-out wait the data is garbage but every barrier is still met
+
+  // Sidecar: bounds of this thread's row list for the first segment (the
+  // next segment's bounds are fetched one segment ahead).
+  constexpr int kPE = 4;  // entries per group held in registers (16 per row)
+  int pr0 = 0, pr1 = 0;
+  {
+    const int n0 = (w0 / n_st) * kTileRows + r;
+    if (w0 < w1 && n0 < L.N) {
+      pr0 = __ldg(L.row_ptr + n0);
+      pr1 = __ldg(L.row_ptr + n0 + 1);
+    }
+  }
 
   for (int seg0 = w0; seg0 < w1;) {  // segments: the CTA's items of one tile
     const int t = seg0 / n_st;
     const int seg1 = min(w1, (t + 1) * n_st);
-    // group 0 adds the sidecar corrections of row n; its list bounds load now
+    const int rows = min(kTileRows, L.N - t * kTileRows);
     const int n = t * kTileRows + r;
-    int pr0 = 0, pr1 = 0;
-    if (g == 0 && n < L.N) {
-      pr0 = __ldg(L.row_ptr + n);
-      pr1 = __ldg(L.row_ptr + n + 1);
+    // this group's share of row n's patch entries (p = pr0 + g + 4j), loaded
+    // now and applied at the segment end
+    int ek[kPE];
+    float ed[kPE];
+#pragma unroll
+    for (int j = 0; j < kPE; ++j) {
+      const int p = pr0 + g + kGroups * j;
+      ek[j] = p < pr1 ? __ldg(L.pk + p) : INT_MAX;
+      ed[j] = p < pr1 ? __ldg(L.pd + p) : 0.f;
+    }
+    const int cur0 = pr0, cur1 = pr1;
+    // next segment's list bounds
+    pr0 = pr1 = 0;
+    if (seg1 < w1 && n + kTileRows < L.N) {
+      pr0 = __ldg(L.row_ptr + n + kTileRows);
+      pr1 = __ldg(L.row_ptr + n + kTileRows + 1);
     }
     float2 acc[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.f, 0.f);
 
-    // this thread's items of the segment: w == w0 + g (mod 4)
+    // this group's items of the segment: w == w0 + g (mod 4)
     for (int w = seg0 + ((w0 + g - seg0) % kGroups + kGroups) % kGroups; w < seg1; w += kGroups) {
-      // next item's loads go out first; they land while this item computes
-      uint4 nxt[NP];
-      if (w + kGroups < w1) load_stage<NP>(L, nt, nst, r, nxt);
-      nst += kGroups;
-      while (nst >= n_st) { nst -= n_st; ++nt; }
+      const int i = w - w0, s = i % R;
+      if (waited_ok) waited_ok = mbar_wait(&bar_full[s], (i / R) & 1, abrt);
+      uint4 cur[NP];
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        cur[j] = r < rows ? *reinterpret_cast<const uint4*>(ring + (size_t)s * SLOT + (j * rows + r) * 16)
+                          : make_uint4(0, 0, 0, 0);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_empty[s]);
 
       const int kst = (w - t * n_st) * kStageK;
       if (MODE == HXQ_MODE_SCALAR8) {
@@ -286,15 +340,16 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
           accumulate16<MT, XF32>(acc, wv, xs, L.Kp, kst + h * 16);
         }
       }
-#pragma unroll
-      for (int j = 0; j < NP; ++j) cur[j] = nxt[j];
     }
 
     // sidecar corrections of this segment's columns: acc += delta * x[k]
-    if (pr1 > pr0) {
+    {
       const int ka = (seg0 - t * n_st) * kStageK, kb = (seg1 - t * n_st) * kStageK;
+#pragma unroll
+      for (int j = 0; j < kPE; ++j)
+        if (ek[j] >= ka && ek[j] < kb) add_patch<MT, XF32>(acc, ed[j], xs, L.Kp, ek[j]);
 #pragma unroll 1
-      for (int p = pr0; p < pr1; ++p) {
+      for (int p = cur0 + g + kGroups * kPE; p < cur1; p += kGroups) {  // rows with > 16 entries
         const int k = __ldg(L.pk + p);
         if (k >= ka && k < kb) add_patch<MT, XF32>(acc, __ldg(L.pd + p), xs, L.Kp, k);
       }
@@ -303,12 +358,11 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
     // segment end: the 4 groups' sums meet in shared memory
 #pragma unroll
     for (int m = 0; m < MT; ++m) red[(g * MT + m) * kTileRows + r] = acc[m].x + acc[m].y;
-    __syncthreads();
-    const int rows = min(kTileRows, L.N - t * kTileRows);
+    consumer_sync();
     const bool full = seg0 == t * n_st && seg1 == (t + 1) * n_st;
     const int slot = (t == w0 / n_st) ? 0 : 1;
     float* part = work + (size_t)(blockIdx.x * 2 + slot) * MT * kTileRows;
-    for (int i = threadIdx.x; i < MT * kTileRows; i += blockDim.x) {
+    for (int i = threadIdx.x; i < MT * kTileRows; i += kGemvThreads) {
       const int m = i / kTileRows, rr = i % kTileRows;
       const float v = red[(0 * MT + m) * kTileRows + rr] + red[(1 * MT + m) * kTileRows + rr] +
                       red[(2 * MT + m) * kTileRows + rr] + red[(3 * MT + m) * kTileRows + rr];
@@ -320,13 +374,13 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
     }
     if (!full) {
       __threadfence();
-      __syncthreads();
+      consumer_sync();
       const int c_first = cta_of(t * n_st, W, G), c_last = cta_of((t + 1) * n_st - 1, W, G);
       if (threadIdx.x == 0) last_flag = atomicAdd(counters + t, 1) == c_last - c_first;
-      __syncthreads();
+      consumer_sync();
       if (last_flag) {
         __threadfence();
-        for (int i = threadIdx.x; i < MT * kTileRows; i += blockDim.x) {
+        for (int i = threadIdx.x; i < MT * kTileRows; i += kGemvThreads) {
           const int m = i / kTileRows, rr = i % kTileRows;
           if (m >= M || rr >= rows) continue;
           float v = 0.f;
@@ -340,24 +394,29 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
         if (threadIdx.x == 0) counters[t] = 0;
       }
     }
-    __syncthreads();
+    consumer_sync();
     seg0 = seg1;
   }
+  if (!waited_ok && threadIdx.x == 0) atomicOr(status, kStatusWaitTimeout);
+  __syncthreads();
 }
 
 template <int MT, bool XF32, int MODE>
 cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t s) {
+  const int R = ring_slots(MODE, MT, h.L.Kp, XF32);
+  if (R < kGroups) return cudaErrorInvalidValue;
   const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32);
   auto kern = gemv_kernel<MT, XF32, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int W = h.L.n_tiles * (h.L.Kp / kStageK);
-  return launch_pdl(kern, grid, kGemvThreads, smem, s, h.L, x, y, M, W, h.d_work, h.d_counters);
+  return launch_pdl(kern, grid, kGemvThreads + 32, smem, s, h.L, x, y, M, W, R, h.d_work, h.d_counters,
+                    h.d_status);
 }
 
 template <int MT, int MODE>
 cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t s) {
-  if (gemv_smem(MODE, MT, h.L.Kp, true) <= kSmemLimit) return launch_cfg<MT, true, MODE>(h, x, y, M, grid, s);
+  if (ring_slots(MODE, MT, h.L.Kp, true) >= kGroups) return launch_cfg<MT, true, MODE>(h, x, y, M, grid, s);
   return launch_cfg<MT, false, MODE>(h, x, y, M, grid, s);
 }
 
@@ -367,16 +426,15 @@ cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M,
   if (M <= 2) return launch_mt<2, MODE>(h, x, y, M, grid, s);
   if (M <= 4) return launch_mt<4, MODE>(h, x, y, M, grid, s);
   if (M <= 8) return launch_mt<8, MODE>(h, x, y, M, grid, s);
-  if (M <= 16) return launch_mt<16, MODE>(h, x, y, M, grid, s);
-  return launch_mt<32, MODE>(h, x, y, M, grid, s);
+  return launch_mt<16, MODE>(h, x, y, M, grid, s);
 }
 
-int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : M <= 16 ? 16 : 32; }
+int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
 
 }  // namespace
 
 bool gemv_supports(const hxq_linear& h, int M) {
-  return M >= 1 && M <= 32 && gemv_smem(h.L.mode, mt_of(M), h.L.Kp, false) <= kSmemLimit;
+  return M >= 1 && M <= 16 && ring_slots(h.L.mode, mt_of(M), h.L.Kp, false) >= kGroups;
 }
 
 // Persistent grid: one CTA per SM, fewer when the layer has fewer work items.

@@ -409,8 +409,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
         const int n = t * kTileRows + r;
         pkn = INT_MAX;
         if (n < L.N) {
-          pp = row_lower_bound(L, n, kst);
-          pe = L.row_ptr[n + 1];
+          pp = kst == 0 ? __ldg(L.row_ptr + n) : row_lower_bound(L, n, kst);
+          pe = __ldg(L.row_ptr + n + 1);
           if (pp < pe) { pkn = __ldg(L.pk + pp); pvn = __ldg(L.pv + pp); }
         }
       }
