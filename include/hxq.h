@@ -139,6 +139,33 @@ int hxq_decode(hxq_linear_t h, float* W_out, void* stream);
  */
 int hxq_linear_check(hxq_linear_t h);
 
+/*
+ * The CUDA-core GEMV (M <= 4) for callers that cannot call cudaMalloc at the
+ * point where they run the layer: code under an allocation-free policy after
+ * start-up (a real-time or latency-critical loop, where an allocation would
+ * synchronise the device), or code that runs handles created elsewhere and
+ * may not assume their workspace is free to use. The paper has no
+ * counterpart: its layers allocate and share a materialisation buffer.
+ *
+ * Same arguments and result as hxq_linear_forward, computed by the same
+ * kernel, but its scratch (per-tile arrival counters and the fp32 partial
+ * sums of tiles split between CTAs) lives in one fixed array of 1 MiB + 16 KiB
+ * compiled into this library, resident on every GPU that loads it until the
+ * process exits; the call itself allocates nothing. The first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress) and
+ * should come before any stream capture. Each call clears the counters on
+ * `stream` before the kernel runs. All calls share the one array, which keeps
+ * the last call's contents: calls that overlap in time on the GPU (other
+ * streams, other threads) race and give wrong results -- serialise them.
+ *
+ * Limits: 1 <= M <= 4, N <= 524288 (4096 tiles of 128 rows), the handle's
+ * device current. Returns HXQ_EINVAL beyond them (nothing is launched), for
+ * the argument errors of hxq_linear_forward, or when another device is
+ * current; HXQ_ECUDA if the symbol lookup, the clear or the launch fails.
+ */
+int hxq_linear_forward_noalloc(hxq_linear_t h, const void* x_bf16, float* y, int M,
+                               void* stream);
+
 /* Shape of a handle: any output pointer may be NULL. HXQ_EINVAL if h is NULL. */
 int hxq_linear_info(hxq_linear_t h, int* mode, int* N, int* K, int64_t* n_sidecar);
 

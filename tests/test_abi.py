@@ -98,5 +98,5 @@ def test_create_without_device_reports_unsupported():
 
 
 def test_build_flags_target_sm100a():
-    from vq_compressed_linear_b200 import build
-    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    import __graft_entry__
+    assert __graft_entry__._builder().ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -3,7 +3,7 @@
 The C ABI (include/hxq.h) is the product: this module only marshals
 arguments. Every step of the forward runs in the library's CUDA kernels;
 there is no Python or CPU fallback, and importing fails loudly when the
-library has not been built (python -m vq_compressed_linear_b200.build).
+library has not been built (python vq_compressed_linear_b200/build.py).
 
 PyTorch is used for device memory and streams only: tensors are passed by
 data pointer, the current torch stream is passed as the cudaStream_t.
@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libhxq.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libhxq.so is missing at {LIB_PATH}: build it with "
-        "`python -m vq_compressed_linear_b200.build` (nvcc, sm_100a)")
+        "`python vq_compressed_linear_b200/build.py` (nvcc, sm_100a)")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -42,6 +42,8 @@ lib.hxq_linear_forward.argtypes = [_vp, _vp, _vp, _i, _vp]
 lib.hxq_linear_forward.restype = _i
 lib.hxq_linear_forward_ex.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp]
 lib.hxq_linear_forward_ex.restype = _i
+lib.hxq_linear_forward_noalloc.argtypes = [_vp, _vp, _vp, _i, _vp]
+lib.hxq_linear_forward_noalloc.restype = _i
 lib.hxq_decode.argtypes = [_vp, _vp, _vp]
 lib.hxq_decode.restype = _i
 lib.hxq_linear_check.argtypes = [_vp]
@@ -54,7 +56,8 @@ lib.hxq_linear_destroy.restype = None
 lib.hxq_strerror.argtypes = [_i]
 lib.hxq_strerror.restype = ctypes.c_char_p
 
-EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_decode",
+EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_linear_forward_noalloc",
+            "hxq_decode",
             "hxq_linear_check", "hxq_linear_info", "hxq_linear_destroy", "hxq_strerror")
 
 
@@ -107,6 +110,11 @@ def hxq_linear_forward(h, x, y, M, stream=None) -> None:
 def hxq_linear_forward_ex(h, x, y, M, kernel, split_k, stream=None) -> None:
     _check(lib.hxq_linear_forward_ex(h, _ptr(x), _ptr(y), int(M), int(kernel), int(split_k),
                                      _stream(stream)), "hxq_linear_forward_ex")
+
+
+def hxq_linear_forward_noalloc(h, x, y, M, stream=None) -> None:
+    _check(lib.hxq_linear_forward_noalloc(h, _ptr(x), _ptr(y), int(M), _stream(stream)),
+           "hxq_linear_forward_noalloc")
 
 
 def hxq_decode(h, W_out, stream=None) -> None:

@@ -1,6 +1,8 @@
 """Build libhxq.so in place: nvcc for sm_100a, static CUDA runtime.
 
-    python -m vq_compressed_linear_b200.build [--verbose]
+    python vq_compressed_linear_b200/build.py [--verbose]
+
+(Run by path: importing the package would load the library being rebuilt.)
 
 Each .cu under csrc/ compiles to an object in _build/ (in parallel), then one
 shared library is linked next to this file. --verbose passes -Xptxas -v

@@ -402,7 +402,8 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
 }
 
 template <int MT, bool XF32, int MODE>
-cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t s) {
+cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
+                       cudaStream_t s) {
   const int R = ring_slots(MODE, MT, h.L.Kp, XF32);
   if (R < kGroups) return cudaErrorInvalidValue;
   const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32);
@@ -410,23 +411,25 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int W = h.L.n_tiles * (h.L.Kp / kStageK);
-  return launch_pdl(kern, grid, kGemvThreads + 32, smem, s, h.L, x, y, M, W, R, h.d_work, h.d_counters,
-                    h.d_status);
+  return launch_pdl(kern, grid, kGemvThreads + 32, smem, s, h.L, x, y, M, W, R, work, counters, h.d_status);
 }
 
 template <int MT, int MODE>
-cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t s) {
-  if (ring_slots(MODE, MT, h.L.Kp, true) >= kGroups) return launch_cfg<MT, true, MODE>(h, x, y, M, grid, s);
-  return launch_cfg<MT, false, MODE>(h, x, y, M, grid, s);
+cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
+                      cudaStream_t s) {
+  if (ring_slots(MODE, MT, h.L.Kp, true) >= kGroups)
+    return launch_cfg<MT, true, MODE>(h, x, y, M, grid, work, counters, s);
+  return launch_cfg<MT, false, MODE>(h, x, y, M, grid, work, counters, s);
 }
 
 template <int MODE>
-cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t s) {
-  if (M <= 1) return launch_mt<1, MODE>(h, x, y, M, grid, s);
-  if (M <= 2) return launch_mt<2, MODE>(h, x, y, M, grid, s);
-  if (M <= 4) return launch_mt<4, MODE>(h, x, y, M, grid, s);
-  if (M <= 8) return launch_mt<8, MODE>(h, x, y, M, grid, s);
-  return launch_mt<16, MODE>(h, x, y, M, grid, s);
+cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
+                        cudaStream_t s) {
+  if (M <= 1) return launch_mt<1, MODE>(h, x, y, M, grid, work, counters, s);
+  if (M <= 2) return launch_mt<2, MODE>(h, x, y, M, grid, work, counters, s);
+  if (M <= 4) return launch_mt<4, MODE>(h, x, y, M, grid, work, counters, s);
+  if (M <= 8) return launch_mt<8, MODE>(h, x, y, M, grid, work, counters, s);
+  return launch_mt<16, MODE>(h, x, y, M, grid, work, counters, s);
 }
 
 int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
@@ -440,16 +443,98 @@ bool gemv_supports(const hxq_linear& h, int M) {
 // Persistent grid: one CTA per SM, fewer when the layer has fewer work items.
 // `split` (when non-zero) sets the grid so that each tile's K is shared by
 // about `split` CTAs.
-cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M, int split, cudaStream_t s) {
-  if (!gemv_supports(h, M)) return cudaErrorInvalidValue;
+int gemv_grid(const hxq_linear& h, int split) {
   const int64_t W = (int64_t)h.L.n_tiles * (h.L.Kp / kStageK);
   int64_t grid = split > 0 ? (int64_t)h.L.n_tiles * split : h.num_sms;
   grid = std::max<int64_t>(1, std::min<int64_t>({grid, (int64_t)h.num_sms, W}));
-  if (W * grid >= INT_MAX) return cudaErrorInvalidValue;  // item arithmetic is 32-bit
+  if (W * grid >= INT_MAX) return 0;  // item arithmetic is 32-bit
+  return (int)grid;
+}
+
+cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M, int split, cudaStream_t s) {
+  if (!gemv_supports(h, M)) return cudaErrorInvalidValue;
+  const int grid = gemv_grid(h, split);
+  if (grid == 0) return cudaErrorInvalidValue;
   // every CTA writes at most two partial tiles of mt_of(M) x 128 floats
   if ((size_t)grid * 2 * mt_of(M) * kTileRows > h.work_floats) return cudaErrorInvalidValue;
-  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, (int)grid, s);
-  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, (int)grid, s);
+  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, grid, h.d_work, h.d_counters, s);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, grid, h.d_work, h.d_counters, s);
 }
 
 }  // namespace hxq
+
+// ----------------------------------------------------------------------------
+// hxq_linear_forward_noalloc: the CUDA-core GEMV with its scratch -- the
+// stream-K arrival counters and partial sums -- in a fixed array compiled
+// into this library instead of the handle's workspace. Nothing is allocated
+// on this path; the array stays resident on every GPU that loads the library
+// until the process exits.
+// ----------------------------------------------------------------------------
+#include <mutex>
+
+namespace hxq {
+namespace {
+constexpr int kNoAllocMaxTiles = 4096;                   // N <= 524288 output features
+constexpr size_t kNoAllocPartialFloats = 256 * 1024;     // 1 MiB of fp32 partial sums
+constexpr size_t kNoAllocScratchBytes = kNoAllocMaxTiles * sizeof(int) + kNoAllocPartialFloats * sizeof(float);
+}  // namespace
+}  // namespace hxq
+
+// [0, 16 KB): per-tile arrival counters (must start at zero); then partials.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[hxq::kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[256];  // device address of g_noalloc_scratch, per device ordinal
+
+// Device address of the scratch array on device `dev` (current). In host code
+// the array's name is only a host-side stand-in, so the address comes from
+// cudaGetSymbolAddress, once per device.
+cudaError_t noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+extern "C" int hxq_linear_forward_noalloc(hxq_linear_t h, const void* x_bf16, float* y, int M, void* stream) {
+  using namespace hxq;
+  if (!h || !x_bf16 || !y || M < 1 || M > 4) return HXQ_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) != 0) return HXQ_EINVAL;
+  if (!gemv_supports(*h, M) || h->L.n_tiles > kNoAllocMaxTiles) return HXQ_EINVAL;
+  const int grid = gemv_grid(*h, 0);
+  if (grid == 0 || (size_t)grid * 2 * mt_of(M) * kTileRows > kNoAllocPartialFloats) return HXQ_EINVAL;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_ECUDA;
+  }
+  if (dev != h->device) return HXQ_EINVAL;
+  void* base = nullptr;
+  if (noalloc_scratch(dev, &base) != cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_ECUDA;
+  }
+  int* counters = static_cast<int*>(base);
+  float* work = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + kNoAllocMaxTiles * sizeof(int));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // a previous call may have been interrupted mid-way: the counters restart at zero
+  cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)h->L.n_tiles * sizeof(int), s);
+  if (e == cudaSuccess) {
+    const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+    e = h->L.mode == HXQ_MODE_SCALAR8 ? launch_mode<HXQ_MODE_SCALAR8>(*h, x, y, M, grid, work, counters, s)
+                                      : launch_mode<HXQ_MODE_VQ2D12>(*h, x, y, M, grid, work, counters, s);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_ECUDA;
+  }
+  return HXQ_OK;
+}

@@ -87,6 +87,7 @@ cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M,
 cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, float* y, int M, int split,
                       cudaStream_t s);
 bool gemv_supports(const hxq_linear& h, int M);
+int gemv_grid(const hxq_linear& h, int split);
 size_t tc_workspace_floats(int num_sms);
 
 // Launch `kern` with programmatic stream serialization: it may start while
