@@ -53,6 +53,21 @@ def peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+def max_over_ranks(torch, dist, world, value, device):
+    """The largest of every rank's `value` (device times: the job ends with the
+    slowest rank). All ranks must call it, in the same order."""
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_step, steps, world, ms_max, scale):
+    """Whole-job throughput: the units all `world` replicas processed over the
+    slowest rank's time, divided by `scale` (1e9 for GB/s, 1e12 for TFLOP/s)."""
+    return units_per_step * steps * world / (ms_max * 1e-3) / scale
+
+
 def layer_bytes(layer, M):
     N, K, mode = layer["N"], layer["K"], layer["mode"]
     idx = N * K if mode == synthetic.MODE_SCALAR8 else 3 * N * K // 4
@@ -423,23 +438,14 @@ def main():
             hxq, torch, items, args.steps, args.warmup, l2, stream, soak_s=1.5)
         barrier()
     clocks = clk.summary()
-    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    total_bytes = step_bytes * args.steps * world
-    total_flops = step_flops * args.steps * world
-    gbs = total_bytes / (ms_max * 1e-3) / 1e9
-    tfs = total_flops / (ms_max * 1e-3) / 1e12
-    value = tfs if is_prefill else gbs
+    ms_max = max_over_ranks(torch, dist, world, ms, "cuda")
+    units, scale = (step_flops, 1e12) if is_prefill else (step_bytes, 1e9)
+    value = job_rate(units, args.steps, world, ms_max, scale)
 
     # e2e through the public call, host buffers
     e_ms, h2d, d2h = e2e_workload(hxq, torch, items, args.steps, args.warmup, stream)
-    te = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e_ms = float(te.item())
-    e_val = (total_flops / (e_ms * 1e-3) / 1e12) if is_prefill else (total_bytes / (e_ms * 1e-3) / 1e9)
+    e_ms = max_over_ranks(torch, dist, world, e_ms, "cuda")
+    e_val = job_rate(units, args.steps, world, e_ms, scale)
 
     # roofline of the dominant kernel (all launches of this workload are one kernel)
     _, l0, M0 = items[0]
