@@ -63,7 +63,7 @@ enum {
 /* Kernel choice for hxq_linear_forward_ex. */
 enum {
     HXQ_KERNEL_AUTO = 0,   /* CUDA-core GEMV for M <= 4, tensor cores above  */
-    HXQ_KERNEL_GEMV = 1,   /* CUDA-core fused-decode GEMV, fp32 weights; M <= 16
+    HXQ_KERNEL_GEMV = 1,   /* CUDA-core fused-decode GEMV, fp32 weights; M <= 8 
                               and the activations must fit in shared memory */
     HXQ_KERNEL_TC = 2      /* tcgen05 fused-decode GEMM; fp32-exact split
                               weights (hi+mid bf16) for M <= 32, bf16 weights
@@ -117,7 +117,7 @@ int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M,
  * count along K (0 = automatic, else 1..64), for tests and benchmarks. The
  * numerics of each kernel are those stated above for its M range.
  * HXQ_EINVAL additionally for an unknown kernel, split_k outside 0..64, or
- * HXQ_KERNEL_GEMV where it does not apply (M > 16, or M * K too large for its
+ * HXQ_KERNEL_GEMV where it does not apply (M > 8, or M * K too large for its
  * shared-memory staging of x; HXQ_KERNEL_AUTO then picks the tensor cores).
  */
 int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M,

@@ -83,7 +83,7 @@ def test_forward_matches_oracle(hxq, mode, N, K, M):
     x = synthetic.activations(M, K, 7)
     _, y_ref, s = oracle.forward_layer(layer, x)
     lin = hxq.HelixLinear.from_layer(layer)
-    kernels = [AUTO, TC] + ([GEMV] if M <= 16 else [])
+    kernels = [AUTO, TC] + ([GEMV] if M <= 8 else [])
     for kernel in kernels:
         for split in (0, 1, 3):
             y = run(hxq, lin, x, kernel, split)
@@ -204,7 +204,7 @@ def test_forward_rejects_bad_arguments(hxq):
     lin = hxq.HelixLinear.from_layer(layer)
     x = torch.zeros((40, 64), dtype=torch.int16, device="cuda")
     y = torch.zeros((40, 128), dtype=torch.float32, device="cuda")
-    for kernel, split, M in ((3, 0, 1), (GEMV, 0, 17), (AUTO, 65, 1), (AUTO, -1, 1), (AUTO, 0, 0)):
+    for kernel, split, M in ((3, 0, 1), (GEMV, 0, 9), (AUTO, 65, 1), (AUTO, -1, 1), (AUTO, 0, 0)):
         rc = hxq.lib.hxq_linear_forward_ex(lin.handle, x.data_ptr(), y.data_ptr(), M, kernel, split, None)
         assert rc == hxq.HXQ_EINVAL
     rc = hxq.lib.hxq_linear_forward(lin.handle, x.data_ptr() + 2, y.data_ptr(), 1, None)

@@ -1,25 +1,30 @@
 // Fused decode + GEMV on CUDA cores for few tokens (M <= 4 by default; up to
-// M = 16 on request): y[m][n] = sum_k x[m][k] * W[n][k] with W decoded on the
+// M = 8 on request): y[m][n] = sum_k x[m][k] * W[n][k] with W decoded on the
 // fly from the codebook and never written anywhere (the pages' buffered path
 // instead materialises W and calls cuBLAS: HXQ whitepaper, method section,
 // buffered forward path paragraph).
 //
-// Work decomposition (stream-K). The work items are the tile-stages of the
-// layer, (tile of 128 rows) x (64 weights along K), numbered tile-major; an
-// item's indices are one contiguous block of the tiled layout. A persistent
-// grid of one CTA per SM takes contiguous item ranges of equal size, so every
+// Work decomposition (stream-K). The layer's stages (tile of 128 rows x 64
+// weights along K), numbered tile-major, are cut into contiguous ranges of
+// equal length, one per CTA of a persistent grid (one CTA per SM), so every
 // CTA streams the same number of index bytes whatever the layer shape.
 //
-// Inside a CTA a producer warp streams the items' index blocks with TMA bulk
-// copies into a ring of shared-memory slots (up to 12 x 8 KB in flight per
-// SM; it starts before the previous kernel has finished, since the indices do
-// not depend on it), and 4 groups of 128 consumer threads take the items
-// round-robin: thread r of a group owns row r of the item's tile, reads its
-// 16-byte pieces from the slot, releases the slot and decodes. At each tile
-// boundary of the CTA's range the groups' sums meet in shared memory; a tile
-// covered by one CTA goes straight to y, a tile split between CTAs leaves one
-// fp32 partial per CTA in the workspace and the last CTA to arrive (integer
-// atomic per tile) adds them in CTA order: results are bitwise repeatable.
+// Inside a CTA a producer warp streams the range in chunks of up to 4 stages
+// of one tile (32 KB of scalar indices, contiguous in the tiled layout) with
+// TMA bulk copies into a ring of shared-memory slots; it starts before the
+// previous kernel has finished, since the indices do not depend on it. The
+// 16 consumer warps share every chunk: warp q takes the q-th 16-weight piece
+// of the chunk (stage q / 4, quarter q % 4) for all 128 rows, lane l for rows
+// l, l + 32, l + 64, l + 96. So each activation a warp loads from shared
+// memory serves four rows: the decode is bound by the shared-memory pipe, and
+// per 32 weights it costs one conflict-free table lookup wavefront plus a
+// quarter wavefront of index bytes plus the activations.
+//
+// At each tile boundary of the CTA's range the warps' sums meet in shared
+// memory; a tile covered by one CTA goes straight to y, a tile split between
+// CTAs leaves one fp32 partial per CTA in the workspace and the last CTA to
+// arrive (integer atomic per tile) adds them in CTA order: results are
+// bitwise repeatable.
 //
 // Scalar codebook in shared memory: replicated once per lane with entry e of
 // lane l at byte e*256 + l*4, so the 32 lanes of a lookup always hit 32
@@ -35,38 +40,46 @@
 // Sidecar (replacement of single weights, HXQ whitepaper, method section,
 // "Sidecar outlier correction"): replacing w = c by v adds (v - c) x to the
 // dot product, so each entry carries delta = v - c (fp32, computed once when
-// the handle is built). The main loop decodes with the codebook alone; each
-// group loads its share of the row's patch entries when a tile segment
-// starts (list bounds fetched one segment ahead) and adds delta * x[k] for
-// those in the segment's columns at its end -- no dependent memory access on
-// the critical path.
+// the handle is built). The main loop decodes with the codebook alone; the
+// thread that finishes row n of a segment loads row n's first patch entries
+// when the segment starts (list bounds fetched one segment ahead) and adds
+// delta * x[k] for those in the segment's columns to the row's sum.
 #include <algorithm>
 #include <climits>
+#include <type_traits>
 
 #include "hxq_internal.cuh"
 
 namespace hxq {
 namespace {
 
-constexpr int kGemvThreads = 512;                  // consumers; one more warp produces
-constexpr int kGroups = kGemvThreads / kTileRows;  // consumer groups (128 rows each)
-constexpr int kMaxRing = 12;                       // index slots in flight per CTA
+constexpr int kGemvThreads = 512;                  // consumers; then a producer and a fixup warp
+constexpr int kConsumerWarps = kGemvThreads / 32;  // 16: one 16-weight piece of a chunk each
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kFixupWarp = kConsumerWarps + 1;
+constexpr int kGemvBlock = kGemvThreads + 64;
+constexpr int kBarConsumers = 1;                   // named barriers: consumers only,
+constexpr int kBarHandoff0 = 2;                    // consumers -> fixup warp
+constexpr int kChunkStages = 4;                    // stages per ring slot (16 pieces per row)
+constexpr int kMaxRing = 6;                        // ring slots
+constexpr int kGemvMaxM = 8;                       // tokens
 constexpr size_t kSmemLimit = 226 * 1024;          // dynamic shared memory per CTA (static kept apart)
 
 // Dynamic shared memory of one CTA: codebook table, activations (fp32 or
-// bf16) and the groups' partial sums, then the index ring.
+// bf16), the warps' partial sums and the split-tile sum handed to the fixup
+// warp, then the index ring.
 inline size_t gemv_smem_fixed(int mode, int MT, int Kp, bool xf32) {
   return (size_t)(mode == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8) + (size_t)MT * Kp * (xf32 ? 4 : 2) +
-         (size_t)kGroups * MT * kTileRows * sizeof(float);
+         (size_t)(kConsumerWarps + 1) * MT * kTileRows * sizeof(float);
 }
-inline int slot_bytes(int mode) { return (mode == HXQ_MODE_SCALAR8 ? 4 : 3) * kTileRows * 16; }
-// Ring slots that fit next to the fixed part (a multiple of the groups; 0 if
-// fewer than one per group fit).
+inline int slot_bytes(int mode) { return kChunkStages * (mode == HXQ_MODE_SCALAR8 ? 4 : 3) * kTileRows * 16; }
+// Ring slots that fit next to the fixed part (0 if fewer than two fit).
+constexpr int kMinRing = 2;
 inline int ring_slots(int mode, int MT, int Kp, bool xf32) {
   const size_t fixed = gemv_smem_fixed(mode, MT, Kp, xf32);
   if (fixed + 128 > kSmemLimit) return 0;
-  const int fit = (int)((kSmemLimit - fixed - 128) / slot_bytes(mode));
-  return std::min(kMaxRing, fit / kGroups * kGroups);
+  const int fit = std::min(kMaxRing, (int)((kSmemLimit - fixed - 128) / slot_bytes(mode)));
+  return fit >= kMinRing ? fit : 0;
 }
 inline size_t gemv_smem(int mode, int MT, int Kp, bool xf32) {
   return gemv_smem_fixed(mode, MT, Kp, xf32) + 128 + (size_t)ring_slots(mode, MT, Kp, xf32) * slot_bytes(mode);
@@ -78,7 +91,7 @@ constexpr int table_bytes() { return MODE == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// CTA whose item range [b W / G, (b+1) W / G) contains item w (W * G < 2^31).
+// CTA whose stage range [b W / G, (b+1) W / G) contains stage w (W * G < 2^31).
 __device__ __forceinline__ int cta_of(int w, int W, int G) {
   int b = (w * G) / W;
   while (b + 1 < G && ((b + 1) * W) / G <= w) ++b;
@@ -111,48 +124,87 @@ __device__ __forceinline__ void x16(const uint8_t* xs, int Kp, int m, int k0, fl
   }
 }
 
-template <int MT, bool XF32>
-__device__ __forceinline__ void accumulate16(float2 (&acc)[MT], const float (&w)[16], const uint8_t* xs, int Kp,
-                                             int k0) {
+__device__ __forceinline__ void fma16(float2& acc, const float (&w)[16], const float (&xv)[16]) {
 #pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    float xv[16];
-    x16<XF32>(xs, Kp, m, k0, xv);
+  for (int j = 0; j < 16; j += 2) acc = __ffma2_rn(make_float2(w[j], w[j + 1]), make_float2(xv[j], xv[j + 1]), acc);
+}
+// One register per sum (scalar FMAs) where paired sums would not fit.
+__device__ __forceinline__ void fma16(float& acc, const float (&w)[16], const float (&xv)[16]) {
 #pragma unroll
-    for (int j = 0; j < 16; j += 2)
-      acc[m] = __ffma2_rn(make_float2(w[j], w[j + 1]), make_float2(xv[j], xv[j + 1]), acc[m]);
+  for (int j = 0; j < 16; ++j) acc = fmaf(w[j], xv[j], acc);
+}
+__device__ __forceinline__ float acc_sum(float2 a) { return a.x + a.y; }
+__device__ __forceinline__ float acc_sum(float a) { return a; }
+__device__ __forceinline__ void acc_zero(float2& a) { a = make_float2(0.f, 0.f); }
+__device__ __forceinline__ void acc_zero(float& a) { a = 0.f; }
+
+__device__ __forceinline__ float x_at(const uint8_t* xs, int Kp, int m, int k, bool xf32) {
+  return xf32 ? *reinterpret_cast<const float*>(xs + ((size_t)m * Kp + k) * 4)
+              : bf16lo(*reinterpret_cast<const uint16_t*>(xs + ((size_t)m * Kp + k) * 2));
+}
+
+// The 16 weights of one row's piece: scalar indices (one 16-byte piece).
+template <int MODE>
+__device__ __forceinline__ void decode16(const uint8_t* smem, const uint8_t* piece, int rows, int quarter,
+                                         uint32_t lane4, float (&wv)[16]) {
+  if (MODE == HXQ_MODE_SCALAR8) {
+    const uint4 cur = *reinterpret_cast<const uint4*>(piece);
+    const uint32_t wd[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t a = prmt(wd[j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
+      wv[j] = *reinterpret_cast<const float*>(smem + a);
+    }
+  } else {
+    // the quarter's 8 pairs are bytes [12 q, 12 q + 12) of the row's 48 in
+    // the stage's three 16-byte planes (`piece` points at plane 0)
+    uint32_t wd[4] = {0, 0, 0, 0};
+    const uint8_t* p1 = piece + rows * 16;
+    const uint8_t* p2 = p1 + rows * 16;
+    if (quarter == 0) {
+      const uint4 v = *reinterpret_cast<const uint4*>(piece);
+      wd[0] = v.x; wd[1] = v.y; wd[2] = v.z;
+    } else if (quarter == 1) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p1);
+      wd[0] = *reinterpret_cast<const uint32_t*>(piece + 12); wd[1] = v.x; wd[2] = v.y;
+    } else if (quarter == 2) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p1 + 8);
+      wd[0] = v.x; wd[1] = v.y; wd[2] = *reinterpret_cast<const uint32_t*>(p2);
+    } else {
+      const uint4 v = *reinterpret_cast<const uint4*>(p2);
+      wd[0] = v.y; wd[1] = v.z; wd[2] = v.w;
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int bit = 12 * jj;
+      const uint32_t e8 = (bit & 31) >= 3
+          ? (__funnelshift_r(wd[bit >> 5], wd[(bit >> 5) + 1], (bit & 31) - 3) & 0x7FF8u)
+          : ((wd[bit >> 5] << (3 - (bit & 31))) & 0x7FF8u);
+      const float2 pr = *reinterpret_cast<const float2*>(smem + e8);
+      wv[2 * jj] = pr.x;
+      wv[2 * jj + 1] = pr.y;
+    }
   }
 }
 
-template <int MT, bool XF32>
-__device__ __forceinline__ void add_patch(float2 (&acc)[MT], float d, const uint8_t* xs, int Kp, int k) {
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    const float xv = XF32 ? *reinterpret_cast<const float*>(xs + ((size_t)m * Kp + k) * 4)
-                          : bf16lo(*reinterpret_cast<const uint16_t*>(xs + ((size_t)m * Kp + k) * 2));
-    acc[m].x = fmaf(d, xv, acc[m].x);
-  }
-}
-
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kGemvThreads) : "memory");
-}
+__device__ __forceinline__ void consumer_sync() { named_bar_sync(kBarConsumers, kGemvThreads); }
 
 template <int MT, bool XF32, int MODE>
-__global__ void __launch_bounds__(kGemvThreads + 32, 1)
+__global__ void __launch_bounds__(kGemvBlock, 1)
 gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int W, int R,
             float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int TB = table_bytes<MODE>();
   constexpr int NP = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per row and stage
   uint8_t* xs = smem + TB;
-  // per-group partial sums [kGroups][MT][kTileRows], after the activations
+  // per-warp partial sums [kConsumerWarps][MT][kTileRows], after the activations
   float* red = reinterpret_cast<float*>(xs + (size_t)MT * L.Kp * (XF32 ? 4 : 2));
+  float* pbuf = red + kConsumerWarps * MT * kTileRows;  // [MT][kTileRows] sum for the fixup warp
   uint8_t* ring = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(red + kGroups * MT * kTileRows) + 127) & ~(uintptr_t)127);
-  constexpr int SLOT = NP * kTileRows * 16;
+      (reinterpret_cast<uintptr_t>(pbuf + MT * kTileRows) + 127) & ~(uintptr_t)127);
+  constexpr int SLOT = kChunkStages * NP * kTileRows * 16;
   __shared__ uint64_t bar_full[kMaxRing], bar_empty[kMaxRing];
-  __shared__ int last_flag, abort_sh;
+  __shared__ int abort_sh, flag_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_st = n_stages(L);
@@ -163,7 +215,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   if (threadIdx.x == 0) {
     for (int i = 0; i < R; ++i) {
       mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], 4);  // the 4 warps of the consuming group
+      mbar_init(&bar_empty[i], kConsumerWarps);  // every consumer warp reads every slot
     }
     abort_sh = 0;
     fence_mbar_init();
@@ -171,21 +223,24 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   __syncthreads();
   pdl_launch_dependents();  // the next kernel in the stream may start its prologue
 
-  if (warp == kGemvThreads / 32) {
-    // ---------------- producer: index blocks of the CTA's items, in order
+  if (warp == kProducerWarp) {
+    // ---------------- producer: the range's chunks, in order
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < w1 - w0; ++i) {
-        const int s = i % R;
-        if (!mbar_wait(&bar_empty[s], ((i / R) & 1) ^ 1, abrt)) break;
-        const int w = w0 + i, t = w / n_st, st = w % n_st;
+      int issued = 0, s = 0;
+      uint32_t ph = 0;
+      for (int w = w0; w < w1;) {
+        const int t = w / n_st, st = w - t * n_st;
+        const int we = min(min(w + kChunkStages, (t + 1) * n_st), w1);
+        if (!mbar_wait(&bar_empty[s], ph ^ 1, abrt)) break;
         const int rows = min(kTileRows, L.N - t * kTileRows);
-        const uint32_t bytes = (uint32_t)(NP * rows * 16);
+        const uint32_t bytes = (uint32_t)((we - w) * NP * rows * 16);
         mbar_arrive_expect_tx(&bar_full[s], bytes);
         bulk_load(ring + (size_t)s * SLOT,
                   L.idx + (size_t)t * kTileRows * L.KC * 16 * L.P + (size_t)st * NP * rows * 16, bytes,
                   &bar_full[s]);
         ++issued;
+        if (++s == R) s = 0, ph ^= 1;
+        w = we;
       }
       if (*abrt) {  // let the copies this thread issued land before the CTA ends
         volatile int never = 0;
@@ -196,8 +251,59 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
     return;
   }
 
+  if (warp == kFixupWarp) {
+    // ---------------- fixup: a split tile at the start of the CTA's range
+    // that is not also its end (the tail of a tile that earlier CTAs began),
+    // handed over by the consumers so that they never wait on global memory:
+    // store this CTA's sum in the workspace and count it on the tile's
+    // counter. The CTA that counts last (almost never this one: the other
+    // contributors finish their part of the tile at the end of their ranges)
+    // adds all sums in CTA order and writes y.
+    pdl_wait();  // y, the workspace and the counters may be in use by the previous kernel
+    const int t = w0 / n_st;
+    const int seg1 = min(w1, (t + 1) * n_st);
+    if (w0 != t * n_st && seg1 < w1) {
+      named_bar_sync(kBarHandoff0, kGemvThreads + 32);
+      const int rows = min(kTileRows, L.N - t * kTileRows);
+      const int c_first = cta_of(t * n_st, W, G), c_last = cta_of((t + 1) * n_st - 1, W, G);
+      float* part = work + (size_t)(blockIdx.x * 2) * MT * kTileRows;
+      for (int i = lane; i < MT * kTileRows; i += 32) part[i] = pbuf[i];
+      __threadfence();
+      __syncwarp();
+      int prev = lane == 0 ? atomicAdd(counters + t, 1) : 0;
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+      if (prev == c_last - c_first) {
+        __threadfence();  // the other contributors' sums are visible past their count
+        for (int i = lane; i < MT * kTileRows; i += 32) {
+          const int m = i / kTileRows, r = i % kTileRows;
+          if (m >= M || r >= rows) continue;
+          float v = 0.f;
+          for (int c = c_first; c <= c_last; ++c) {
+            const int cs = (t == ((c * W) / G) / n_st) ? 0 : 1;
+            v += __ldcg(work + (size_t)(c * 2 + cs) * MT * kTileRows + i);
+          }
+          y[(size_t)m * L.N + t * kTileRows + r] = v;
+        }
+        if (lane == 0) counters[t] = 0;
+      }
+    }
+    __syncthreads();
+    return;
+  }
+
   // ---------------- consumers
-  const int g = threadIdx.x >> 7, r = threadIdx.x & (kTileRows - 1);
+  const int rr = threadIdx.x & (kTileRows - 1);  // row this thread finishes at segment ends
+  // Sidecar: bounds of row rr's list for the first segment, requested before
+  // anything else (the next segment's bounds are fetched one segment ahead).
+  constexpr int kPE = 4;  // entries held in registers per row and segment
+  int pr0 = 0, pr1 = 0;
+  {
+    const int n0 = (w0 / n_st) * kTileRows + rr;
+    if (w0 < w1 && n0 < L.N) {
+      pr0 = __ldg(L.row_ptr + n0);
+      pr1 = __ldg(L.row_ptr + n0 + 1);
+    }
+  }
   // shared-memory codebook (compile-time trip counts: a thread's codebook
   // loads are all in flight together)
   if (MODE == HXQ_MODE_SCALAR8) {
@@ -252,32 +358,24 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   consumer_sync();
 
   const uint32_t lane4 = (uint32_t)lane * 4u;
+  const int q = warp;                                  // piece of the chunk this warp decodes
+  const int q_stage = q >> 2, q_quarter = q & 3;
+  int rs = 0;        // ring slot of the next chunk
+  uint32_t rph = 0;  // its phase parity
   bool waited_ok = true;  // after a timed-out wait the data is garbage but every barrier is still met
 
-  // Sidecar: bounds of this thread's row list for the first segment (the
-  // next segment's bounds are fetched one segment ahead).
-  constexpr int kPE = 4;  // entries per group held in registers (16 per row)
-  int pr0 = 0, pr1 = 0;
-  {
-    const int n0 = (w0 / n_st) * kTileRows + r;
-    if (w0 < w1 && n0 < L.N) {
-      pr0 = __ldg(L.row_ptr + n0);
-      pr1 = __ldg(L.row_ptr + n0 + 1);
-    }
-  }
 
-  for (int seg0 = w0; seg0 < w1;) {  // segments: the CTA's items of one tile
+  for (int seg0 = w0; seg0 < w1;) {  // segments: the CTA's stages of one tile
     const int t = seg0 / n_st;
     const int seg1 = min(w1, (t + 1) * n_st);
     const int rows = min(kTileRows, L.N - t * kTileRows);
-    const int n = t * kTileRows + r;
-    // this group's share of row n's patch entries (p = pr0 + g + 4j), loaded
-    // now and applied at the segment end
+    const int n = t * kTileRows + rr;
+    // row rr's first patch entries, applied at the segment end
     int ek[kPE];
     float ed[kPE];
 #pragma unroll
     for (int j = 0; j < kPE; ++j) {
-      const int p = pr0 + g + kGroups * j;
+      const int p = pr0 + j;
       ek[j] = p < pr1 ? __ldg(L.pk + p) : INT_MAX;
       ed[j] = p < pr1 ? __ldg(L.pd + p) : 0.f;
     }
@@ -288,106 +386,137 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       pr0 = __ldg(L.row_ptr + n + kTileRows);
       pr1 = __ldg(L.row_ptr + n + kTileRows + 1);
     }
-    float2 acc[MT];
+    // sums of 4 rows x MT tokens: even/odd column pairs (paired FMAs) for
+    // up to 2 tokens, one register each beyond
+    typename std::conditional<(MT >= 4), float, float2>::type acc[4][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.f, 0.f);
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc_zero(acc[j][m]);
 
-    // this group's items of the segment: w == w0 + g (mod 4)
-    for (int w = seg0 + ((w0 + g - seg0) % kGroups + kGroups) % kGroups; w < seg1; w += kGroups) {
-      const int i = w - w0, s = i % R;
-      if (waited_ok) waited_ok = mbar_wait(&bar_full[s], (i / R) & 1, abrt);
-      uint4 cur[NP];
+    for (int w = seg0; w < seg1;) {  // chunks
+      const int we = min(w + kChunkStages, seg1);
+      if (waited_ok) waited_ok = mbar_wait(&bar_full[rs], rph, abrt);
+      if (q < (we - w) * 4) {
+        const uint8_t* base = ring + (size_t)rs * SLOT + (size_t)q_stage * NP * rows * 16 +
+                              (MODE == HXQ_MODE_SCALAR8 ? q_quarter * rows * 16 : 0) + lane * 16;
+        const int k0 = (w - t * n_st + q_stage) * kStageK + q_quarter * 16;
+        // All four rows are decoded without a per-row test: in a tile of
+        // fewer than 128 rows the reads past the last row stay inside the
+        // slot (the pieces of a stage are packed at `rows` x 16 bytes) and
+        // their sums are never stored.
+        if (MT == 1) {
+          float xv[16];
+          x16<XF32>(xs, L.Kp, 0, k0, xv);
 #pragma unroll
-      for (int j = 0; j < NP; ++j)
-        cur[j] = r < rows ? *reinterpret_cast<const uint4*>(ring + (size_t)s * SLOT + (j * rows + r) * 16)
-                          : make_uint4(0, 0, 0, 0);
+          for (int j = 0; j < 4; ++j) {
+            float wv[16];
+            decode16<MODE>(smem, base + j * 512, rows, q_quarter, lane4, wv);
+            fma16(acc[j][0], wv, xv);
+          }
+        } else {
+          // several tokens: rows two at a time, so that two rows' weights,
+          // one token's activations and all the sums fit in registers
+#pragma unroll
+          for (int jp = 0; jp < 2; ++jp) {
+            asm volatile("" ::: "memory");
+            float wv0[16], wv1[16];
+            decode16<MODE>(smem, base + (2 * jp) * 512, rows, q_quarter, lane4, wv0);
+            decode16<MODE>(smem, base + (2 * jp + 1) * 512, rows, q_quarter, lane4, wv1);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              if (MT >= 4) asm volatile("" ::: "memory");  // one token's activations live at a time
+              float xv[16];
+              x16<XF32>(xs, L.Kp, m, k0, xv);
+              fma16(acc[2 * jp][m], wv0, xv);
+              fma16(acc[2 * jp + 1][m], wv1, xv);
+            }
+          }
+        }
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_empty[s]);
-
-      const int kst = (w - t * n_st) * kStageK;
-      if (MODE == HXQ_MODE_SCALAR8) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t wd[4] = {cur[c].x, cur[c].y, cur[c].z, cur[c].w};
-          float wv[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const uint32_t a = prmt(wd[j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
-            wv[j] = *reinterpret_cast<const float*>(smem + a);
-          }
-          accumulate16<MT, XF32>(acc, wv, xs, L.Kp, kst + c * 16);
-        }
-      } else {
-        uint32_t wd[13];
-#pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          wd[4 * c] = cur[c].x; wd[4 * c + 1] = cur[c].y; wd[4 * c + 2] = cur[c].z; wd[4 * c + 3] = cur[c].w;
-        }
-        wd[12] = 0;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          float wv[16];
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int j = h * 8 + jj, bit = 12 * j;
-            const uint32_t e8 = (bit & 31) >= 3
-                ? (__funnelshift_r(wd[bit >> 5], wd[(bit >> 5) + 1], (bit & 31) - 3) & 0x7FF8u)
-                : ((wd[bit >> 5] << (3 - (bit & 31))) & 0x7FF8u);
-            const float2 pr = *reinterpret_cast<const float2*>(smem + e8);
-            wv[2 * jj] = pr.x;
-            wv[2 * jj + 1] = pr.y;
-          }
-          accumulate16<MT, XF32>(acc, wv, xs, L.Kp, kst + h * 16);
-        }
-      }
+      if (lane == 0) mbar_arrive(&bar_empty[rs]);
+      if (++rs == R) rs = 0, rph ^= 1;
+      w = we;
     }
 
-    // sidecar corrections of this segment's columns: acc += delta * x[k]
-    {
-      const int ka = (seg0 - t * n_st) * kStageK, kb = (seg1 - t * n_st) * kStageK;
+    // segment end: the warps' sums meet in shared memory
 #pragma unroll
-      for (int j = 0; j < kPE; ++j)
-        if (ek[j] >= ka && ek[j] < kb) add_patch<MT, XF32>(acc, ed[j], xs, L.Kp, ek[j]);
-#pragma unroll 1
-      for (int p = cur0 + g + kGroups * kPE; p < cur1; p += kGroups) {  // rows with > 16 entries
-        const int k = __ldg(L.pk + p);
-        if (k >= ka && k < kb) add_patch<MT, XF32>(acc, __ldg(L.pd + p), xs, L.Kp, k);
-      }
-    }
-
-    // segment end: the 4 groups' sums meet in shared memory
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int m = 0; m < MT; ++m) red[(g * MT + m) * kTileRows + r] = acc[m].x + acc[m].y;
+      for (int m = 0; m < MT; ++m) red[(q * MT + m) * kTileRows + lane + 32 * j] = acc_sum(acc[j][m]);
     consumer_sync();
     const bool full = seg0 == t * n_st && seg1 == (t + 1) * n_st;
-    const int slot = (t == w0 / n_st) ? 0 : 1;
-    float* part = work + (size_t)(blockIdx.x * 2 + slot) * MT * kTileRows;
-    for (int i = threadIdx.x; i < MT * kTileRows; i += kGemvThreads) {
-      const int m = i / kTileRows, rr = i % kTileRows;
-      const float v = red[(0 * MT + m) * kTileRows + rr] + red[(1 * MT + m) * kTileRows + rr] +
-                      red[(2 * MT + m) * kTileRows + rr] + red[(3 * MT + m) * kTileRows + rr];
-      if (full) {
-        if (m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
-      } else {
-        part[i] = v;
+    const bool handoff = !full && seg1 < w1;  // split tile at the start of the range: to the fixup warp
+    const int ka = (seg0 - t * n_st) * kStageK, kb = (seg1 - t * n_st) * kStageK;
+    float vout[(MT * kTileRows + kGemvThreads - 1) / kGemvThreads];
+#pragma unroll
+    for (int u = 0; u < (MT * kTileRows + kGemvThreads - 1) / kGemvThreads; ++u) {
+      const int i = threadIdx.x + u * kGemvThreads;  // i % kTileRows == rr
+      const int m = i / kTileRows;
+      float v = 0.f;
+      if (i < MT * kTileRows) {
+#pragma unroll
+        for (int qq = 0; qq < kConsumerWarps; ++qq) v += red[(qq * MT + m) * kTileRows + rr];
+        // sidecar corrections of this segment's columns: delta * x[m][k]
+#pragma unroll
+        for (int j = 0; j < kPE; ++j)
+          if (ek[j] >= ka && ek[j] < kb) v = fmaf(ed[j], x_at(xs, L.Kp, m, ek[j], XF32), v);
+#pragma unroll 1
+        for (int p = cur0 + kPE; p < cur1; ++p) {  // rows with more entries
+          const int k = __ldg(L.pk + p);
+          if (k >= kb) break;
+          if (k >= ka) v = fmaf(__ldg(L.pd + p), x_at(xs, L.Kp, m, k, XF32), v);
+        }
+        if (full && m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
+        if (handoff) pbuf[i] = v;
       }
+      vout[u] = v;
     }
-    if (!full) {
-      __threadfence();
-      consumer_sync();
+    if (handoff) named_bar_arrive(kBarHandoff0, kGemvThreads + 32);
+    if (!full && !handoff) {
+      // The split tile at the end of the range: this CTA is usually the last
+      // of its contributors to finish. If every other one has already
+      // counted, add their sums straight away; otherwise store this sum,
+      // count, and the last to count adds them all. Either way the tile's
+      // sums are added in CTA order.
       const int c_first = cta_of(t * n_st, W, G), c_last = cta_of((t + 1) * n_st - 1, W, G);
-      if (threadIdx.x == 0) last_flag = atomicAdd(counters + t, 1) == c_last - c_first;
+      const int others = c_last - c_first;
+      if (threadIdx.x == 0) flag_sh = ld_acquire_gpu(counters + t) == others;
       consumer_sync();
-      if (last_flag) {
+      bool last = flag_sh;
+      if (!last) {
+        float* part = work + (size_t)(blockIdx.x * 2 + (t == w0 / n_st ? 0 : 1)) * MT * kTileRows;
+#pragma unroll
+        for (int u = 0; u < (MT * kTileRows + kGemvThreads - 1) / kGemvThreads; ++u) {
+          const int i = threadIdx.x + u * kGemvThreads;
+          if (i < MT * kTileRows) part[i] = vout[u];
+        }
         __threadfence();
-        for (int i = threadIdx.x; i < MT * kTileRows; i += kGemvThreads) {
-          const int m = i / kTileRows, rr = i % kTileRows;
-          if (m >= M || rr >= rows) continue;
+        consumer_sync();
+        if (threadIdx.x == 0) flag_sh = atomicAdd(counters + t, 1) == others;
+        consumer_sync();
+        last = flag_sh;
+      }
+      if (last) {
+        __threadfence();  // the other contributors' sums are visible past their count
+#pragma unroll
+        for (int u = 0; u < (MT * kTileRows + kGemvThreads - 1) / kGemvThreads; ++u) {
+          const int i = threadIdx.x + u * kGemvThreads;
+          const int m = i / kTileRows;
+          if (i >= MT * kTileRows || m >= M || rr >= rows) continue;
           float v = 0.f;
-#pragma unroll 4
-          for (int c = c_first; c <= c_last; ++c) {
-            const int cs = (t == ((c * W) / G) / n_st) ? 0 : 1;
-            v += __ldcg(work + (size_t)(c * 2 + cs) * MT * kTileRows + i);
+          for (int c0 = c_first; c0 <= c_last; c0 += 4) {  // four contributors' loads in flight
+            float pv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = min(c0 + e, c_last);
+              const int cs = (t == ((c * W) / G) / n_st) ? 0 : 1;
+              pv[e] = __ldcg(work + (size_t)(c * 2 + cs) * MT * kTileRows + i);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (c0 + e <= c_last) v += (c0 + e == (int)blockIdx.x) ? vout[u] : pv[e];
           }
           y[(size_t)m * L.N + t * kTileRows + rr] = v;
         }
@@ -405,19 +534,19 @@ template <int MT, bool XF32, int MODE>
 cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
                        cudaStream_t s) {
   const int R = ring_slots(MODE, MT, h.L.Kp, XF32);
-  if (R < kGroups) return cudaErrorInvalidValue;
+  if (R < kMinRing) return cudaErrorInvalidValue;
   const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32);
   auto kern = gemv_kernel<MT, XF32, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int W = h.L.n_tiles * (h.L.Kp / kStageK);
-  return launch_pdl(kern, grid, kGemvThreads + 32, smem, s, h.L, x, y, M, W, R, work, counters, h.d_status);
+  return launch_pdl(kern, grid, kGemvBlock, smem, s, h.L, x, y, M, W, R, work, counters, h.d_status);
 }
 
 template <int MT, int MODE>
 cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
                       cudaStream_t s) {
-  if (ring_slots(MODE, MT, h.L.Kp, true) >= kGroups)
+  if (ring_slots(MODE, MT, h.L.Kp, true) >= kMinRing)
     return launch_cfg<MT, true, MODE>(h, x, y, M, grid, work, counters, s);
   return launch_cfg<MT, false, MODE>(h, x, y, M, grid, work, counters, s);
 }
@@ -428,16 +557,15 @@ cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M,
   if (M <= 1) return launch_mt<1, MODE>(h, x, y, M, grid, work, counters, s);
   if (M <= 2) return launch_mt<2, MODE>(h, x, y, M, grid, work, counters, s);
   if (M <= 4) return launch_mt<4, MODE>(h, x, y, M, grid, work, counters, s);
-  if (M <= 8) return launch_mt<8, MODE>(h, x, y, M, grid, work, counters, s);
-  return launch_mt<16, MODE>(h, x, y, M, grid, work, counters, s);
+  return launch_mt<8, MODE>(h, x, y, M, grid, work, counters, s);
 }
 
-int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
 }  // namespace
 
 bool gemv_supports(const hxq_linear& h, int M) {
-  return M >= 1 && M <= 16 && ring_slots(h.L.mode, mt_of(M), h.L.Kp, false) >= kGroups;
+  return M >= 1 && M <= kGemvMaxM && ring_slots(h.L.mode, mt_of(M), h.L.Kp, false) >= kMinRing;
 }
 
 // Persistent grid: one CTA per SM, fewer when the layer has fewer work items.

@@ -159,18 +159,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete. Gives up after
 // kWaitLimitNs of wall time or as soon as another thread of the CTA has set
 // *abort; on giving up it sets *abort and returns false. A normal launch never
-// comes near the limit (kernels here run for microseconds).
+// comes near the limit (kernels here run for microseconds). A waiter off the
+// critical path passes sleep_ns > 0 to sleep between polls, so that its warp
+// does not take issue slots from the warps doing the work.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      return false;
+    if ((i & 63) == 0) {  // the abort flag and the clock are read now and then, not on every poll
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        return false;
+      }
     }
   }
 }
@@ -290,6 +296,21 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
 // prologue now / wait until the previous kernel's results are visible.
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Load with acquire semantics at GPU scope (pairs with a writer's fence +
+// atomic, e.g. the stream-K arrival counters).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 __device__ __forceinline__ uint4 ldg_stream16(const void* p) {
   uint4 v;

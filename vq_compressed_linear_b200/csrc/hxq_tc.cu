@@ -5,13 +5,17 @@
 // and B = a tile of BN tokens of x, so D = y^T for that tile and lives in
 // tensor memory (TMEM): lane = output feature, column = token.
 //
-//  * A is written by the decoding warps straight from registers into TMEM
+//  * A is written by 16 decoding warps straight from registers into TMEM
 //    with tcgen05.st (the "A from tensor memory" form of tcgen05.mma): the
-//    decoded weights never touch shared or global memory. Thread r of a
-//    decoding warp group owns TMEM lane r = row r of the tile; it reads its
-//    16-byte index pieces (a warp reads 512 contiguous bytes), looks the
-//    indices up in a shared-memory table, substitutes sidecar values, packs
-//    two bf16 per 32-bit TMEM cell and stores 64 weights (one stage) at a time.
+//    decoded weights never touch shared or global memory. Thread r of
+//    decoding group g (4 warps, one per TMEM lane quadrant) owns TMEM lane
+//    r = row r of the tile and columns [16 g, 16 g + 16) of every stage. A
+//    producer warp streams each item's index block (contiguous in the tiled
+//    layout) with TMA bulk copies into a ring of shared-memory slots; the
+//    thread reads its 16 indices from the slot, looks them up in a
+//    shared-memory table, substitutes sidecar values, packs two bf16 per
+//    32-bit TMEM cell and stores them. All decoding warps work on the same
+//    item, so the MMA receives items at an even pace.
 //  * B (x) arrives by TMA into 128-byte-swizzled shared memory, 64 columns of
 //    K per stage; rows past M and columns past K read as zero.
 //  * One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32 in TMEM)
@@ -62,17 +66,19 @@ constexpr int kMaxTokBlocks = 64;                       // token blocks per laun
 constexpr int kMaxContrib = 4;                          // CTAs sharing one tile's K at most
 constexpr int kPrefetchItems = 16;                      // index bytes streamed into L2 this far ahead
 
-// Decoding groups of 4 warps (128 rows each): 4 for bf16 weights, 3 for the
-// hi+mid split, whose decoders need more registers.
-template <int TERMS>
-constexpr int dec_groups() { return TERMS == 1 ? 4 : 3; }
-template <int TERMS>
-constexpr int tc_threads() { return 32 * (kDecWarp0 + 4 * dec_groups<TERMS>()); }
-// Pipeline stages in flight: a multiple of the decoding groups (each slot
-// belongs to one group), as many as shared memory (x slots next to the
-// table) and TMEM (A slots next to the accumulators) allow.
+// Decoding warps: 4 groups of 4 (one warp per TMEM lane quadrant). Every
+// decoding warp takes part in every item: group g decodes columns
+// [16 g, 16 g + 16) of the stage for the 32 rows of its quadrant.
+constexpr int kDecWarps = 16;
+constexpr int kTcThreads = 32 * (kDecWarp0 + kDecWarps);
+constexpr size_t kTcSmemLimit = 226 * 1024;  // dynamic shared memory (the barriers are static)
+
+// x / A pipeline slots, as many as TMEM (accumulators + A slots of 32 columns
+// per term) and shared memory (x slots of BN x 128 bytes) allow.
 template <int BN, int TERMS>
-constexpr int num_slots() { return TERMS == 2 ? 6 : (BN >= 256 ? 4 : 8); }
+constexpr int num_slots() {
+  return TERMS == 2 ? 7 : (BN <= 64 ? 12 : BN <= 128 ? 6 : 4);
+}
 
 __device__ __forceinline__ uint32_t bf16_bits(float f) {
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
@@ -106,9 +112,21 @@ constexpr size_t table_bytes() {
 template <int BN>
 constexpr int num_acc() { return BN <= 128 ? 2 : 1; }
 
+// Index ring: one slot holds one item's index block (all rows of the tile).
+template <int MODE>
+constexpr int idx_slot_bytes() { return (MODE == HXQ_MODE_SCALAR8 ? 4 : 3) * kTileRows * 16; }
+
+template <int BN, int TERMS, int MODE>
+constexpr size_t tc_fixed_bytes() {
+  return table_bytes<MODE, TERMS>() + 1024 /* alignment slack */ + (size_t)num_slots<BN, TERMS>() * BN * 128;
+}
+template <int BN, int TERMS, int MODE>
+constexpr int idx_slots() {
+  return (int)std::min<size_t>(16, (kTcSmemLimit - tc_fixed_bytes<BN, TERMS, MODE>()) / idx_slot_bytes<MODE>());
+}
 template <int BN, int TERMS, int MODE>
 constexpr size_t tc_smem_bytes() {
-  return table_bytes<MODE, TERMS>() + 1024 /* alignment slack */ + (size_t)num_slots<BN, TERMS>() * BN * 128;
+  return tc_fixed_bytes<BN, TERMS, MODE>() + (size_t)idx_slots<BN, TERMS, MODE>() * idx_slot_bytes<MODE>();
 }
 
 // Replace the word at offset j (0..15) of a 16-weight chunk by pw.
@@ -132,25 +150,50 @@ __device__ __forceinline__ int cta_of(int w, int W, int G) {
   return b;
 }
 
+// The 12 index bytes [12 g, 12 g + 12) of a row's 48-byte stage (8 pairs),
+// from the three 16-byte planes of the row in an index slot.
+__device__ __forceinline__ void quarter_words_2d(const uint8_t* p0, int rows, int g, uint32_t (&wd)[4]) {
+  const uint8_t* p1 = p0 + rows * 16;
+  const uint8_t* p2 = p1 + rows * 16;
+  wd[3] = 0;
+  if (g == 0) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p0);
+    wd[0] = v.x; wd[1] = v.y; wd[2] = v.z;
+  } else if (g == 1) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p1);
+    wd[0] = *reinterpret_cast<const uint32_t*>(p0 + 12); wd[1] = v.x; wd[2] = v.y;
+  } else if (g == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p1 + 8);
+    wd[0] = v.x; wd[1] = v.y; wd[2] = *reinterpret_cast<const uint32_t*>(p2);
+  } else {
+    const uint4 v = *reinterpret_cast<const uint4*>(p2);
+    wd[0] = v.y; wd[1] = v.z; wd[2] = v.w;
+  }
+}
+
 template <int BN, int TERMS, int MODE>
-__global__ void __launch_bounds__(tc_threads<TERMS>(), 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
 tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ y, int M, int tok0, int n_tb,
           float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
   constexpr int XSLOT = BN * 128;
   constexpr int kSlots = num_slots<BN, TERMS>();
-  constexpr int kDecGroups = dec_groups<TERMS>();
-  static_assert(kSlots % kDecGroups == 0, "each slot belongs to one decoding group");
+  constexpr int kIS = idx_slots<BN, TERMS, MODE>();
+  constexpr int ISLOT = idx_slot_bytes<MODE>();
+  static_assert(kIS >= 2, "index ring");
   constexpr int TB = (int)table_bytes<MODE, TERMS>();
   constexpr int NACC = num_acc<BN>();
   constexpr int ACOL0 = NACC * BN < 64 ? 64 : NACC * BN;  // first TMEM column of the A slots
   static_assert(ACOL0 + kSlots * 32 * TERMS <= kTmemCols, "TMEM budget");
+  constexpr int NPC = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per row and stage
   // The decode table sits at the start of dynamic shared memory so lookups
   // address it from the array symbol (plain LDS); the x slots follow,
-  // aligned to 1024 bytes for the 128-byte swizzle.
+  // aligned to 1024 bytes for the 128-byte swizzle, then the index ring.
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t xs_pad = (1024u - ((smem_u32(smem) + TB) & 1023u)) & 1023u;
   uint8_t* xs = smem + TB + xs_pad;
+  uint8_t* ring = xs + kSlots * XSLOT;
   __shared__ uint64_t bar_x[kSlots], bar_a[kSlots], bar_empty[kSlots], bar_acc[NACC], bar_dfree[NACC], bar_drain;
+  __shared__ uint64_t bar_ifull[kIS], bar_ifree[kIS];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -165,8 +208,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(&bar_x[i], 1);
-      mbar_init(&bar_a[i], 4);
+      mbar_init(&bar_a[i], kDecWarps);
       mbar_init(&bar_empty[i], 1);
+    }
+    for (int i = 0; i < kIS; ++i) {
+      mbar_init(&bar_ifull[i], 1);
+      mbar_init(&bar_ifree[i], kDecWarps);
     }
     for (int i = 0; i < NACC; ++i) {
       mbar_init(&bar_acc[i], 1);
@@ -183,7 +230,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
   }
   // shared-memory decode table (compile-time trip counts: a thread's
   // codebook loads are all in flight together)
-  constexpr int NT = tc_threads<TERMS>();
+  constexpr int NT = kTcThreads;
   if (MODE == HXQ_MODE_SCALAR8) {
     constexpr int PER = (256 * 32 + NT - 1) / NT;
     float cv[PER];
@@ -228,26 +275,27 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
   if (warp == 0) {
     // ---------------- TMA producer: x tiles
     if (lane == 0) {
-      // the decoders' index bytes: streamed into L2 kPrefetchItems ahead
-      constexpr int NPC = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;
+      // index bytes of later items: streamed into L2 ahead of the index ring
       auto prefetch_item = [&](int i) {
         const int w = w0 + i, t = (w / n_st) % L.n_tiles, st = w % n_st;
         const int rows = min(kTileRows, L.N - t * kTileRows);
         prefetch_l2_bulk(L.idx + piece_offset(L, t, MODE == HXQ_MODE_SCALAR8 ? st * 4 : st, 0, 0),
                          (uint32_t)(NPC * rows * 16));
       };
-      for (int i = 0; i < min(n_items, kPrefetchItems); ++i) prefetch_item(i);
+      for (int i = kIS; i < min(n_items, kIS + kPrefetchItems); ++i) prefetch_item(i);
       pdl_wait();  // x may be the previous kernel's output
-      int issued = 0;
+      int issued = 0, b = 0;
+      uint32_t ph = 0;
       for (int i = 0; i < n_items; ++i) {
-        const int w = w0 + i, b = i % kSlots;
-        const int T = w / n_st, st = w % n_st;
+        const int w = w0 + i;
+        const int T = w / n_st, st = w - T * n_st;
         const int tb = T / L.n_tiles;
-        if (i + kPrefetchItems < n_items) prefetch_item(i + kPrefetchItems);
-        if (!mbar_wait(&bar_empty[b], ((i / kSlots) & 1) ^ 1, abrt)) break;
+        if (i + kIS + kPrefetchItems < n_items) prefetch_item(i + kIS + kPrefetchItems);
+        if (!mbar_wait(&bar_empty[b], ph ^ 1, abrt)) break;
         mbar_arrive_expect_tx(&bar_x[b], XSLOT);
         tma_load_2d(xs + b * XSLOT, &tmx, &bar_x[b], st * kStageK, tok0 + tb * BN);
         ++issued;
+        if (++b == kSlots) b = 0, ph ^= 1;
       }
       if (*abrt) {  // drain the loads this thread issued before leaving
         volatile int never = 0;
@@ -259,9 +307,10 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16<BN>();
-      int seg = -1;
+      int seg = -1, b = 0;
+      uint32_t par = 0;
       for (int i = 0; i < n_items; ++i) {
-        const int w = w0 + i, b = i % kSlots;
+        const int w = w0 + i;
         const bool first = (i == 0) || (w % n_st == 0);
         const bool last = (i == n_items - 1) || ((w + 1) % n_st == 0);
         if (first) {
@@ -269,7 +318,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
           const int u = seg / NACC;
           if (u >= 1 && !mbar_wait(&bar_dfree[seg % NACC], (u - 1) & 1, abrt)) break;
         }
-        const uint32_t par = (i / kSlots) & 1;
         if (!mbar_wait(&bar_x[b], par, abrt) || !mbar_wait(&bar_a[b], par, abrt)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(xs + b * XSLOT);
@@ -285,11 +333,34 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
         }
         tc_commit(&bar_empty[b]);
         if (last) tc_commit(&bar_acc[seg % NACC]);
+        if (++b == kSlots) b = 0, par ^= 1;
       }
       if (*abrt) {  // let issued MMAs finish before TMEM is freed
         volatile int never = 0;
         tc_commit(&bar_drain);
         mbar_wait(&bar_drain, 0, &never);
+      }
+    }
+  } else if (warp == 2) {
+    // ---------------- index producer: the items' index blocks into the ring
+    // (they do not depend on the previous kernel: no wait for it)
+    if (lane == 0) {
+      int issued = 0, s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < n_items; ++i) {
+        if (!mbar_wait(&bar_ifree[s], ph ^ 1, abrt)) break;
+        const int w = w0 + i, T = w / n_st, st = w - T * n_st, t = T % L.n_tiles;
+        const int rows = min(kTileRows, L.N - t * kTileRows);
+        const uint32_t bytes = (uint32_t)(NPC * rows * 16);
+        mbar_arrive_expect_tx(&bar_ifull[s], bytes);
+        bulk_load(ring + (size_t)s * ISLOT,
+                  L.idx + piece_offset(L, t, MODE == HXQ_MODE_SCALAR8 ? st * 4 : st, 0, 0), bytes, &bar_ifull[s]);
+        ++issued;
+        if (++s == kIS) s = 0, ph ^= 1;
+      }
+      if (*abrt) {  // let the copies this thread issued land before the CTA ends
+        volatile int never = 0;
+        for (int i = max(0, issued - kIS); i < issued; ++i) mbar_wait(&bar_ifull[i % kIS], (i / kIS) & 1, &never);
       }
     }
   } else if (warp >= kEpiWarp0 && warp < kDecWarp0) {
@@ -309,7 +380,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
       const int n = t * kTileRows + r;
       const int tok_b = tok0 + tb * BN;           // first token of this block
       const int ntok = min(BN, M - tok_b);
-      if (!mbar_wait(&bar_acc[seg % NACC], (seg / NACC) & 1, abrt)) break;
+      // a whole segment of MMAs away: sleep between polls
+      if (!mbar_wait(&bar_acc[seg % NACC], (seg / NACC) & 1, abrt, 200)) break;
       tc_fence_after();
       const int slot = (T == w0 / n_st) ? 0 : 1;
       float* part = work + ((size_t)(blockIdx.x * 2 + slot) * BN) * kTileRows + r;
@@ -365,137 +437,112 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
       }
     }
   } else if (warp >= kDecWarp0) {
-    // ---------------- decoders
-    const int dg = (warp - kDecWarp0) >> 2;  // decoding group
+    // ---------------- decoders: group g, columns [16 g, 16 g + 16) of every stage
+    const int g = (warp - kDecWarp0) >> 2;
     const int q = warp & 3;                  // TMEM lane quadrant
     const int r = q * 32 + lane;             // row of the tile
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const uint32_t lane4 = (uint32_t)lane * 4u;
-    constexpr int NPC = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per stage
-
-    // index pieces of one item
-    auto load_item = [&](int i, uint4 (&qd)[NPC]) {
-      const int w = w0 + i;
-      const int T = w / n_st, st = w % n_st, t = T % L.n_tiles;
-      const int rows = min(kTileRows, L.N - t * kTileRows);
-#pragma unroll
-      for (int c = 0; c < NPC; ++c) {
-        if (r < rows) {
-          const int chunk = MODE == HXQ_MODE_SCALAR8 ? st * 4 + c : st;
-          const int plane = MODE == HXQ_MODE_SCALAR8 ? 0 : c;
-          qd[c] = ldg_stream16(L.idx + piece_offset(L, t, chunk, plane, r));
-        } else {
-          qd[c] = make_uint4(0, 0, 0, 0);
-        }
-      }
-    };
-    uint4 qc[NPC];
-    if (dg < n_items) load_item(dg, qc);
     // Sidecar cursor over this row's patch list (ascending columns): the
     // next entry's column and value are always already in registers, so an
-    // item without a patch costs one compare per 16 weights.
+    // item without a patch in this quarter costs two compares.
     int cur_T = -1, pp = 0, pe = 0, pkn = INT_MAX;
     float pvn = 0.f;
+    int b = 0, is = 0;         // A / x slot and index slot of the next item
+    uint32_t bph = 0, iph = 0;  // their phase parities
 
-    for (int i = dg; i < n_items; i += kDecGroups) {
-      const int b = i % kSlots;
-      const int w = w0 + i, T = w / n_st, st = w % n_st, t = T % L.n_tiles;
-      // the group's next item loads first: they land while this one decodes
-      uint4 qn[NPC];
-      if (i + kDecGroups < n_items) load_item(i + kDecGroups, qn);
-      const int kst = st * kStageK;
+    for (int i = 0; i < n_items; ++i) {
+      const int w = w0 + i, T = w / n_st, st = w - T * n_st, t = T % L.n_tiles;
+      const int rows = min(kTileRows, L.N - t * kTileRows);
+      // this quarter's index bytes, then the slot goes back to the producer
+      if (!mbar_wait(&bar_ifull[is], iph, abrt)) break;
+      const uint8_t* src = ring + (size_t)is * ISLOT + r * 16;
+      uint32_t wd[4] = {0, 0, 0, 0};
+      if (r < rows) {
+        if (MODE == HXQ_MODE_SCALAR8) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + g * rows * 16);
+          wd[0] = v.x; wd[1] = v.y; wd[2] = v.z; wd[3] = v.w;
+        } else {
+          quarter_words_2d(src, rows, g, wd);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_ifree[is]);
+      if (++is == kIS) is = 0, iph ^= 1;
+
+      const int k0 = st * kStageK + g * 16;
       if (T != cur_T) {  // new tile: position the cursor at this stage
         cur_T = T;
         const int n = t * kTileRows + r;
         pkn = INT_MAX;
         if (n < L.N) {
-          pp = kst == 0 ? __ldg(L.row_ptr + n) : row_lower_bound(L, n, kst);
+          pp = st == 0 ? __ldg(L.row_ptr + n) : row_lower_bound(L, n, k0);
           pe = __ldg(L.row_ptr + n + 1);
           if (pp < pe) { pkn = __ldg(L.pk + pp); pvn = __ldg(L.pv + pp); }
         }
       }
-      while (pkn < kst) {  // entries in other groups' stages
+      while (pkn < k0) {  // entries in other quarters
         ++pp;
         pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
         pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
       }
-      if (!mbar_wait(&bar_empty[b], ((i / kSlots) & 1) ^ 1, abrt)) break;
+      if (!mbar_wait(&bar_empty[b], bph ^ 1, abrt)) break;
       tc_fence_after();
-      const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS;
+      const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS + g * 8;
+      uint32_t hi[8], mid[8];
       if (MODE == HXQ_MODE_SCALAR8) {
+        uint32_t v[16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t wd[4] = {qc[c].x, qc[c].y, qc[c].z, qc[c].w};
-          uint32_t v[16];
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t a = prmt(wd[j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
+          v[j] = *reinterpret_cast<const uint32_t*>(smem + a);
+        }
+        while (pkn < k0 + 16) {  // sidecar: substitute the stored value
+          patch16(v, pkn - k0, TERMS == 1 ? (bf16_bits(pvn) << 16) : split_word(pvn));
+          ++pp;
+          pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
+          pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
+        }
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const uint32_t a = prmt(wd[j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
-            v[j] = *reinterpret_cast<const uint32_t*>(smem + a);
-          }
-          const int k0 = kst + c * 16;
-          while (pkn < k0 + 16) {  // sidecar: substitute the stored value
-            patch16(v, pkn - k0, TERMS == 1 ? (bf16_bits(pvn) << 16) : split_word(pvn));
-            ++pp;
-            pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
-            pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
-          }
-          uint32_t hi[8];
+        for (int j = 0; j < 8; ++j) hi[j] = prmt(v[2 * j], v[2 * j + 1], 0x7632);
+        if (TERMS == 2) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) hi[j] = prmt(v[2 * j], v[2 * j + 1], 0x7632);
-          tmem_st8(acol + c * 8, hi);
-          if (TERMS == 2) {
-            uint32_t mid[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) mid[j] = prmt(v[2 * j], v[2 * j + 1], 0x5410);
-            tmem_st8(acol + 32 + c * 8, mid);
-          }
+          for (int j = 0; j < 8; ++j) mid[j] = prmt(v[2 * j], v[2 * j + 1], 0x5410);
         }
       } else {
-        uint32_t wd[13];
 #pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          wd[4 * c] = qc[c].x; wd[4 * c + 1] = qc[c].y; wd[4 * c + 2] = qc[c].z; wd[4 * c + 3] = qc[c].w;
+        for (int jj = 0; jj < 8; ++jj) {  // 8 pairs = 16 weights
+          const int bit = 12 * jj;
+          const uint32_t e = __funnelshift_r(wd[bit >> 5], wd[(bit >> 5) + 1], bit & 31) & 0xFFF;
+          if (TERMS == 1) {
+            hi[jj] = *reinterpret_cast<const uint32_t*>(smem + e * 4);
+          } else {
+            const uint2 hm = *reinterpret_cast<const uint2*>(smem + e * 8);
+            hi[jj] = hm.x;
+            mid[jj] = hm.y;
+          }
         }
-        wd[12] = 0;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {  // 8 pairs = 16 weights per step
-          uint32_t hi[8], mid[8];
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int j = h * 8 + jj, bit = 12 * j;
-            const uint32_t e = __funnelshift_r(wd[bit >> 5], wd[(bit >> 5) + 1], bit & 31) & 0xFFF;
-            if (TERMS == 1) {
-              hi[jj] = *reinterpret_cast<const uint32_t*>(smem + e * 4);
-            } else {
-              const uint2 hm = *reinterpret_cast<const uint2*>(smem + e * 8);
-              hi[jj] = hm.x;
-              mid[jj] = hm.y;
-            }
+        while (pkn < k0 + 16) {  // sidecar: substitute the stored value
+          const int o = pkn - k0;
+          if (TERMS == 1) {
+            patch8_half(hi, o >> 1, o & 1, bf16_bits(pvn));
+          } else {
+            const uint32_t sw = split_word(pvn);
+            patch8_half(hi, o >> 1, o & 1, sw >> 16);
+            patch8_half(mid, o >> 1, o & 1, sw & 0xFFFFu);
           }
-          const int k0 = kst + h * 16;
-          while (pkn < k0 + 16) {  // sidecar: substitute the stored value
-            const int o = pkn - k0;
-            if (TERMS == 1) {
-              patch8_half(hi, o >> 1, o & 1, bf16_bits(pvn));
-            } else {
-              const uint32_t sw = split_word(pvn);
-              patch8_half(hi, o >> 1, o & 1, sw >> 16);
-              patch8_half(mid, o >> 1, o & 1, sw & 0xFFFFu);
-            }
-            ++pp;
-            pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
-            pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
-          }
-          tmem_st8(acol + h * 8, hi);
-          if (TERMS == 2) tmem_st8(acol + 32 + h * 8, mid);
+          ++pp;
+          pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
+          pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
         }
       }
+      tmem_st8(acol, hi);
+      if (TERMS == 2) tmem_st8(acol + 32, mid);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_a[b]);
-#pragma unroll
-      for (int c = 0; c < NPC; ++c) qc[c] = qn[c];
+      if (++b == kSlots) b = 0, bph ^= 1;
     }
   }
 
@@ -536,7 +583,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
   // at least 116 KB of shared memory keeps one CTA per SM (each CTA takes all
   // 512 TMEM columns)
-  static_assert(tc_smem_bytes<BN, TERMS, MODE>() <= 227 * 1024, "shared memory budget");
+  static_assert(tc_smem_bytes<BN, TERMS, MODE>() <= kTcSmemLimit, "shared memory budget");
   const size_t smem = std::max<size_t>(tc_smem_bytes<BN, TERMS, MODE>(), 116 * 1024);
   auto kern = tc_kernel<BN, TERMS, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -552,7 +599,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
     grid = std::max<int64_t>(1, std::min<int64_t>({grid, (int64_t)h.num_sms, W}));
     if (W * grid >= INT_MAX) return cudaErrorInvalidValue;  // item arithmetic is 32-bit
     if ((size_t)grid * 2 * BN * kTileRows > h.work_floats) return cudaErrorInvalidValue;
-    e = launch_pdl(kern, (unsigned)grid, tc_threads<TERMS>(), smem, st, tm, h.L, y, M, tb0 * BN, n_tb, h.d_work,
+    e = launch_pdl(kern, (unsigned)grid, kTcThreads, smem, st, tm, h.L, y, M, tb0 * BN, n_tb, h.d_work,
                    h.d_counters, h.d_status);
     if (e != cudaSuccess) return e;
   }
