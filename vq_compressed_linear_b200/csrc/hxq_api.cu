@@ -74,6 +74,7 @@ void free_handle(hxq_linear* h) {
   cudaFree(h->d_codebook);
   cudaFree(h->d_idx);
   cudaFree(h->d_row_ptr);
+  cudaFree(h->d_seg_ptr);
   cudaFree(h->d_pk);
   cudaFree(h->d_pv);
   cudaFree(h->d_pd);
@@ -174,6 +175,15 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
     ppos[i] = p;
   }
   for (int n = 0; n < N; ++n) row_ptr[n + 1] += row_ptr[n];
+  const int n_st = L.Kp / hxq::kStageK;
+  std::vector<int> seg_ptr((size_t)(n_st + 1) * N);
+  for (int n = 0; n < N; ++n) {
+    int p = row_ptr[n];
+    for (int st = 0; st <= n_st; ++st) {
+      while (p < row_ptr[n + 1] && pk[p] < st * hxq::kStageK) ++p;
+      seg_ptr[(size_t)st * N + n] = p;
+    }
+  }
 
   const size_t cb_floats = mode == HXQ_MODE_SCALAR8 ? 256 : 8192;
   const size_t idx_bytes = (size_t)N * L.KC * 16 * L.P;
@@ -190,6 +200,7 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   if ((e = dalloc(&h->d_codebook, cb_floats)) != cudaSuccess ||
       (e = dalloc(&h->d_idx, idx_bytes)) != cudaSuccess ||
       (e = dalloc(&h->d_row_ptr, (size_t)N + 1)) != cudaSuccess ||
+      (e = dalloc(&h->d_seg_ptr, seg_ptr.size())) != cudaSuccess ||
       (e = dalloc(&h->d_pk, (size_t)n_sidecar)) != cudaSuccess ||
       (e = dalloc(&h->d_pv, (size_t)n_sidecar)) != cudaSuccess ||
       (e = dalloc(&h->d_pd, (size_t)n_sidecar)) != cudaSuccess ||
@@ -207,6 +218,7 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   L.codebook = h->d_codebook;
   L.idx = h->d_idx;
   L.row_ptr = h->d_row_ptr;
+  L.seg_ptr = h->d_seg_ptr;
   L.pk = h->d_pk;
   L.pv = h->d_pv;
   L.pd = h->d_pd;
@@ -214,6 +226,8 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   if ((e = cudaMemcpy(h->d_codebook, codebook, cb_floats * sizeof(float), cudaMemcpyDefault)) != cudaSuccess ||
       (e = cudaMemcpy(d_src, indices, src_bytes, cudaMemcpyDefault)) != cudaSuccess ||
       (e = cudaMemcpy(h->d_row_ptr, row_ptr.data(), row_ptr.size() * sizeof(int), cudaMemcpyHostToDevice)) !=
+          cudaSuccess ||
+      (e = cudaMemcpy(h->d_seg_ptr, seg_ptr.data(), seg_ptr.size() * sizeof(int), cudaMemcpyHostToDevice)) !=
           cudaSuccess ||
       (n_sidecar > 0 &&
        ((e = cudaMemcpy(h->d_pk, pk.data(), n_sidecar * sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess ||

@@ -40,10 +40,11 @@
 // Sidecar (replacement of single weights, HXQ whitepaper, method section,
 // "Sidecar outlier correction"): replacing w = c by v adds (v - c) x to the
 // dot product, so each entry carries delta = v - c (fp32, computed once when
-// the handle is built). The main loop decodes with the codebook alone; the
-// thread that finishes row n of a segment loads row n's first patch entries
-// when the segment starts (list bounds fetched one segment ahead) and adds
-// delta * x[k] for those in the segment's columns to the row's sum.
+// the handle is built). The main loop decodes with the codebook alone. When a
+// segment starts, the four threads that finish row n load up to four each of
+// the row's entries in the segment's columns (found through a per-stage
+// lower-bound table, the bounds fetched one segment ahead); at the segment
+// end they add delta * x[m][k] to the row's sum.
 #include <algorithm>
 #include <climits>
 #include <type_traits>
@@ -58,11 +59,12 @@ constexpr int kConsumerWarps = kGemvThreads / 32;  // 16: one 16-weight piece of
 constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kFixupWarp = kConsumerWarps + 1;
 constexpr int kGemvBlock = kGemvThreads + 64;
-constexpr int kBarConsumers = 1;                   // named barriers: consumers only,
-constexpr int kBarHandoff0 = 2;                    // consumers -> fixup warp
+constexpr int kBarConsumers = 1;                   // named barrier of the consumers
 constexpr int kChunkStages = 4;                    // stages per ring slot (16 pieces per row)
 constexpr int kMaxRing = 6;                        // ring slots
 constexpr int kGemvMaxM = 8;                       // tokens
+constexpr int kSideGroups = kGemvThreads / kTileRows;  // 4 threads per row share its patch entries
+constexpr int kPE = 4;                             // patch entries per thread and segment in registers
 constexpr size_t kSmemLimit = 226 * 1024;          // dynamic shared memory per CTA (static kept apart)
 
 // Dynamic shared memory of one CTA: codebook table, activations (fp32 or
@@ -70,11 +72,12 @@ constexpr size_t kSmemLimit = 226 * 1024;          // dynamic shared memory per 
 // warp, then the index ring.
 inline size_t gemv_smem_fixed(int mode, int MT, int Kp, bool xf32) {
   return (size_t)(mode == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8) + (size_t)MT * Kp * (xf32 ? 4 : 2) +
-         (size_t)(kConsumerWarps + 1) * MT * kTileRows * sizeof(float);
+         (size_t)(kConsumerWarps + 2 + kSideGroups) * MT * kTileRows * sizeof(float);
 }
 inline int slot_bytes(int mode) { return kChunkStages * (mode == HXQ_MODE_SCALAR8 ? 4 : 3) * kTileRows * 16; }
-// Ring slots that fit next to the fixed part (0 if fewer than two fit).
-constexpr int kMinRing = 2;
+// Ring slots that fit next to the fixed part (0 if none fits; a single slot
+// -- no overlap of copies and decoding -- only happens for 8 tokens).
+constexpr int kMinRing = 1;
 inline int ring_slots(int mode, int MT, int Kp, bool xf32) {
   const size_t fixed = gemv_smem_fixed(mode, MT, Kp, xf32);
   if (fixed + 128 > kSmemLimit) return 0;
@@ -189,6 +192,60 @@ __device__ __forceinline__ void decode16(const uint8_t* smem, const uint8_t* pie
 
 __device__ __forceinline__ void consumer_sync() { named_bar_sync(kBarConsumers, kGemvThreads); }
 
+// The CTA's stage range [w0, w1) as segments (its stages of one tile each),
+// in processing order. A range that ends inside a tile shared with the next
+// CTA processes that split tile first: the next CTA reaches its own part of
+// the tile at the end of its range, so by then this CTA's sum has long been
+// counted, and the CTA that finishes a split tile last finds the other sums
+// ready. Split segments take partial-sum slot 0 (the range's first tile) or
+// 1 (its last tile).
+struct Segments {
+  int w0, w1, n_st, tf, tl, n;
+  bool reorder;
+  __device__ Segments(int w0_, int w1_, int n_st_) : w0(w0_), w1(w1_), n_st(n_st_) {
+    tf = w0 / n_st;
+    tl = (w1 - 1) / n_st;
+    n = tl - tf + 1;
+    reorder = n >= 2 && w1 != (tl + 1) * n_st;
+  }
+  __device__ int tile(int k) const { return reorder ? (k == 0 ? tl : tf + k - 1) : tf + k; }
+  __device__ int begin(int k) const { return max(w0, tile(k) * n_st); }
+  __device__ int end(int k) const { return min(w1, (tile(k) + 1) * n_st); }
+  __device__ bool split(int k) const {
+    const int t = tile(k);
+    return begin(k) != t * n_st || end(k) != (t + 1) * n_st;
+  }
+  __device__ int slot(int k) const { return tile(k) == tf ? 0 : 1; }
+};
+
+// y rows of tile t from the sums of its contributors c_first..c_last, added
+// in CTA order: this CTA's own sum from `own` (shared memory), the others'
+// from the workspace (a batch of contributors' loads in flight per sum).
+template <int MT>
+__device__ __forceinline__ void finish_tile(const Layer& L, float* __restrict__ y, const float* __restrict__ work,
+                                            const float* own, int M, int t, int c_first, int c_last, int W, int G,
+                                            int n_st, int tid, int nthreads) {
+  const int rows = min(kTileRows, L.N - t * kTileRows);
+  for (int i = tid; i < MT * kTileRows; i += nthreads) {
+    const int m = i / kTileRows, r = i % kTileRows;
+    if (m >= M || r >= rows) continue;
+    float v = 0.f;
+    for (int c0 = c_first; c0 <= c_last; c0 += 16) {
+      float q[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int c = min(c0 + e, c_last);
+        const int cs = (t == ((c * W) / G) / n_st) ? 0 : 1;
+        q[e] = __ldcg(work + (size_t)(c * 2 + cs) * MT * kTileRows + i);
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (c0 + e <= c_last) v += c0 + e == (int)blockIdx.x ? own[i] : q[e];
+    }
+    y[(size_t)m * L.N + t * kTileRows + r] = v;
+  }
+}
+
 template <int MT, bool XF32, int MODE>
 __global__ void __launch_bounds__(kGemvBlock, 1)
 gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int W, int R,
@@ -196,20 +253,23 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int TB = table_bytes<MODE>();
   constexpr int NP = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per row and stage
+  constexpr int TS = MT * kTileRows;                    // sums per tile
   uint8_t* xs = smem + TB;
   // per-warp partial sums [kConsumerWarps][MT][kTileRows], after the activations
   float* red = reinterpret_cast<float*>(xs + (size_t)MT * L.Kp * (XF32 ? 4 : 2));
-  float* pbuf = red + kConsumerWarps * MT * kTileRows;  // [MT][kTileRows] sum for the fixup warp
+  float* pbuf = red + kConsumerWarps * TS;  // [2][TS] this CTA's sums of its split tiles (by slot)
+  float* side = pbuf + 2 * TS;              // [kSideGroups][TS] sidecar corrections
   uint8_t* ring = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(pbuf + MT * kTileRows) + 127) & ~(uintptr_t)127);
+      (reinterpret_cast<uintptr_t>(side + kSideGroups * TS) + 127) & ~(uintptr_t)127);
   constexpr int SLOT = kChunkStages * NP * kTileRows * 16;
   __shared__ uint64_t bar_full[kMaxRing], bar_empty[kMaxRing];
+  __shared__ uint64_t bar_handoff[2];  // a split tile's sums (by slot) are in pbuf: consumers -> fixup warp
   __shared__ int abort_sh, flag_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_st = n_stages(L);
   const int G = gridDim.x;
-  const int w0 = (blockIdx.x * W) / G, w1 = ((blockIdx.x + 1) * W) / G;
+  const Segments S((blockIdx.x * W) / G, ((blockIdx.x + 1) * W) / G, n_st);
   volatile int* abrt = &abort_sh;
 
   if (threadIdx.x == 0) {
@@ -217,6 +277,8 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       mbar_init(&bar_full[i], 1);
       mbar_init(&bar_empty[i], kConsumerWarps);  // every consumer warp reads every slot
     }
+    mbar_init(&bar_handoff[0], kConsumerWarps);
+    mbar_init(&bar_handoff[1], kConsumerWarps);
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -224,23 +286,26 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   pdl_launch_dependents();  // the next kernel in the stream may start its prologue
 
   if (warp == kProducerWarp) {
-    // ---------------- producer: the range's chunks, in order
+    // ---------------- producer: the segments' chunks, in processing order
     if (lane == 0) {
       int issued = 0, s = 0;
       uint32_t ph = 0;
-      for (int w = w0; w < w1;) {
-        const int t = w / n_st, st = w - t * n_st;
-        const int we = min(min(w + kChunkStages, (t + 1) * n_st), w1);
-        if (!mbar_wait(&bar_empty[s], ph ^ 1, abrt)) break;
+      for (int k = 0; k < S.n && !*abrt; ++k) {
+        const int t = S.tile(k), seg1 = S.end(k);
         const int rows = min(kTileRows, L.N - t * kTileRows);
-        const uint32_t bytes = (uint32_t)((we - w) * NP * rows * 16);
-        mbar_arrive_expect_tx(&bar_full[s], bytes);
-        bulk_load(ring + (size_t)s * SLOT,
-                  L.idx + (size_t)t * kTileRows * L.KC * 16 * L.P + (size_t)st * NP * rows * 16, bytes,
-                  &bar_full[s]);
-        ++issued;
-        if (++s == R) s = 0, ph ^= 1;
-        w = we;
+        for (int w = S.begin(k); w < seg1;) {
+          const int st = w - t * n_st;
+          const int we = min(w + kChunkStages, seg1);
+          if (!mbar_wait(&bar_empty[s], ph ^ 1, abrt)) break;
+          const uint32_t bytes = (uint32_t)((we - w) * NP * rows * 16);
+          mbar_arrive_expect_tx(&bar_full[s], bytes);
+          bulk_load(ring + (size_t)s * SLOT,
+                    L.idx + (size_t)t * kTileRows * L.KC * 16 * L.P + (size_t)st * NP * rows * 16, bytes,
+                    &bar_full[s]);
+          ++issued;
+          if (++s == R) s = 0, ph ^= 1;
+          w = we;
+        }
       }
       if (*abrt) {  // let the copies this thread issued land before the CTA ends
         volatile int never = 0;
@@ -252,38 +317,27 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   }
 
   if (warp == kFixupWarp) {
-    // ---------------- fixup: a split tile at the start of the CTA's range
-    // that is not also its end (the tail of a tile that earlier CTAs began),
-    // handed over by the consumers so that they never wait on global memory:
-    // store this CTA's sum in the workspace and count it on the tile's
-    // counter. The CTA that counts last (almost never this one: the other
-    // contributors finish their part of the tile at the end of their ranges)
-    // adds all sums in CTA order and writes y.
+    // ---------------- fixup: split tiles processed before the range's last
+    // segment, handed over by the consumers so that they never wait on
+    // global memory: store this CTA's sum in the workspace and count it on
+    // the tile's counter; the last to count (rarely this CTA) adds all sums
+    // in CTA order and writes y.
     pdl_wait();  // y, the workspace and the counters may be in use by the previous kernel
-    const int t = w0 / n_st;
-    const int seg1 = min(w1, (t + 1) * n_st);
-    if (w0 != t * n_st && seg1 < w1) {
-      named_bar_sync(kBarHandoff0, kGemvThreads + 32);
-      const int rows = min(kTileRows, L.N - t * kTileRows);
+    volatile int never = 0;  // the consumers meet every handoff, even after a timed-out wait
+    for (int k = 0; k + 1 < S.n; ++k) {
+      if (!S.split(k)) continue;
+      const int t = S.tile(k), slot = S.slot(k);
+      mbar_wait(&bar_handoff[slot], 0, &never, 64);
       const int c_first = cta_of(t * n_st, W, G), c_last = cta_of((t + 1) * n_st - 1, W, G);
-      float* part = work + (size_t)(blockIdx.x * 2) * MT * kTileRows;
-      for (int i = lane; i < MT * kTileRows; i += 32) part[i] = pbuf[i];
+      float* part = work + (size_t)(blockIdx.x * 2 + slot) * TS;
+      for (int i = lane; i < TS; i += 32) part[i] = pbuf[slot * TS + i];
       __threadfence();
       __syncwarp();
       int prev = lane == 0 ? atomicAdd(counters + t, 1) : 0;
       prev = __shfl_sync(0xffffffffu, prev, 0);
       if (prev == c_last - c_first) {
         __threadfence();  // the other contributors' sums are visible past their count
-        for (int i = lane; i < MT * kTileRows; i += 32) {
-          const int m = i / kTileRows, r = i % kTileRows;
-          if (m >= M || r >= rows) continue;
-          float v = 0.f;
-          for (int c = c_first; c <= c_last; ++c) {
-            const int cs = (t == ((c * W) / G) / n_st) ? 0 : 1;
-            v += __ldcg(work + (size_t)(c * 2 + cs) * MT * kTileRows + i);
-          }
-          y[(size_t)m * L.N + t * kTileRows + r] = v;
-        }
+        finish_tile<MT>(L, y, work, pbuf + slot * TS, M, t, c_first, c_last, W, G, n_st, lane, 32);
         if (lane == 0) counters[t] = 0;
       }
     }
@@ -293,17 +347,21 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
 
   // ---------------- consumers
   const int rr = threadIdx.x & (kTileRows - 1);  // row this thread finishes at segment ends
-  // Sidecar: bounds of row rr's list for the first segment, requested before
-  // anything else (the next segment's bounds are fetched one segment ahead).
-  constexpr int kPE = 4;  // entries held in registers per row and segment
-  int pr0 = 0, pr1 = 0;
-  {
-    const int n0 = (w0 / n_st) * kTileRows + rr;
-    if (w0 < w1 && n0 < L.N) {
-      pr0 = __ldg(L.row_ptr + n0);
-      pr1 = __ldg(L.row_ptr + n0 + 1);
+  const int sg = threadIdx.x / kTileRows;         // its share of the row's patch entries
+  // Sidecar: the bounds of row rr's entries in the first segment's columns,
+  // requested before anything else (those of the next segment are fetched
+  // one segment ahead). Thread sg of the row takes entries
+  // [lo + kPE sg, lo + kPE (sg + 1)).
+  auto seg_bounds = [&](int k, int& lo, int& hi) {
+    const int t = S.tile(k), n = t * kTileRows + rr;
+    lo = hi = 0;
+    if (n < L.N) {
+      lo = __ldg(L.seg_ptr + (size_t)(S.begin(k) - t * n_st) * L.N + n);
+      hi = __ldg(L.seg_ptr + (size_t)(S.end(k) - t * n_st) * L.N + n);
     }
-  }
+  };
+  int pr0, pr1;
+  seg_bounds(0, pr0, pr1);
   // shared-memory codebook (compile-time trip counts: a thread's codebook
   // loads are all in flight together)
   if (MODE == HXQ_MODE_SCALAR8) {
@@ -358,34 +416,28 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   consumer_sync();
 
   const uint32_t lane4 = (uint32_t)lane * 4u;
-  const int q = warp;                                  // piece of the chunk this warp decodes
+  const int q = warp;  // piece of the chunk this warp decodes
   const int q_stage = q >> 2, q_quarter = q & 3;
   int rs = 0;        // ring slot of the next chunk
   uint32_t rph = 0;  // its phase parity
   bool waited_ok = true;  // after a timed-out wait the data is garbage but every barrier is still met
 
-
-  for (int seg0 = w0; seg0 < w1;) {  // segments: the CTA's stages of one tile
-    const int t = seg0 / n_st;
-    const int seg1 = min(w1, (t + 1) * n_st);
+  for (int k = 0; k < S.n; ++k) {
+    const int t = S.tile(k), seg0 = S.begin(k), seg1 = S.end(k);
     const int rows = min(kTileRows, L.N - t * kTileRows);
-    const int n = t * kTileRows + rr;
-    // row rr's first patch entries, applied at the segment end
+    const bool split = S.split(k), last_seg = k + 1 == S.n;
+    // this thread's share of row rr's patch entries in the segment's
+    // columns, applied at the segment end
     int ek[kPE];
     float ed[kPE];
 #pragma unroll
     for (int j = 0; j < kPE; ++j) {
-      const int p = pr0 + j;
-      ek[j] = p < pr1 ? __ldg(L.pk + p) : INT_MAX;
+      const int p = pr0 + kPE * sg + j;
+      ek[j] = p < pr1 ? __ldg(L.pk + p) : -1;
       ed[j] = p < pr1 ? __ldg(L.pd + p) : 0.f;
     }
     const int cur0 = pr0, cur1 = pr1;
-    // next segment's list bounds
-    pr0 = pr1 = 0;
-    if (seg1 < w1 && n + kTileRows < L.N) {
-      pr0 = __ldg(L.row_ptr + n + kTileRows);
-      pr1 = __ldg(L.row_ptr + n + kTileRows + 1);
-    }
+    if (!last_seg) seg_bounds(k + 1, pr0, pr1);  // the next segment's bounds
     // sums of 4 rows x MT tokens: even/odd column pairs (paired FMAs) for
     // up to 2 tokens, one register each beyond
     typename std::conditional<(MT >= 4), float, float2>::type acc[4][MT];
@@ -440,58 +492,69 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       w = we;
     }
 
-    // segment end: the warps' sums meet in shared memory
+    // segment end: sidecar corrections delta * x[m][k] of this thread's
+    // entries (rows with more than kSideGroups * kPE entries in the segment
+    // are rare: the last share walks the rest), then the warps' sums meet in
+    // shared memory
+    {
+      float sp[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) sp[m] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kPE; ++j)
+        if (ek[j] >= 0) {
+#pragma unroll
+          for (int m = 0; m < MT; ++m) sp[m] = fmaf(ed[j], x_at(xs, L.Kp, m, ek[j], XF32), sp[m]);
+        }
+      if (sg == kSideGroups - 1) {
+#pragma unroll 1
+        for (int p = cur0 + kSideGroups * kPE; p < cur1; ++p) {
+          const int kk = __ldg(L.pk + p);
+          const float d = __ldg(L.pd + p);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) sp[m] = fmaf(d, x_at(xs, L.Kp, m, kk, XF32), sp[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) side[(sg * MT + m) * kTileRows + rr] = sp[m];
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int m = 0; m < MT; ++m) red[(q * MT + m) * kTileRows + lane + 32 * j] = acc_sum(acc[j][m]);
     consumer_sync();
-    const bool full = seg0 == t * n_st && seg1 == (t + 1) * n_st;
-    const bool handoff = !full && seg1 < w1;  // split tile at the start of the range: to the fixup warp
-    const int ka = (seg0 - t * n_st) * kStageK, kb = (seg1 - t * n_st) * kStageK;
-    float vout[(MT * kTileRows + kGemvThreads - 1) / kGemvThreads];
-#pragma unroll
-    for (int u = 0; u < (MT * kTileRows + kGemvThreads - 1) / kGemvThreads; ++u) {
-      const int i = threadIdx.x + u * kGemvThreads;  // i % kTileRows == rr
+    const int slot = S.slot(k);
+    for (int i = threadIdx.x; i < TS; i += kGemvThreads) {  // i % kTileRows == rr
       const int m = i / kTileRows;
       float v = 0.f;
-      if (i < MT * kTileRows) {
 #pragma unroll
-        for (int qq = 0; qq < kConsumerWarps; ++qq) v += red[(qq * MT + m) * kTileRows + rr];
-        // sidecar corrections of this segment's columns: delta * x[m][k]
+      for (int qq = 0; qq < kConsumerWarps; ++qq) v += red[(qq * MT + m) * kTileRows + rr];
 #pragma unroll
-        for (int j = 0; j < kPE; ++j)
-          if (ek[j] >= ka && ek[j] < kb) v = fmaf(ed[j], x_at(xs, L.Kp, m, ek[j], XF32), v);
-#pragma unroll 1
-        for (int p = cur0 + kPE; p < cur1; ++p) {  // rows with more entries
-          const int k = __ldg(L.pk + p);
-          if (k >= kb) break;
-          if (k >= ka) v = fmaf(__ldg(L.pd + p), x_at(xs, L.Kp, m, k, XF32), v);
-        }
-        if (full && m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
-        if (handoff) pbuf[i] = v;
+      for (int g = 0; g < kSideGroups; ++g) v += side[(g * MT + m) * kTileRows + rr];
+      if (!split) {
+        if (m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
+      } else {
+        pbuf[slot * TS + i] = v;
       }
-      vout[u] = v;
     }
-    if (handoff) named_bar_arrive(kBarHandoff0, kGemvThreads + 32);
-    if (!full && !handoff) {
-      // The split tile at the end of the range: this CTA is usually the last
-      // of its contributors to finish. If every other one has already
-      // counted, add their sums straight away; otherwise store this sum,
-      // count, and the last to count adds them all. Either way the tile's
+    if (split && !last_seg) {  // to the fixup warp
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_handoff[slot]);
+    }
+    if (split && last_seg) {
+      // The range's last segment is a split tile. If every other contributor
+      // has already counted, add all sums now; otherwise store this CTA's sum
+      // and count, and the last to count adds them. Either way the tile's
       // sums are added in CTA order.
       const int c_first = cta_of(t * n_st, W, G), c_last = cta_of((t + 1) * n_st - 1, W, G);
       const int others = c_last - c_first;
       if (threadIdx.x == 0) flag_sh = ld_acquire_gpu(counters + t) == others;
       consumer_sync();
       bool last = flag_sh;
+      const float* own = pbuf + slot * TS;
       if (!last) {
-        float* part = work + (size_t)(blockIdx.x * 2 + (t == w0 / n_st ? 0 : 1)) * MT * kTileRows;
-#pragma unroll
-        for (int u = 0; u < (MT * kTileRows + kGemvThreads - 1) / kGemvThreads; ++u) {
-          const int i = threadIdx.x + u * kGemvThreads;
-          if (i < MT * kTileRows) part[i] = vout[u];
-        }
+        float* part = work + (size_t)(blockIdx.x * 2 + slot) * TS;
+        for (int i = threadIdx.x; i < TS; i += kGemvThreads) part[i] = own[i];
         __threadfence();
         consumer_sync();
         if (threadIdx.x == 0) flag_sh = atomicAdd(counters + t, 1) == others;
@@ -500,31 +563,11 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       }
       if (last) {
         __threadfence();  // the other contributors' sums are visible past their count
-#pragma unroll
-        for (int u = 0; u < (MT * kTileRows + kGemvThreads - 1) / kGemvThreads; ++u) {
-          const int i = threadIdx.x + u * kGemvThreads;
-          const int m = i / kTileRows;
-          if (i >= MT * kTileRows || m >= M || rr >= rows) continue;
-          float v = 0.f;
-          for (int c0 = c_first; c0 <= c_last; c0 += 4) {  // four contributors' loads in flight
-            float pv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = min(c0 + e, c_last);
-              const int cs = (t == ((c * W) / G) / n_st) ? 0 : 1;
-              pv[e] = __ldcg(work + (size_t)(c * 2 + cs) * MT * kTileRows + i);
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (c0 + e <= c_last) v += (c0 + e == (int)blockIdx.x) ? vout[u] : pv[e];
-          }
-          y[(size_t)m * L.N + t * kTileRows + rr] = v;
-        }
+        finish_tile<MT>(L, y, work, own, M, t, c_first, c_last, W, G, n_st, threadIdx.x, kGemvThreads);
         if (threadIdx.x == 0) counters[t] = 0;
       }
     }
     consumer_sync();
-    seg0 = seg1;
   }
   if (!waited_ok && threadIdx.x == 0) atomicOr(status, kStatusWaitTimeout);
   __syncthreads();

@@ -44,6 +44,10 @@ struct Layer {
   // Sidecar as per-row patch lists: the entries of row n are
   // [row_ptr[n], row_ptr[n+1]), in ascending column order.
   const int* row_ptr;        // [N+1]
+  // seg_ptr[s * N + n]: the first of row n's entries whose column is at
+  // least s * kStageK (s = 0 .. Kp / kStageK), so that a run of stages
+  // finds its entries without a search.
+  const int* seg_ptr;
   const int* pk;             // column k
   const float* pv;           // the replacement value v
   const float* pd;           // v - (codebook value it replaces), rounded to fp32
@@ -68,6 +72,7 @@ struct hxq_linear {
   float* d_codebook;
   uint8_t* d_idx;
   int* d_row_ptr;
+  int* d_seg_ptr;
   int* d_pk;
   float* d_pv;
   float* d_pd;
@@ -307,6 +312,19 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+// Named barrier that also returns whether `v` held in every participating thread.
+__device__ __forceinline__ bool named_bar_and(int id, int threads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %3, 0;\n\t"
+      "barrier.cta.red.and.pred p, %1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(threads), "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
 }
 __device__ __forceinline__ void named_bar_arrive(int id, int threads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
