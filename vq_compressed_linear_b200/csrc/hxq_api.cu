@@ -217,6 +217,7 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   }
   L.codebook = h->d_codebook;
   L.idx = h->d_idx;
+  L.n_side = (int)n_sidecar;
   L.row_ptr = h->d_row_ptr;
   L.seg_ptr = h->d_seg_ptr;
   L.pk = h->d_pk;

@@ -428,13 +428,18 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
     const bool split = S.split(k), last_seg = k + 1 == S.n;
     // this thread's share of row rr's patch entries in the segment's
     // columns, applied at the segment end
+    // (loaded from a valid index whatever the bounds, so that nothing waits
+    // for the loads before the segment end)
     int ek[kPE];
     float ed[kPE];
+    const int pbase = pr0 + kPE * sg, n_mine = min(kPE, pr1 - pbase);
+    if (L.n_side > 0) {
 #pragma unroll
-    for (int j = 0; j < kPE; ++j) {
-      const int p = pr0 + kPE * sg + j;
-      ek[j] = p < pr1 ? __ldg(L.pk + p) : -1;
-      ed[j] = p < pr1 ? __ldg(L.pd + p) : 0.f;
+      for (int j = 0; j < kPE; ++j) {
+        const int p = min(pbase + j, L.n_side - 1);
+        ek[j] = __ldg(L.pk + p);
+        ed[j] = __ldg(L.pd + p);
+      }
     }
     const int cur0 = pr0, cur1 = pr1;
     if (!last_seg) seg_bounds(k + 1, pr0, pr1);  // the next segment's bounds
@@ -502,7 +507,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       for (int m = 0; m < MT; ++m) sp[m] = 0.f;
 #pragma unroll
       for (int j = 0; j < kPE; ++j)
-        if (ek[j] >= 0) {
+        if (j < n_mine) {
 #pragma unroll
           for (int m = 0; m < MT; ++m) sp[m] = fmaf(ed[j], x_at(xs, L.Kp, m, ek[j], XF32), sp[m]);
         }

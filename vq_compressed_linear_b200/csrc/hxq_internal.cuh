@@ -51,6 +51,7 @@ struct Layer {
   const int* pk;             // column k
   const float* pv;           // the replacement value v
   const float* pd;           // v - (codebook value it replaces), rounded to fp32
+  int n_side;                // number of entries
 };
 
 constexpr int kQuads = kTileRows / 32;
