@@ -42,7 +42,8 @@
 //
 // Sidecar (HXQ whitepaper, method section, "Sidecar outlier correction"):
 // each decoding thread keeps a cursor into its row's column-sorted patch list
-// with the next entry already in registers, and substitutes the stored value
+// (placed at a tile's first stage through a per-stage lower-bound table) with
+// the next two entries already requested, and substitutes the stored value
 // (as bf16, or as its hi+mid split) before the store.
 //
 // Every mbarrier wait is bounded (2 s): on timeout the CTA sets a status bit,
@@ -444,10 +445,23 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const uint32_t lane4 = (uint32_t)lane * 4u;
     // Sidecar cursor over this row's patch list (ascending columns): the
-    // next entry's column and value are always already in registers, so an
-    // item without a patch in this quarter costs two compares.
-    int cur_T = -1, pp = 0, pe = 0, pkn = INT_MAX;
-    float pvn = 0.f;
+    // next two entries are always already requested, so an item without a
+    // patch in this quarter costs two compares and stepping past an entry
+    // of another quarter does not wait on memory.
+    int cur_T = -1, pp = 0, pe = 0, pkn = INT_MAX, pk2 = INT_MAX;
+    float pvn = 0.f, pv2 = 0.f;
+    // entry p's column and value, loaded from a valid index whatever p
+    auto fetch = [&](int p, int& k, float& v) {
+      const int pc = min(p, L.n_side - 1);
+      k = __ldg(L.pk + pc);
+      v = __ldg(L.pv + pc);
+    };
+    auto step = [&]() {  // the cursor moves to the next entry
+      ++pp;
+      pkn = pp < pe ? pk2 : INT_MAX;
+      pvn = pv2;
+      if (pp + 1 < pe) fetch(pp + 1, pk2, pv2);
+    };
     int b = 0, is = 0;         // A / x slot and index slot of the next item
     uint32_t bph = 0, iph = 0;  // their phase parities
 
@@ -471,21 +485,21 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
       if (++is == kIS) is = 0, iph ^= 1;
 
       const int k0 = st * kStageK + g * 16;
-      if (T != cur_T) {  // new tile: position the cursor at this stage
+      if (T != cur_T) {  // new tile: position the cursor at this stage (per-stage table)
         cur_T = T;
         const int n = t * kTileRows + r;
         pkn = INT_MAX;
+        pp = pe = 0;
         if (n < L.N) {
-          pp = st == 0 ? __ldg(L.row_ptr + n) : row_lower_bound(L, n, k0);
+          pp = __ldg(L.seg_ptr + (size_t)st * L.N + n);
           pe = __ldg(L.row_ptr + n + 1);
-          if (pp < pe) { pkn = __ldg(L.pk + pp); pvn = __ldg(L.pv + pp); }
+          if (pp < pe) {
+            fetch(pp, pkn, pvn);
+            if (pp + 1 < pe) fetch(pp + 1, pk2, pv2);
+          }
         }
       }
-      while (pkn < k0) {  // entries in other quarters
-        ++pp;
-        pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
-        pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
-      }
+      while (pkn < k0) step();  // entries in other quarters
       if (!mbar_wait(&bar_empty[b], bph ^ 1, abrt)) break;
       tc_fence_after();
       const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS + g * 8;
@@ -499,9 +513,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
         }
         while (pkn < k0 + 16) {  // sidecar: substitute the stored value
           patch16(v, pkn - k0, TERMS == 1 ? (bf16_bits(pvn) << 16) : split_word(pvn));
-          ++pp;
-          pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
-          pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
+          step();
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) hi[j] = prmt(v[2 * j], v[2 * j + 1], 0x7632);
@@ -531,9 +543,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
             patch8_half(hi, o >> 1, o & 1, sw >> 16);
             patch8_half(mid, o >> 1, o & 1, sw & 0xFFFFu);
           }
-          ++pp;
-          pkn = pp < pe ? __ldg(L.pk + pp) : INT_MAX;
-          pvn = pp < pe ? __ldg(L.pv + pp) : 0.f;
+          step();
         }
       }
       tmem_st8(acol, hi);
