@@ -70,22 +70,22 @@ constexpr size_t kSmemLimit = 226 * 1024;          // dynamic shared memory per 
 // Dynamic shared memory of one CTA: codebook table, activations (fp32 or
 // bf16), the warps' partial sums and the split-tile sum handed to the fixup
 // warp, then the index ring.
-inline size_t gemv_smem_fixed(int mode, int MT, int Kp, bool xf32) {
+inline size_t gemv_smem_fixed(int mode, int MT, int Kp, bool xf32, int cs = 0) {
   return (size_t)(mode == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8) + (size_t)MT * Kp * (xf32 ? 4 : 2) +
-         (size_t)(kConsumerWarps + 2 + kSideGroups) * MT * kTileRows * sizeof(float);
+         (size_t)(kConsumerWarps + 2 + kSideGroups + cs) * MT * kTileRows * sizeof(float);
 }
 inline int slot_bytes(int mode) { return kChunkStages * (mode == HXQ_MODE_SCALAR8 ? 4 : 3) * kTileRows * 16; }
 // Ring slots that fit next to the fixed part (0 if none fits; a single slot
 // -- no overlap of copies and decoding -- only happens for 8 tokens).
 constexpr int kMinRing = 1;
-inline int ring_slots(int mode, int MT, int Kp, bool xf32) {
-  const size_t fixed = gemv_smem_fixed(mode, MT, Kp, xf32);
+inline int ring_slots(int mode, int MT, int Kp, bool xf32, int cs = 0) {
+  const size_t fixed = gemv_smem_fixed(mode, MT, Kp, xf32, cs);
   if (fixed + 128 > kSmemLimit) return 0;
   const int fit = std::min(kMaxRing, (int)((kSmemLimit - fixed - 128) / slot_bytes(mode)));
   return fit >= kMinRing ? fit : 0;
 }
-inline size_t gemv_smem(int mode, int MT, int Kp, bool xf32) {
-  return gemv_smem_fixed(mode, MT, Kp, xf32) + 128 + (size_t)ring_slots(mode, MT, Kp, xf32) * slot_bytes(mode);
+inline size_t gemv_smem(int mode, int MT, int Kp, bool xf32, int cs = 0) {
+  return gemv_smem_fixed(mode, MT, Kp, xf32, cs) + 128 + (size_t)ring_slots(mode, MT, Kp, xf32, cs) * slot_bytes(mode);
 }
 
 template <int MODE>
@@ -248,7 +248,7 @@ __device__ __forceinline__ void finish_tile(const Layer& L, float* __restrict__ 
 
 template <int MT, bool XF32, int MODE>
 __global__ void __launch_bounds__(kGemvBlock, 1)
-gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int W, int R,
+gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int W, int R, int cs,
             float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int TB = table_bytes<MODE>();
@@ -259,8 +259,9 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   float* red = reinterpret_cast<float*>(xs + (size_t)MT * L.Kp * (XF32 ? 4 : 2));
   float* pbuf = red + kConsumerWarps * TS;  // [2][TS] this CTA's sums of its split tiles (by slot)
   float* side = pbuf + 2 * TS;              // [kSideGroups][TS] sidecar corrections
+  float* cbuf = side + kSideGroups * TS;    // [cs][TS] the cluster's sums of its tile (rank 0's copy)
   uint8_t* ring = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(side + kSideGroups * TS) + 127) & ~(uintptr_t)127);
+      (reinterpret_cast<uintptr_t>(cbuf + cs * TS) + 127) & ~(uintptr_t)127);
   constexpr int SLOT = kChunkStages * NP * kTileRows * 16;
   __shared__ uint64_t bar_full[kMaxRing], bar_empty[kMaxRing];
   __shared__ uint64_t bar_handoff[2];  // a split tile's sums (by slot) are in pbuf: consumers -> fixup warp
@@ -269,7 +270,18 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_st = n_stages(L);
   const int G = gridDim.x;
-  const Segments S((blockIdx.x * W) / G, ((blockIdx.x + 1) * W) / G, n_st);
+  // Stage range: stream-K (cs == 0), or with cs > 0 rank r of cluster t
+  // takes stages [r n_st / cs, (r + 1) n_st / cs) of tile t.
+  int rw0, rw1;
+  if (cs > 0) {
+    const int t = blockIdx.x / cs, r = blockIdx.x - t * cs;
+    rw0 = t * n_st + (r * n_st) / cs;
+    rw1 = t * n_st + ((r + 1) * n_st) / cs;
+  } else {
+    rw0 = (blockIdx.x * W) / G;
+    rw1 = ((blockIdx.x + 1) * W) / G;
+  }
+  const Segments S(rw0, rw1, n_st);
   volatile int* abrt = &abort_sh;
 
   if (threadIdx.x == 0) {
@@ -283,6 +295,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
     fence_mbar_init();
   }
   __syncthreads();
+  if (cs > 0) cluster_arrive_relaxed();  // (its wait precedes the first access to another CTA's memory)
   pdl_launch_dependents();  // the next kernel in the stream may start its prologue
 
   if (warp == kProducerWarp) {
@@ -312,6 +325,11 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
         for (int i = max(0, issued - R); i < issued; ++i) mbar_wait(&bar_full[i % R], (i / R) & 1, &never);
       }
     }
+    if (cs > 0) {  // the cluster barrier's two phases (see the consumers' segment end)
+      cluster_wait();
+      cluster_arrive_release();
+      cluster_wait();
+    }
     __syncthreads();
     return;
   }
@@ -340,6 +358,11 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
         finish_tile<MT>(L, y, work, pbuf + slot * TS, M, t, c_first, c_last, W, G, n_st, lane, 32);
         if (lane == 0) counters[t] = 0;
       }
+    }
+    if (cs > 0) {  // the cluster barrier's two phases (see the consumers' segment end)
+      cluster_wait();
+      cluster_arrive_release();
+      cluster_wait();
     }
     __syncthreads();
     return;
@@ -529,6 +552,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       for (int m = 0; m < MT; ++m) red[(q * MT + m) * kTileRows + lane + 32 * j] = acc_sum(acc[j][m]);
     consumer_sync();
     const int slot = S.slot(k);
+    if (cs > 0) cluster_wait();  // every CTA of the cluster has started: rank 0's memory may be written
     for (int i = threadIdx.x; i < TS; i += kGemvThreads) {  // i % kTileRows == rr
       const int m = i / kTileRows;
       float v = 0.f;
@@ -538,15 +562,32 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       for (int g = 0; g < kSideGroups; ++g) v += side[(g * MT + m) * kTileRows + rr];
       if (!split) {
         if (m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
+      } else if (cs > 0) {
+        st_cluster_f32(map_to_rank(smem_u32(cbuf + (blockIdx.x % cs) * TS + i), 0), v);
       } else {
         pbuf[slot * TS + i] = v;
       }
     }
-    if (split && !last_seg) {  // to the fixup warp
+    if (cs > 0) {
+      // Cluster split: the ranks' sums of the tile are in rank 0's shared
+      // memory once every thread of the cluster has passed the barrier;
+      // rank 0 adds them in rank order and writes y.
+      cluster_arrive_release();
+      cluster_wait();
+      if (blockIdx.x % cs == 0) {
+        for (int i = threadIdx.x; i < TS; i += kGemvThreads) {
+          const int m = i / kTileRows;
+          float v = 0.f;
+          for (int r = 0; r < cs; ++r) v += cbuf[r * TS + i];
+          if (m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
+        }
+      }
+    }
+    if (split && !last_seg && cs == 0) {  // to the fixup warp
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_handoff[slot]);
     }
-    if (split && last_seg) {
+    if (split && last_seg && cs == 0) {
       // The range's last segment is a split tile. If every other contributor
       // has already counted, add all sums now; otherwise store this CTA's sum
       // and count, and the last to count adds them. Either way the tile's
@@ -578,34 +619,72 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   __syncthreads();
 }
 
+// Cluster split (no global-memory reduction): when the tiles times a
+// cluster size of 2, 4 or 8 fill at least 85 % of the SMs without
+// exceeding them, each tile gets a cluster whose CTAs split its K. Returns
+// the cluster size, or 0 for the stream-K decomposition.
+inline int pick_cluster(const hxq_linear& h, int MT) {
+  if (MT > 4) return 0;
+  const int n_st = h.L.Kp / kStageK;
+  for (int cs : {2, 4, 8}) {
+    const int g = h.L.n_tiles * cs;
+    if (g <= h.num_sms && 100 * g >= 85 * h.num_sms && n_st >= cs) return cs;
+  }
+  return 0;
+}
+
 template <int MT, bool XF32, int MODE>
 cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
-                       cudaStream_t s) {
+                       bool allow_cluster, cudaStream_t s) {
+  auto kern = gemv_kernel<MT, XF32, MODE>;
+  const int W = h.L.n_tiles * (h.L.Kp / kStageK);
+  const int cs = allow_cluster ? pick_cluster(h, MT) : 0;
+  if (cs > 0 && ring_slots(MODE, MT, h.L.Kp, XF32, cs) >= kMinRing) {
+    const int Rc = ring_slots(MODE, MT, h.L.Kp, XF32, cs);
+    const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32, cs);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // all the clusters must fit on the GPU at once, else stream-K
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(h.L.n_tiles * cs);
+    cfg.blockDim = dim3(kGemvBlock);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n_clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&n_clusters, kern, &cfg) == cudaSuccess && n_clusters >= h.L.n_tiles)
+      return launch_pdl_cluster(kern, h.L.n_tiles * cs, kGemvBlock, smem, cs, s, h.L, x, y, M, W, Rc, cs, work,
+                                counters, h.d_status);
+    cudaGetLastError();
+  }
   const int R = ring_slots(MODE, MT, h.L.Kp, XF32);
   if (R < kMinRing) return cudaErrorInvalidValue;
   const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32);
-  auto kern = gemv_kernel<MT, XF32, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int W = h.L.n_tiles * (h.L.Kp / kStageK);
-  return launch_pdl(kern, grid, kGemvBlock, smem, s, h.L, x, y, M, W, R, work, counters, h.d_status);
+  return launch_pdl(kern, grid, kGemvBlock, smem, s, h.L, x, y, M, W, R, 0, work, counters, h.d_status);
 }
 
 template <int MT, int MODE>
 cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
-                      cudaStream_t s) {
+                      bool allow_cluster, cudaStream_t s) {
   if (ring_slots(MODE, MT, h.L.Kp, true) >= kMinRing)
-    return launch_cfg<MT, true, MODE>(h, x, y, M, grid, work, counters, s);
-  return launch_cfg<MT, false, MODE>(h, x, y, M, grid, work, counters, s);
+    return launch_cfg<MT, true, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
+  return launch_cfg<MT, false, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
 }
 
 template <int MODE>
 cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
-                        cudaStream_t s) {
-  if (M <= 1) return launch_mt<1, MODE>(h, x, y, M, grid, work, counters, s);
-  if (M <= 2) return launch_mt<2, MODE>(h, x, y, M, grid, work, counters, s);
-  if (M <= 4) return launch_mt<4, MODE>(h, x, y, M, grid, work, counters, s);
-  return launch_mt<8, MODE>(h, x, y, M, grid, work, counters, s);
+                        bool allow_cluster, cudaStream_t s) {
+  if (M <= 1) return launch_mt<1, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
+  if (M <= 2) return launch_mt<2, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
+  if (M <= 4) return launch_mt<4, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
+  return launch_mt<8, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
 }
 
 int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
@@ -633,8 +712,9 @@ cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M,
   if (grid == 0) return cudaErrorInvalidValue;
   // every CTA writes at most two partial tiles of mt_of(M) x 128 floats
   if ((size_t)grid * 2 * mt_of(M) * kTileRows > h.work_floats) return cudaErrorInvalidValue;
-  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, grid, h.d_work, h.d_counters, s);
-  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, grid, h.d_work, h.d_counters, s);
+  if (h.L.mode == HXQ_MODE_SCALAR8)
+    return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, grid, h.d_work, h.d_counters, split == 0, s);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, grid, h.d_work, h.d_counters, split == 0, s);
 }
 
 }  // namespace hxq
@@ -705,8 +785,8 @@ extern "C" int hxq_linear_forward_noalloc(hxq_linear_t h, const void* x_bf16, fl
   cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)h->L.n_tiles * sizeof(int), s);
   if (e == cudaSuccess) {
     const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-    e = h->L.mode == HXQ_MODE_SCALAR8 ? launch_mode<HXQ_MODE_SCALAR8>(*h, x, y, M, grid, work, counters, s)
-                                      : launch_mode<HXQ_MODE_VQ2D12>(*h, x, y, M, grid, work, counters, s);
+    e = h->L.mode == HXQ_MODE_SCALAR8 ? launch_mode<HXQ_MODE_SCALAR8>(*h, x, y, M, grid, work, counters, true, s)
+                                      : launch_mode<HXQ_MODE_VQ2D12>(*h, x, y, M, grid, work, counters, true, s);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
