@@ -242,3 +242,33 @@ def test_full_size_prefill_sampled_rows(hxq, name, M):
                                      [0, 127, 128, layer["N"] - 1]]))
     y_ref, s = oracle.forward_rows(layer, x, rows)
     assert_within(y[:, rows], y_ref, s, TAU_PREFILL, f"prefill {name} M={M}")
+
+
+def _cluster_shapes(num_sms):
+    """Layer heights whose tile counts select each cluster size (2, 4, 8):
+    tiles x size between 85 % and 100 % of the SMs, last tile partial."""
+    out = []
+    for cs in (2, 4, 8):
+        tiles = num_sms // cs
+        if 100 * tiles * cs >= 85 * num_sms:
+            out.append((cs, tiles * 128 - 37))
+    return out
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gemv_cluster_split_shapes(hxq, mode):
+    """Decode GEMV shapes that run as cluster splits of each tile's K (the
+    ranks' sums meet in distributed shared memory), with sidecar entries and
+    a partial last tile, against the oracle."""
+    import torch
+    num_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    K = 1024
+    for cs, N in _cluster_shapes(num_sms):
+        layer = synthetic.make_layer(mode, N, K, 40 + cs, sidecar_count=N * K // 500)
+        lin = hxq.HelixLinear.from_layer(layer)
+        W = oracle.decode(mode, layer["codebook"], layer["indices"], layer["sidecar_pos"], layer["sidecar_val"], N, K)
+        for M in (1, 2, 4):
+            x = synthetic.activations(M, K, 50 + M)
+            y = run(hxq, lin, x, AUTO)
+            assert_within(y, oracle.forward(x, W), oracle.abs_scale(x, W), TAU_GEMV, f"cluster {cs} N={N} M={M}")
+        lin.close()

@@ -162,6 +162,7 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   h->n_sidecar = n_sidecar;
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
+  for (int& c : h->gemv_cluster) c = -1;
 
   // position order = row-major order: rows, then ascending columns
   std::vector<int> row_ptr((size_t)N + 1, 0), pk((size_t)n_sidecar);

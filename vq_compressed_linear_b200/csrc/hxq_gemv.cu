@@ -619,34 +619,29 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
   __syncthreads();
 }
 
-// Cluster split (no global-memory reduction): when the tiles times a
-// cluster size of 2, 4 or 8 fill at least 85 % of the SMs without
-// exceeding them, each tile gets a cluster whose CTAs split its K. Returns
-// the cluster size, or 0 for the stream-K decomposition.
-inline int pick_cluster(const hxq_linear& h, int MT) {
-  if (MT > 4) return 0;
-  const int n_st = h.L.Kp / kStageK;
-  for (int cs : {2, 4, 8}) {
-    const int g = h.L.n_tiles * cs;
-    if (g <= h.num_sms && 100 * g >= 85 * h.num_sms && n_st >= cs) return cs;
-  }
-  return 0;
-}
-
+// Cluster split (no global-memory reduction): each tile gets a cluster of
+// cs CTAs (2..8) that split its K, for the largest cs whose grid (tiles x cs)
+// fills at least 70 % of the SMs without exceeding them and whose clusters
+// all fit on the GPU at once. 0 = the stream-K decomposition.
 template <int MT, bool XF32, int MODE>
-cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
-                       bool allow_cluster, cudaStream_t s) {
+int pick_cluster(const hxq_linear& h) {
+  int& cached = h.gemv_cluster[(XF32 ? 4 : 0) + (MT <= 1 ? 0 : MT <= 2 ? 1 : MT <= 4 ? 2 : 3)];
+  if (cached >= 0) return cached;
+  cached = 0;
+  if (MT > 4) return 0;
   auto kern = gemv_kernel<MT, XF32, MODE>;
-  const int W = h.L.n_tiles * (h.L.Kp / kStageK);
-  const int cs = allow_cluster ? pick_cluster(h, MT) : 0;
-  if (cs > 0 && ring_slots(MODE, MT, h.L.Kp, XF32, cs) >= kMinRing) {
-    const int Rc = ring_slots(MODE, MT, h.L.Kp, XF32, cs);
+  const int n_st = h.L.Kp / kStageK;
+  for (int cs = 8; cs >= 2; --cs) {
+    const int g = h.L.n_tiles * cs;
+    if (g > h.num_sms || 100 * g < 70 * h.num_sms || n_st < cs) continue;
+    if (ring_slots(MODE, MT, h.L.Kp, XF32, cs) < kMinRing) continue;
     const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32, cs);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    // all the clusters must fit on the GPU at once, else stream-K
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(h.L.n_tiles * cs);
+    cfg.gridDim = dim3(g);
     cfg.blockDim = dim3(kGemvBlock);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
@@ -657,10 +652,28 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n_clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&n_clusters, kern, &cfg) == cudaSuccess && n_clusters >= h.L.n_tiles)
-      return launch_pdl_cluster(kern, h.L.n_tiles * cs, kGemvBlock, smem, cs, s, h.L, x, y, M, W, Rc, cs, work,
-                                counters, h.d_status);
+    if (cudaOccupancyMaxActiveClusters(&n_clusters, kern, &cfg) == cudaSuccess && n_clusters >= h.L.n_tiles) {
+      cached = cs;
+      return cs;
+    }
     cudaGetLastError();
+  }
+  return 0;
+}
+
+template <int MT, bool XF32, int MODE>
+cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
+                       bool allow_cluster, cudaStream_t s) {
+  auto kern = gemv_kernel<MT, XF32, MODE>;
+  const int W = h.L.n_tiles * (h.L.Kp / kStageK);
+  const int cs = allow_cluster ? pick_cluster<MT, XF32, MODE>(h) : 0;
+  if (cs > 0) {
+    const int Rc = ring_slots(MODE, MT, h.L.Kp, XF32, cs);
+    const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32, cs);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl_cluster(kern, h.L.n_tiles * cs, kGemvBlock, smem, cs, s, h.L, x, y, M, W, Rc, cs, work, counters,
+                              h.d_status);
   }
   const int R = ring_slots(MODE, MT, h.L.Kp, XF32);
   if (R < kMinRing) return cudaErrorInvalidValue;

@@ -82,6 +82,9 @@ struct hxq_linear {
   int* d_counters;      // per output tile: arrivals of split-K partials
   int n_counters;
   int* d_status;        // device-side error word (bounded waits that gave up)
+  // GEMV cluster size chosen per (token count class, activation staging):
+  // -1 = not yet chosen, 0 = stream-K
+  mutable int gemv_cluster[8];
 };
 
 namespace hxq {
