@@ -123,6 +123,27 @@ int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M,
 int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M,
                           int kernel, int split_k, void* stream);
 
+/* Output element type for hxq_linear_forward_out. */
+enum {
+    HXQ_OUT_F32 = 0,       /* float                                          */
+    HXQ_OUT_BF16 = 1       /* bfloat16 bits, rounded to nearest even         */
+};
+
+/*
+ * The layer as a drop-in linear module: y[M][N] = x[M][K] . W^T + bias[N]
+ * (HelixLinear replaces nn.Linear, Zamba2-1.2B-HXQ model card, "What is
+ * HelixCode?"; the bias is kept uncompressed). `bias` is a device pointer
+ * to N floats or NULL (no bias); `y` is a device pointer to M*N floats
+ * (HXQ_OUT_F32) or M*N bf16 values (HXQ_OUT_BF16). The sum x . W^T + bias
+ * is formed in fp32 with the numerics of hxq_linear_forward and, for
+ * HXQ_OUT_BF16, rounded to bf16 (round to nearest even) as it is stored.
+ * Kernel choice as hxq_linear_forward. Asynchronous on `stream`.
+ * Returns HXQ_EINVAL for a NULL handle/x/y, M < 1, a misaligned x or an
+ * unknown out_dtype; HXQ_ECUDA if a launch fails.
+ */
+int hxq_linear_forward_out(hxq_linear_t h, const void* x_bf16, const float* bias,
+                           void* y, int out_dtype, int M, void* stream);
+
 /*
  * Test helper: write the decoded fp32 weights W[N][K] (sidecar applied) to
  * the device buffer W_out on `stream`. Bit-exact with the definition above.

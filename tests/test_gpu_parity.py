@@ -272,3 +272,47 @@ def test_gemv_cluster_split_shapes(hxq, mode):
             y = run(hxq, lin, x, AUTO)
             assert_within(y, oracle.forward(x, W), oracle.abs_scale(x, W), TAU_GEMV, f"cluster {cs} N={N} M={M}")
         lin.close()
+
+
+@pytest.mark.parametrize("mode,N,K", [(0, 300, 200), (1, 200, 136), (0, 8512, 2048)])
+@pytest.mark.parametrize("M", [1, 4, 16, 64])
+def test_forward_out_bias_and_bf16(hxq, mode, N, K, M):
+    """hxq_linear_forward_out: y = x.W^T + bias as fp32 (within the kernel's
+    tolerance of the exact value) and as bf16, which must be the
+    round-to-nearest-even of the same kernel's fp32 result, bit for bit."""
+    import torch
+    layer = synthetic.make_layer(mode, N, K, 60, sidecar_count=max(1, N * K // 1000))
+    lin = hxq.HelixLinear.from_layer(layer)
+    W = oracle.decode(mode, layer["codebook"], layer["indices"], layer["sidecar_pos"], layer["sidecar_val"], N, K)
+    x = synthetic.activations(M, K, 61)
+    bias = np.random.default_rng(62).normal(0.0, 0.5, N).astype(np.float32)
+    bias_d = torch.from_numpy(bias).cuda()
+    xd = xdev(x)
+    y32 = lin.forward_out(xd, bias_d, hxq.HXQ_OUT_F32)
+    y16 = lin.forward_out(xd, bias_d, hxq.HXQ_OUT_BF16)
+    ynb = lin.forward_out(xd, None, hxq.HXQ_OUT_F32)
+    torch.cuda.synchronize()
+    lin.check()
+    y32 = y32.cpu().numpy()
+    ynb = ynb.cpu().numpy()
+    y16_bits = y16.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref = oracle.forward(x, W) + bias.astype(np.float64)[None, :]
+    s = oracle.abs_scale(x, W)
+    tau = tau_for(M, AUTO)
+    assert_within(y32, ref, s + np.abs(bias)[None, :], tau, f"fp32+bias M={M}")
+    # no bias: the plain forward
+    assert_within(ynb, oracle.forward(x, W), s, tau, f"no bias M={M}")
+    # bf16: exactly the rounding of this kernel's fp32 value
+    want = (oracle.round_to_bf16(y32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(y16_bits, want), "bf16 output is not the RNE of the fp32 output"
+    lin.close()
+
+
+def test_forward_out_rejects_bad_dtype(hxq):
+    import torch
+    layer = synthetic.scalar_layer(256, 64, 3, sidecar_count=0)
+    lin = hxq.HelixLinear.from_layer(layer)
+    x = xdev(synthetic.activations(1, 64, 3))
+    y = torch.empty((1, 256), dtype=torch.float32, device="cuda")
+    assert hxq.lib.hxq_linear_forward_out(lin.handle, x.data_ptr(), None, y.data_ptr(), 2, 1, None) == hxq.HXQ_EINVAL
+    assert hxq.lib.hxq_linear_forward_out(lin.handle, x.data_ptr(), None, None, 0, 1, None) == hxq.HXQ_EINVAL

@@ -34,6 +34,8 @@ HXQ_ETIMEOUT = -5
 HXQ_KERNEL_AUTO = 0
 HXQ_KERNEL_GEMV = 1
 HXQ_KERNEL_TC = 2
+HXQ_OUT_F32 = 0
+HXQ_OUT_BF16 = 1
 
 _vp, _i, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
 lib.hxq_linear_create.argtypes = [_vp, _vp, _i, _vp, _vp, _i64, _i, _i, ctypes.POINTER(_vp)]
@@ -42,6 +44,8 @@ lib.hxq_linear_forward.argtypes = [_vp, _vp, _vp, _i, _vp]
 lib.hxq_linear_forward.restype = _i
 lib.hxq_linear_forward_ex.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp]
 lib.hxq_linear_forward_ex.restype = _i
+lib.hxq_linear_forward_out.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _vp]
+lib.hxq_linear_forward_out.restype = _i
 lib.hxq_linear_forward_noalloc.argtypes = [_vp, _vp, _vp, _i, _vp]
 lib.hxq_linear_forward_noalloc.restype = _i
 lib.hxq_decode.argtypes = [_vp, _vp, _vp]
@@ -56,8 +60,8 @@ lib.hxq_linear_destroy.restype = None
 lib.hxq_strerror.argtypes = [_i]
 lib.hxq_strerror.restype = ctypes.c_char_p
 
-EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_linear_forward_noalloc",
-            "hxq_decode",
+EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_linear_forward_out",
+            "hxq_linear_forward_noalloc", "hxq_decode",
             "hxq_linear_check", "hxq_linear_info", "hxq_linear_destroy", "hxq_strerror")
 
 
@@ -110,6 +114,11 @@ def hxq_linear_forward(h, x, y, M, stream=None) -> None:
 def hxq_linear_forward_ex(h, x, y, M, kernel, split_k, stream=None) -> None:
     _check(lib.hxq_linear_forward_ex(h, _ptr(x), _ptr(y), int(M), int(kernel), int(split_k),
                                      _stream(stream)), "hxq_linear_forward_ex")
+
+
+def hxq_linear_forward_out(h, x, bias, y, out_dtype, M, stream=None) -> None:
+    _check(lib.hxq_linear_forward_out(h, _ptr(x), _ptr(bias), _ptr(y), int(out_dtype), int(M), _stream(stream)),
+           "hxq_linear_forward_out")
 
 
 def hxq_linear_forward_noalloc(h, x, y, M, stream=None) -> None:
@@ -168,6 +177,17 @@ class HelixLinear:
         return y
 
     __call__ = forward
+
+    def forward_out(self, x, bias=None, out_dtype=HXQ_OUT_F32, y=None, stream=None):
+        """y = x . W^T (+ bias) as float32, or as bfloat16 (rounded to nearest
+        even) with out_dtype=HXQ_OUT_BF16."""
+        import torch
+        M = int(x.shape[0])
+        if y is None:
+            dt = torch.bfloat16 if out_dtype == HXQ_OUT_BF16 else torch.float32
+            y = torch.empty((M, self.N), dtype=dt, device=x.device)
+        hxq_linear_forward_out(self.handle, x, bias, y, out_dtype, M, stream)
+        return y
 
     def forward_host(self, x_host, y_host, x_dev, y_dev, stream=None):
         """End-to-end call on host buffers: copy x (pinned) in, run, copy y out.

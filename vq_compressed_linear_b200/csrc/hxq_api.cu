@@ -263,9 +263,10 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   return HXQ_OK;
 }
 
-int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M, int kernel, int split_k,
-                          void* stream) {
-  if (!h || !x_bf16 || !y || M < 1) return HXQ_EINVAL;
+namespace {
+int forward_impl(hxq_linear_t h, const void* x_bf16, const hxq::Out& out, int M, int kernel, int split_k,
+                 void* stream) {
+  if (!h || !x_bf16 || !out.y || M < 1) return HXQ_EINVAL;
   if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) != 0) return HXQ_EINVAL;
   if (kernel < HXQ_KERNEL_AUTO || kernel > HXQ_KERNEL_TC) return HXQ_EINVAL;
   if (split_k < 0 || split_k > hxq::kMaxSplitK) return HXQ_EINVAL;
@@ -275,9 +276,9 @@ int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M, i
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   cudaError_t e;
   if (kernel == HXQ_KERNEL_GEMV) {
-    e = hxq::launch_gemv(*h, x, y, M, split_k, s);
+    e = hxq::launch_gemv(*h, x, out, M, split_k, s);
   } else {
-    e = hxq::launch_tc(*h, x, y, M, split_k, s);
+    e = hxq::launch_tc(*h, x, out, M, split_k, s);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -285,9 +286,22 @@ int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M, i
   }
   return HXQ_OK;
 }
+}  // namespace
+
+int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M, int kernel, int split_k,
+                          void* stream) {
+  return forward_impl(h, x_bf16, hxq::Out{y, nullptr, 0}, M, kernel, split_k, stream);
+}
 
 int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M, void* stream) {
-  return hxq_linear_forward_ex(h, x_bf16, y, M, HXQ_KERNEL_AUTO, 0, stream);
+  return forward_impl(h, x_bf16, hxq::Out{y, nullptr, 0}, M, HXQ_KERNEL_AUTO, 0, stream);
+}
+
+int hxq_linear_forward_out(hxq_linear_t h, const void* x_bf16, const float* bias, void* y, int out_dtype, int M,
+                           void* stream) {
+  if (out_dtype != HXQ_OUT_F32 && out_dtype != HXQ_OUT_BF16) return HXQ_EINVAL;
+  return forward_impl(h, x_bf16, hxq::Out{y, bias, out_dtype == HXQ_OUT_BF16 ? 1 : 0}, M, HXQ_KERNEL_AUTO, 0,
+                      stream);
 }
 
 int hxq_decode(hxq_linear_t h, float* W_out, void* stream) {

@@ -222,7 +222,7 @@ struct Segments {
 // in CTA order: this CTA's own sum from `own` (shared memory), the others'
 // from the workspace (a batch of contributors' loads in flight per sum).
 template <int MT>
-__device__ __forceinline__ void finish_tile(const Layer& L, float* __restrict__ y, const float* __restrict__ work,
+__device__ __forceinline__ void finish_tile(const Layer& L, const Out& out, const float* __restrict__ work,
                                             const float* own, int M, int t, int c_first, int c_last, int W, int G,
                                             int n_st, int tid, int nthreads) {
   const int rows = min(kTileRows, L.N - t * kTileRows);
@@ -242,13 +242,13 @@ __device__ __forceinline__ void finish_tile(const Layer& L, float* __restrict__ 
       for (int e = 0; e < 16; ++e)
         if (c0 + e <= c_last) v += c0 + e == (int)blockIdx.x ? own[i] : q[e];
     }
-    y[(size_t)m * L.N + t * kTileRows + r] = v;
+    store_out(out, (size_t)m * L.N + t * kTileRows + r, t * kTileRows + r, v);
   }
 }
 
 template <int MT, bool XF32, int MODE>
 __global__ void __launch_bounds__(kGemvBlock, 1)
-gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int M, int W, int R, int cs,
+gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int R, int cs,
             float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int TB = table_bytes<MODE>();
@@ -355,7 +355,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       prev = __shfl_sync(0xffffffffu, prev, 0);
       if (prev == c_last - c_first) {
         __threadfence();  // the other contributors' sums are visible past their count
-        finish_tile<MT>(L, y, work, pbuf + slot * TS, M, t, c_first, c_last, W, G, n_st, lane, 32);
+        finish_tile<MT>(L, out, work, pbuf + slot * TS, M, t, c_first, c_last, W, G, n_st, lane, 32);
         if (lane == 0) counters[t] = 0;
       }
     }
@@ -561,7 +561,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
 #pragma unroll
       for (int g = 0; g < kSideGroups; ++g) v += side[(g * MT + m) * kTileRows + rr];
       if (!split) {
-        if (m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
+        if (m < M && rr < rows) store_out(out, (size_t)m * L.N + t * kTileRows + rr, t * kTileRows + rr, v);
       } else if (cs > 0) {
         st_cluster_f32(map_to_rank(smem_u32(cbuf + (blockIdx.x % cs) * TS + i), 0), v);
       } else {
@@ -579,7 +579,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
           const int m = i / kTileRows;
           float v = 0.f;
           for (int r = 0; r < cs; ++r) v += cbuf[r * TS + i];
-          if (m < M && rr < rows) y[(size_t)m * L.N + t * kTileRows + rr] = v;
+          if (m < M && rr < rows) store_out(out, (size_t)m * L.N + t * kTileRows + rr, t * kTileRows + rr, v);
         }
       }
     }
@@ -609,7 +609,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, float* __restrict__ y, int 
       }
       if (last) {
         __threadfence();  // the other contributors' sums are visible past their count
-        finish_tile<MT>(L, y, work, own, M, t, c_first, c_last, W, G, n_st, threadIdx.x, kGemvThreads);
+        finish_tile<MT>(L, out, work, own, M, t, c_first, c_last, W, G, n_st, threadIdx.x, kGemvThreads);
         if (threadIdx.x == 0) counters[t] = 0;
       }
     }
@@ -662,7 +662,7 @@ int pick_cluster(const hxq_linear& h) {
 }
 
 template <int MT, bool XF32, int MODE>
-cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
+cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, float* work, int* counters,
                        bool allow_cluster, cudaStream_t s) {
   auto kern = gemv_kernel<MT, XF32, MODE>;
   const int W = h.L.n_tiles * (h.L.Kp / kStageK);
@@ -672,7 +672,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
     const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32, cs);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl_cluster(kern, h.L.n_tiles * cs, kGemvBlock, smem, cs, s, h.L, x, y, M, W, Rc, cs, work, counters,
+    return launch_pdl_cluster(kern, h.L.n_tiles * cs, kGemvBlock, smem, cs, s, h.L, x, out, M, W, Rc, cs, work, counters,
                               h.d_status);
   }
   const int R = ring_slots(MODE, MT, h.L.Kp, XF32);
@@ -680,24 +680,24 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
   const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, grid, kGemvBlock, smem, s, h.L, x, y, M, W, R, 0, work, counters, h.d_status);
+  return launch_pdl(kern, grid, kGemvBlock, smem, s, h.L, x, out, M, W, R, 0, work, counters, h.d_status);
 }
 
 template <int MT, int MODE>
-cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
+cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, float* work, int* counters,
                       bool allow_cluster, cudaStream_t s) {
   if (ring_slots(MODE, MT, h.L.Kp, true) >= kMinRing)
-    return launch_cfg<MT, true, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
-  return launch_cfg<MT, false, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
+    return launch_cfg<MT, true, MODE>(h, x, out, M, grid, work, counters, allow_cluster, s);
+  return launch_cfg<MT, false, MODE>(h, x, out, M, grid, work, counters, allow_cluster, s);
 }
 
 template <int MODE>
-cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, float* work, int* counters,
+cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, float* work, int* counters,
                         bool allow_cluster, cudaStream_t s) {
-  if (M <= 1) return launch_mt<1, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
-  if (M <= 2) return launch_mt<2, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
-  if (M <= 4) return launch_mt<4, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
-  return launch_mt<8, MODE>(h, x, y, M, grid, work, counters, allow_cluster, s);
+  if (M <= 1) return launch_mt<1, MODE>(h, x, out, M, grid, work, counters, allow_cluster, s);
+  if (M <= 2) return launch_mt<2, MODE>(h, x, out, M, grid, work, counters, allow_cluster, s);
+  if (M <= 4) return launch_mt<4, MODE>(h, x, out, M, grid, work, counters, allow_cluster, s);
+  return launch_mt<8, MODE>(h, x, out, M, grid, work, counters, allow_cluster, s);
 }
 
 int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
@@ -719,15 +719,15 @@ int gemv_grid(const hxq_linear& h, int split) {
   return (int)grid;
 }
 
-cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M, int split, cudaStream_t s) {
+cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split, cudaStream_t s) {
   if (!gemv_supports(h, M)) return cudaErrorInvalidValue;
   const int grid = gemv_grid(h, split);
   if (grid == 0) return cudaErrorInvalidValue;
   // every CTA writes at most two partial tiles of mt_of(M) x 128 floats
   if ((size_t)grid * 2 * mt_of(M) * kTileRows > h.work_floats) return cudaErrorInvalidValue;
   if (h.L.mode == HXQ_MODE_SCALAR8)
-    return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, grid, h.d_work, h.d_counters, split == 0, s);
-  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, grid, h.d_work, h.d_counters, split == 0, s);
+    return launch_mode<HXQ_MODE_SCALAR8>(h, x, out, M, grid, h.d_work, h.d_counters, split == 0, s);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, out, M, grid, h.d_work, h.d_counters, split == 0, s);
 }
 
 }  // namespace hxq
@@ -798,8 +798,9 @@ extern "C" int hxq_linear_forward_noalloc(hxq_linear_t h, const void* x_bf16, fl
   cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)h->L.n_tiles * sizeof(int), s);
   if (e == cudaSuccess) {
     const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-    e = h->L.mode == HXQ_MODE_SCALAR8 ? launch_mode<HXQ_MODE_SCALAR8>(*h, x, y, M, grid, work, counters, true, s)
-                                      : launch_mode<HXQ_MODE_VQ2D12>(*h, x, y, M, grid, work, counters, true, s);
+    const Out out{y, nullptr, 0};
+    e = h->L.mode == HXQ_MODE_SCALAR8 ? launch_mode<HXQ_MODE_SCALAR8>(*h, x, out, M, grid, work, counters, true, s)
+                                      : launch_mode<HXQ_MODE_VQ2D12>(*h, x, out, M, grid, work, counters, true, s);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();

@@ -3,6 +3,7 @@
 // wrappers for mbarriers, TMA and tcgen05 (sm_100a).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -56,6 +57,14 @@ struct Layer {
 
 constexpr int kQuads = kTileRows / 32;
 
+// Where a forward writes: y[m][n] (+ bias[n]) as fp32, or rounded to bf16
+// (round to nearest even).
+struct Out {
+  void* y;
+  const float* bias;  // [N] fp32, or null
+  int bf16;           // 0: fp32 y, 1: bf16 y
+};
+
 __host__ __device__ inline int n_stages(const Layer& L) { return L.Kp / kStageK; }
 
 __host__ __device__ inline size_t piece_offset(const Layer& L, int t, int c, int p, int r) {
@@ -91,9 +100,9 @@ namespace hxq {
 
 // Launchers (each returns a cudaError_t from the launch).
 cudaError_t launch_decode(const hxq_linear& h, float* W, cudaStream_t s);
-cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, float* y, int M, int split,
+cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split,
                         cudaStream_t s);
-cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, float* y, int M, int split,
+cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split,
                       cudaStream_t s);
 bool gemv_supports(const hxq_linear& h, int M);
 int gemv_grid(const hxq_linear& h, int split);
@@ -326,6 +335,16 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
 // prologue now / wait until the previous kernel's results are visible.
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Stores output element idx (feature n) of a forward.
+__device__ __forceinline__ void store_out(const Out& o, size_t idx, int n, float v) {
+  if (o.bias) v += __ldg(o.bias + n);
+  if (o.bf16) {
+    reinterpret_cast<__nv_bfloat16*>(o.y)[idx] = __float2bfloat16_rn(v);
+  } else {
+    reinterpret_cast<float*>(o.y)[idx] = v;
+  }
+}
 
 // Load with acquire semantics at GPU scope (pairs with a writer's fence +
 // atomic, e.g. the stream-K arrival counters).

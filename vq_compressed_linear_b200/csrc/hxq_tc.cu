@@ -174,7 +174,7 @@ __device__ __forceinline__ void quarter_words_2d(const uint8_t* p0, int rows, in
 
 template <int BN, int TERMS, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
-tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ y, int M, int tok0, int n_tb,
+tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int tok0, int n_tb,
           float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
   constexpr int XSLOT = BN * 128;
   constexpr int kSlots = num_slots<BN, TERMS>();
@@ -396,7 +396,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
           if (r < rows) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (cc + j < ntok) y[(size_t)(tok_b + cc + j) * L.N + n] = __uint_as_float(v[j]);
+              if (cc + j < ntok) store_out(out, (size_t)(tok_b + cc + j) * L.N + n, n, __uint_as_float(v[j]));
           }
         } else {
 #pragma unroll
@@ -430,7 +430,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, float* __restrict__ 
               }
 #pragma unroll
               for (int u = 0; u < 4; ++u)
-                if (j0 + u < ntok) y[(size_t)(tok_b + j0 + u) * L.N + n] = s4[u];
+                if (j0 + u < ntok) store_out(out, (size_t)(tok_b + j0 + u) * L.N + n, n, s4[u]);
             }
           }
           if (lane == 0) counters[T * kQuads + q] = 0;
@@ -579,7 +579,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int BN, int TERMS, int MODE>
-cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid_req, cudaStream_t st) {
+cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid_req, cudaStream_t st) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tm;
@@ -609,7 +609,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
     grid = std::max<int64_t>(1, std::min<int64_t>({grid, (int64_t)h.num_sms, W}));
     if (W * grid >= INT_MAX) return cudaErrorInvalidValue;  // item arithmetic is 32-bit
     if ((size_t)grid * 2 * BN * kTileRows > h.work_floats) return cudaErrorInvalidValue;
-    e = launch_pdl(kern, (unsigned)grid, kTcThreads, smem, st, tm, h.L, y, M, tb0 * BN, n_tb, h.d_work,
+    e = launch_pdl(kern, (unsigned)grid, kTcThreads, smem, st, tm, h.L, out, M, tb0 * BN, n_tb, h.d_work,
                    h.d_counters, h.d_status);
     if (e != cudaSuccess) return e;
   }
@@ -617,12 +617,12 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, float* y, int M, 
 }
 
 template <int MODE>
-cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, float* y, int M, int grid, cudaStream_t st) {
-  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, y, M, grid, st);
-  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, y, M, grid, st);
-  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, y, M, grid, st);
-  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, y, M, grid, st);
-  return launch_cfg<256, 1, MODE>(h, x, y, M, grid, st);
+cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, cudaStream_t st) {
+  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, out, M, grid, st);
+  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, out, M, grid, st);
+  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, out, M, grid, st);
+  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, out, M, grid, st);
+  return launch_cfg<256, 1, MODE>(h, x, out, M, grid, st);
 }
 
 }  // namespace
@@ -631,7 +631,7 @@ size_t tc_workspace_floats(int num_sms) { return (size_t)num_sms * 2 * 256 * kTi
 
 // `split` (when non-zero) sets the persistent grid so that each tile's K is
 // shared by about `split` CTAs; 0 = one CTA per SM.
-cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, float* y, int M, int split, cudaStream_t st) {
+cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split, cudaStream_t st) {
   int grid = 0;
   if (split > 0) {
     const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
@@ -639,8 +639,8 @@ cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, float* y, int M, i
     grid = std::max(1, n_tb * h.L.n_tiles * split);
     grid = std::min(grid, n_tb * h.L.n_tiles * kMaxContrib * 4);
   }
-  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, y, M, grid, st);
-  return launch_mode<HXQ_MODE_VQ2D12>(h, x, y, M, grid, st);
+  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, out, M, grid, st);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, out, M, grid, st);
 }
 
 }  // namespace hxq
