@@ -81,6 +81,8 @@ def test_forward_and_decode_reject_null_handle():
     y = np.zeros(64, np.float32)
     assert m.lib.hxq_linear_forward(None, m._ptr(x), m._ptr(y), 1, None) == m.HXQ_EINVAL
     assert m.lib.hxq_linear_forward_ex(None, m._ptr(x), m._ptr(y), 1, 0, 0, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_linear_forward_out(None, m._ptr(x), None, m._ptr(y), m.HXQ_OUT_F32, 1, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_linear_forward_noalloc(None, m._ptr(x), m._ptr(y), 1, None) == m.HXQ_EINVAL
     assert m.lib.hxq_decode(None, m._ptr(y), None) == m.HXQ_EINVAL
     assert m.lib.hxq_linear_check(None) == m.HXQ_EINVAL
     assert m.lib.hxq_linear_info(None, None, None, None, None) == m.HXQ_EINVAL
