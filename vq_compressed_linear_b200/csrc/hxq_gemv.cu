@@ -4,10 +4,14 @@
 // instead materialises W and calls cuBLAS: HXQ whitepaper, method section,
 // buffered forward path paragraph).
 //
-// Work decomposition (stream-K). The layer's stages (tile of 128 rows x 64
-// weights along K), numbered tile-major, are cut into contiguous ranges of
-// equal length, one per CTA of a persistent grid (one CTA per SM), so every
-// CTA streams the same number of index bytes whatever the layer shape.
+// Work decomposition. The layer's stages (tile of 128 rows x 64 weights along
+// K) are numbered tile-major. Two ways of cutting them, chosen per handle:
+// - cluster split: when some cluster size cs in 2..8 gives one cluster per
+//   tile that fills at least 70 % of the SMs, all clusters resident, tile t
+//   goes to cluster t and rank r of it takes the r-th of cs equal K ranges;
+// - stream-K otherwise: the stages are cut into contiguous ranges of equal
+//   length, one per CTA of a persistent grid (one CTA per SM), so every CTA
+//   streams the same number of index bytes whatever the layer shape.
 //
 // Inside a CTA a producer warp streams the range in chunks of up to 4 stages
 // of one tile (32 KB of scalar indices, contiguous in the tiled layout) with
@@ -21,10 +25,12 @@
 // quarter wavefront of index bytes plus the activations.
 //
 // At each tile boundary of the CTA's range the warps' sums meet in shared
-// memory; a tile covered by one CTA goes straight to y, a tile split between
-// CTAs leaves one fp32 partial per CTA in the workspace and the last CTA to
-// arrive (integer atomic per tile) adds them in CTA order: results are
-// bitwise repeatable.
+// memory. Under the cluster split every rank writes its sums into rank 0's
+// shared memory (distributed shared memory) and, after a cluster barrier,
+// rank 0 adds them in rank order. Under stream-K a tile covered by one CTA
+// goes straight to y; a tile split between CTAs leaves one fp32 partial per
+// CTA in the workspace and the last CTA to arrive (integer atomic per tile)
+// adds them in CTA order. Either way results are bitwise repeatable.
 //
 // Scalar codebook in shared memory: replicated once per lane with entry e of
 // lane l at byte e*256 + l*4, so the 32 lanes of a lookup always hit 32
