@@ -91,6 +91,21 @@ def workload(name, seed=0, M_override=None):
 
 DEFAULT_M = {"mamba2": None, "tiny": 1, "qwen25_3b": 1, "vq2d": 1, "prefill": 2048}
 
+# Layers of a workload that read the same activations (grouped runs: one
+# hxq_group_forward per group): attention q, k, v and MLP gate, up.
+SHARED_INPUT = {"qwen25_3b": [("q", "k", "v"), ("gate", "up")]}
+
+
+def item_groups(name, items):
+    """Index tuples of the items that share their input, per SHARED_INPUT."""
+    names = [lbl.split("/")[0] for lbl, _, _ in items]
+    out = []
+    for grp in SHARED_INPUT.get(name, []):
+        idx = tuple(names.index(n) for n in grp if n in names)
+        if len(idx) > 1:
+            out.append(idx)
+    return out
+
 
 # ----------------------------------------------------------------------------- clocks
 
@@ -172,23 +187,33 @@ def dominant_kernel(layer, M):
         ("scalar" if layer["mode"] == synthetic.MODE_SCALAR8 else "vq2d")
 
 
-def time_workload(hxq, torch, items, steps, warmup, l2_bytes, stream, soak_s=0.0, max_replica_bytes=48 << 30):
-    """Device time of `steps` steps (CUDA graph, rotating replicas).
+def time_workload(hxq, torch, items, steps, warmup, l2_bytes, stream, soak_s=0.0, max_replica_bytes=48 << 30,
+                  groups=()):
+    """Device time of `steps` steps (CUDA graph, rotating replicas). `groups`
+    (index tuples into items) run as one grouped forward each, on one shared x.
     Returns (ms total, bytes per step, flops per step, launches per step, replicas)."""
     step_bytes = sum(layer_bytes(l, M) for _, l, M in items)
+    # a group reads its activations once
+    step_bytes -= sum(2 * items[j][2] * items[j][1]["K"] for g in groups for j in g[1:])
+    grouped = {j for g in groups for j in g}
     step_flops = sum(layer_flops(l, M) for _, l, M in items)
     dev_bytes_step = sum(l["indices"].size + 8 * l["sidecar_pos"].size for _, l, _ in items)
     R = max(1, math.ceil(4 * l2_bytes / max(1, dev_bytes_step)))
     R = min(R, max(1, max_replica_bytes // max(1, dev_bytes_step)), steps + warmup)
-    reps = []
+    reps, greps = [], []
     for _ in range(R):
-        reps.append([hxq.HelixLinear.from_layer(l) for _, l, _ in items])
+        lins = [hxq.HelixLinear.from_layer(l) for _, l, _ in items]
+        reps.append(lins)
+        greps.append([hxq.HelixGroup([lins[j] for j in g]) for g in groups])
     xs = [torch.from_numpy(synthetic.activations(M, l["K"], 1).view(np.int16)).cuda() for _, l, M in items]
     ys = [torch.empty((M, l["N"]), dtype=torch.float32, device="cuda") for _, l, M in items]
 
     def step(i):
+        for gi, g in enumerate(groups):
+            greps[i % R][gi].forward(xs[g[0]], ys=[ys[j] for j in g], stream=stream)
         for j, lin in enumerate(reps[i % R]):
-            lin.forward(xs[j], ys[j], stream=stream)
+            if j not in grouped:
+                lin.forward(xs[j], ys[j], stream=stream)
 
     with torch.cuda.stream(stream):
         step(0)  # first launches set kernel attributes outside capture
@@ -218,23 +243,37 @@ def time_workload(hxq, torch, items, steps, warmup, l2_bytes, stream, soak_s=0.0
     for lin in reps[0]:
         lin.check()
     del g_warm, g_run
+    for grep in greps:
+        for grp in grep:
+            grp.close()
     for rep in reps:
         for lin in rep:
             lin.close()
-    return ms, step_bytes, step_flops, len(items), R
+    return ms, step_bytes, step_flops, len(items) - len(grouped) + len(groups), R
 
 
-def e2e_workload(hxq, torch, items, steps, warmup, stream):
+def e2e_workload(hxq, torch, items, steps, warmup, stream, groups=()):
     """Same metric through HelixLinear.forward_host semantics: pinned host x
-    in, y out, every step. Returns (ms, h2d bytes/step, d2h bytes/step)."""
+    in, y out, every step (one x per group for `groups`). Returns (ms, h2d
+    bytes/step, d2h bytes/step)."""
     lins = [hxq.HelixLinear.from_layer(l) for _, l, _ in items]
+    grps = [hxq.HelixGroup([lins[j] for j in g]) for g in groups]
+    grouped = {j for g in groups for j in g}
+    skip_x = {j for g in groups for j in g[1:]}
     xh = [torch.from_numpy(synthetic.activations(M, l["K"], 2).view(np.int16)).pin_memory() for _, l, M in items]
     yh = [torch.empty((M, l["N"]), dtype=torch.float32).pin_memory() for _, l, M in items]
     xd = [torch.empty_like(x, device="cuda") for x in xh]
     yd = [torch.empty_like(y, device="cuda") for y in yh]
 
     def step():
+        for gi, g in enumerate(groups):
+            xd[g[0]].copy_(xh[g[0]], non_blocking=True)
+            grps[gi].forward(xd[g[0]], ys=[yd[j] for j in g], stream=stream)
+            for j in g:
+                yh[j].copy_(yd[j], non_blocking=True)
         for j, lin in enumerate(lins):
+            if j in grouped:
+                continue
             xd[j].copy_(xh[j], non_blocking=True)
             lin.forward(xd[j], yd[j], stream=stream)
             yh[j].copy_(yd[j], non_blocking=True)
@@ -250,9 +289,11 @@ def e2e_workload(hxq, torch, items, steps, warmup, stream):
         e1.record(stream)
         e1.synchronize()
     ms = e0.elapsed_time(e1)
+    for grp in grps:
+        grp.close()
     for lin in lins:
         lin.close()
-    h2d = sum(x.numel() * 2 for x in xh)
+    h2d = sum(x.numel() * 2 for j, x in enumerate(xh) if j not in skip_x)
     d2h = sum(y.numel() * 4 for y in yh)
     return ms, h2d, d2h
 
@@ -377,6 +418,8 @@ def main():
     ap.add_argument("--workload", default="mamba2", choices=list(synthetic.CONFIGS))
     ap.add_argument("--M", type=int, default=None, help="token count (default: the workload's bench M)")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--grouped", action="store_true",
+                    help="run the layers that share their input as one grouped forward each")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true",
                     help="minimal run for profilers: enough layer replicas to exceed L2, then "
@@ -394,6 +437,9 @@ def main():
     unit = "TFLOP/s" if is_prefill else "GB/s"
     wl_name = {"mamba2": "mamba2_1.3b_decode_scalar8_M1 (in_proj 8512x2048 + out_proj 2048x4096)"}.get(
         args.workload, args.workload + ":" + ",".join(lbl for lbl, _, _ in items))
+    if args.grouped:
+        wl_name += " grouped " + "|".join(",".join(items[j][0].split("/")[0] for j in g)
+                                          for g in item_groups(args.workload, items))
 
     if args.impl == "reference":
         if rank != 0:
@@ -435,7 +481,8 @@ def main():
     with ClockSampler(local_rank) as clk:
         barrier()
         ms, step_bytes, step_flops, launches, R = time_workload(
-            hxq, torch, items, args.steps, args.warmup, l2, stream, soak_s=1.5)
+            hxq, torch, items, args.steps, args.warmup, l2, stream, soak_s=1.5,
+            groups=item_groups(args.workload, items) if args.grouped else ())
         barrier()
     clocks = clk.summary()
     ms_max = max_over_ranks(torch, dist, world, ms, "cuda")
@@ -443,7 +490,8 @@ def main():
     value = job_rate(units, args.steps, world, ms_max, scale)
 
     # e2e through the public call, host buffers
-    e_ms, h2d, d2h = e2e_workload(hxq, torch, items, args.steps, args.warmup, stream)
+    e_ms, h2d, d2h = e2e_workload(hxq, torch, items, args.steps, args.warmup, stream,
+                                  groups=item_groups(args.workload, items) if args.grouped else ())
     e_ms = max_over_ranks(torch, dist, world, e_ms, "cuda")
     e_val = job_rate(units, args.steps, world, e_ms, scale)
 
@@ -480,19 +528,22 @@ def main():
 
     if not args.no_secondary and world == 1:
         sec = []
-        for wl in ("qwen25_3b", "vq2d", "prefill"):
-            for M in synthetic.CONFIGS[wl][0][4]:
-                its = workload(wl, 0, M)
-                s_ms, sb, sf, sl, sR = time_workload(hxq, torch, its, 20, 3, l2, stream)
-                pre = M > 32
-                v = (sf * 20 / (s_ms * 1e-3) / 1e12) if pre else (sb * 20 / (s_ms * 1e-3) / 1e9)
-                pkv = float(pk["bf16_tflops"]) if pre else float(pk["hbm_gbs"])
-                # roofline time: slower of bytes at HBM peak and flops at tensor peak
-                t_roof = max(sb / (float(pk["hbm_gbs"]) * 1e9), sf / (float(pk["bf16_tflops"]) * 1e12))
-                sec.append({"workload": f"{wl} M={M}", "value": round(v, 1), "unit": "TFLOP/s" if pre else "GB/s",
-                            "frac_of_peak": round(v / pkv, 3),
-                            "frac_of_roofline": round(t_roof / (s_ms * 1e-3 / 20), 3),
-                            "us_per_step": round(s_ms * 1e3 / 20, 2), "launches_per_step": sl})
+        runs = [(wl, M, False) for wl in ("qwen25_3b", "vq2d", "prefill") for M in synthetic.CONFIGS[wl][0][4]]
+        runs.insert(1, ("qwen25_3b", 1, True))  # q|k|v and gate|up as grouped forwards
+        for wl, M, grp in runs:
+            its = workload(wl, 0, M)
+            s_ms, sb, sf, sl, sR = time_workload(hxq, torch, its, 20, 3, l2, stream,
+                                                 groups=item_groups(wl, its) if grp else ())
+            pre = M > 32
+            v = (sf * 20 / (s_ms * 1e-3) / 1e12) if pre else (sb * 20 / (s_ms * 1e-3) / 1e9)
+            pkv = float(pk["bf16_tflops"]) if pre else float(pk["hbm_gbs"])
+            # roofline time: slower of bytes at HBM peak and flops at tensor peak
+            t_roof = max(sb / (float(pk["hbm_gbs"]) * 1e9), sf / (float(pk["bf16_tflops"]) * 1e12))
+            sec.append({"workload": f"{wl} M={M}" + (" grouped" if grp else ""), "value": round(v, 1),
+                        "unit": "TFLOP/s" if pre else "GB/s",
+                        "frac_of_peak": round(v / pkv, 3),
+                        "frac_of_roofline": round(t_roof / (s_ms * 1e-3 / 20), 3),
+                        "us_per_step": round(s_ms * 1e3 / 20, 2), "launches_per_step": sl})
         line["secondary"] = sec
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

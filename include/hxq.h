@@ -45,6 +45,7 @@ extern "C" {
 #endif
 
 typedef struct hxq_linear* hxq_linear_t;
+typedef struct hxq_group* hxq_group_t;
 
 enum {
     HXQ_MODE_SCALAR8 = 0, /* 256 x fp32 codebook, one uint8 index per weight */
@@ -143,6 +144,60 @@ enum {
  */
 int hxq_linear_forward_out(hxq_linear_t h, const void* x_bf16, const float* bias,
                            void* y, int out_dtype, int M, void* stream);
+
+/* Most layers in one group (hxq_group_create). */
+enum { HXQ_MAX_GROUP = 4 };
+
+/*
+ * A group of layers that read the same activations -- the query, key and
+ * value projections of an attention block, the gate and up projections of an
+ * MLP -- so that one launch runs them all. Every compressed weight tensor is
+ * its own layer with its own codebook and sidecar (HXQ whitepaper, method
+ * section: the pipeline runs independently on each tensor, "Per-tensor
+ * k-means"); the pages' forward decompresses and multiplies one module at a
+ * time and pays a fixed cost for each (HXQ whitepaper, the profiling
+ * paragraph after the buffered forward path: 0.93 ms per module against
+ * 0.39 ms for the matmul alone). At decode sizes a small projection (a key
+ * or value projection of 256 x 2048 with 2 KV heads, Qwen2.5-3B-Instruct-HXQ
+ * model card, "Compression Benchmark") reads half a megabyte, under 0.1 us
+ * at full HBM bandwidth, against the microseconds a launch of its own takes
+ * to start, stage its codebook and drain; in a group it shares one grid with
+ * its neighbours.
+ *
+ *  layers    n_layers handles, 1 <= n_layers <= HXQ_MAX_GROUP, pairwise
+ *            distinct, all of one mode and one K, created on one device
+ *  out       receives the group
+ *
+ * The group refers to the handles without owning or copying them: they must
+ * outlive it. Returns HXQ_EINVAL for a NULL array, handle or out, n_layers
+ * outside 1..HXQ_MAX_GROUP, a repeated handle, mixed modes, mixed K or mixed
+ * devices; HXQ_ENOMEM if the small host object cannot be allocated.
+ */
+int hxq_group_create(const hxq_linear_t* layers, int n_layers, hxq_group_t* out);
+
+/*
+ * For every layer i of the group: y[i] = x . W_i^T + bias[i], [M][N_i], with
+ * the output types and numerics of hxq_linear_forward_out.
+ *
+ *  x       device pointer, bf16 [M][K], 16-byte aligned, read by all layers
+ *  bias    host array of n_layers device pointers (N_i floats each, or NULL
+ *          for none), or NULL for no bias on any layer
+ *  y       host array of n_layers device pointers (M*N_i floats or bf16
+ *          values, by out_dtype); the outputs must not overlap
+ *
+ * For M <= 4 (the CUDA-core GEMV) the layers run in one launch, each on a
+ * share of the grid in proportion to its weights; above, each layer runs its
+ * own kernel in turn on `stream`, as hxq_linear_forward_out would. A group
+ * forward uses its layers' workspaces: it must not overlap in time on the GPU
+ * with another forward of any of them. Asynchronous on `stream`.
+ * Returns HXQ_EINVAL for a NULL group, x, y or y[i], M < 1, a misaligned x or
+ * an unknown out_dtype; HXQ_ECUDA if a launch fails.
+ */
+int hxq_group_forward(hxq_group_t g, const void* x_bf16, const float* const* bias,
+                      void* const* y, int out_dtype, int M, void* stream);
+
+/* Free a group (NULL is ignored); its layers are untouched. */
+void hxq_group_destroy(hxq_group_t g);
 
 /*
  * Test helper: write the decoded fp32 weights W[N][K] (sidecar applied) to

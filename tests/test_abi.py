@@ -89,6 +89,22 @@ def test_forward_and_decode_reject_null_handle():
     m.lib.hxq_linear_destroy(None)  # ignored
 
 
+def test_group_entry_points_reject_null_arguments():
+    import ctypes
+    import vq_compressed_linear_b200 as m
+    g = ctypes.c_void_p()
+    none2 = (ctypes.c_void_p * 2)(None, None)
+    assert m.lib.hxq_group_create(None, 1, ctypes.byref(g)) == m.HXQ_EINVAL
+    assert m.lib.hxq_group_create(none2, 2, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_group_create(none2, 2, ctypes.byref(g)) == m.HXQ_EINVAL   # NULL handles
+    assert g.value is None                                                      # *out cleared
+    for n in (0, -1, m.HXQ_MAX_GROUP + 1):
+        assert m.lib.hxq_group_create(none2, n, ctypes.byref(g)) == m.HXQ_EINVAL
+    x = np.zeros(64, np.uint16)
+    assert m.lib.hxq_group_forward(None, m._ptr(x), None, none2, m.HXQ_OUT_F32, 1, None) == m.HXQ_EINVAL
+    m.lib.hxq_group_destroy(None)  # ignored
+
+
 def test_create_without_device_reports_unsupported():
     import torch
     if torch.cuda.is_available():

@@ -99,3 +99,15 @@ def test_reference_arm_line_rank0():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["value"] > 0
+
+
+def test_item_groups_pick_layers_sharing_input():
+    """Grouped runs: q, k, v and gate, up of the Qwen2.5-3B set share their
+    input; other workloads have no groups."""
+    sys.path.insert(0, ROOT)
+    import bench
+    items = [(f"{n}/M=1", None, 1) for n in ("q", "k", "v", "o", "gate", "up", "down")]
+    assert bench.item_groups("qwen25_3b", items) == [(0, 1, 2), (4, 5)]
+    assert bench.item_groups("mamba2", [("in_proj/M=1", None, 1), ("out_proj/M=1", None, 1)]) == []
+    # a group with one member left is no group
+    assert bench.item_groups("qwen25_3b", [("q/M=1", None, 1), ("o/M=1", None, 1)]) == []

@@ -36,6 +36,7 @@ HXQ_KERNEL_GEMV = 1
 HXQ_KERNEL_TC = 2
 HXQ_OUT_F32 = 0
 HXQ_OUT_BF16 = 1
+HXQ_MAX_GROUP = 4
 
 _vp, _i, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
 lib.hxq_linear_create.argtypes = [_vp, _vp, _i, _vp, _vp, _i64, _i, _i, ctypes.POINTER(_vp)]
@@ -55,13 +56,19 @@ lib.hxq_linear_check.restype = _i
 lib.hxq_linear_info.argtypes = [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i),
                                 ctypes.POINTER(_i64)]
 lib.hxq_linear_info.restype = _i
+lib.hxq_group_create.argtypes = [ctypes.POINTER(_vp), _i, ctypes.POINTER(_vp)]
+lib.hxq_group_create.restype = _i
+lib.hxq_group_forward.argtypes = [_vp, _vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _i, _vp]
+lib.hxq_group_forward.restype = _i
+lib.hxq_group_destroy.argtypes = [_vp]
+lib.hxq_group_destroy.restype = None
 lib.hxq_linear_destroy.argtypes = [_vp]
 lib.hxq_linear_destroy.restype = None
 lib.hxq_strerror.argtypes = [_i]
 lib.hxq_strerror.restype = ctypes.c_char_p
 
 EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_linear_forward_out",
-            "hxq_linear_forward_noalloc", "hxq_decode",
+            "hxq_linear_forward_noalloc", "hxq_group_create", "hxq_group_forward", "hxq_group_destroy", "hxq_decode",
             "hxq_linear_check", "hxq_linear_info", "hxq_linear_destroy", "hxq_strerror")
 
 
@@ -124,6 +131,30 @@ def hxq_linear_forward_out(h, x, bias, y, out_dtype, M, stream=None) -> None:
 def hxq_linear_forward_noalloc(h, x, y, M, stream=None) -> None:
     _check(lib.hxq_linear_forward_noalloc(h, _ptr(x), _ptr(y), int(M), _stream(stream)),
            "hxq_linear_forward_noalloc")
+
+
+def _ptr_array(ts):
+    """A C array of data pointers (None entries stay NULL), or NULL for None."""
+    if ts is None:
+        return None
+    return (_vp * len(ts))(*[_ptr(t) for t in ts])
+
+
+def hxq_group_create(handles) -> int:
+    """Returns the group (an integer); raises HXQError on failure."""
+    g = _vp()
+    arr = (_vp * len(handles))(*handles)
+    _check(lib.hxq_group_create(arr, len(handles), ctypes.byref(g)), "hxq_group_create")
+    return g.value
+
+
+def hxq_group_forward(g, x, biases, ys, out_dtype, M, stream=None) -> None:
+    _check(lib.hxq_group_forward(g, _ptr(x), _ptr_array(biases), _ptr_array(ys), int(out_dtype), int(M),
+                                 _stream(stream)), "hxq_group_forward")
+
+
+def hxq_group_destroy(g) -> None:
+    lib.hxq_group_destroy(g)
 
 
 def hxq_decode(h, W_out, stream=None) -> None:
@@ -214,6 +245,39 @@ class HelixLinear:
     def close(self) -> None:
         if getattr(self, "handle", None):
             hxq_linear_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class HelixGroup:
+    """HelixLinear layers that read the same activations (one mode, one K),
+    run by one launch for M <= 4 tokens. Borrows the layers: keep them alive
+    while the group is used."""
+
+    def __init__(self, layers):
+        self.layers = list(layers)
+        self.handle = hxq_group_create([l.handle for l in self.layers])
+
+    def forward(self, x, biases=None, out_dtype=HXQ_OUT_F32, ys=None, stream=None):
+        """[y_i = x . W_i^T (+ bias_i)] for every layer, float32 or bfloat16."""
+        import torch
+        M = int(x.shape[0])
+        if ys is None:
+            dt = torch.bfloat16 if out_dtype == HXQ_OUT_BF16 else torch.float32
+            ys = [torch.empty((M, l.N), dtype=dt, device=x.device) for l in self.layers]
+        hxq_group_forward(self.handle, x, biases, ys, out_dtype, M, stream)
+        return ys
+
+    __call__ = forward
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            hxq_group_destroy(self.handle)
             self.handle = None
 
     def __del__(self):

@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <new>
 #include <numeric>
 #include <vector>
 
@@ -303,6 +304,57 @@ int hxq_linear_forward_out(hxq_linear_t h, const void* x_bf16, const float* bias
   return forward_impl(h, x_bf16, hxq::Out{y, bias, out_dtype == HXQ_OUT_BF16 ? 1 : 0}, M, HXQ_KERNEL_AUTO, 0,
                       stream);
 }
+
+int hxq_group_create(const hxq_linear_t* layers, int n_layers, hxq_group_t* out) {
+  if (!out) return HXQ_EINVAL;
+  *out = nullptr;
+  if (!layers || n_layers < 1 || n_layers > hxq::kMaxGroup) return HXQ_EINVAL;
+  for (int i = 0; i < n_layers; ++i) {
+    const hxq_linear* h = layers[i];
+    if (!h) return HXQ_EINVAL;
+    for (int j = 0; j < i; ++j)
+      if (layers[j] == h) return HXQ_EINVAL;  // one workspace cannot serve two layers of a launch
+    if (h->L.mode != layers[0]->L.mode || h->L.K != layers[0]->L.K || h->device != layers[0]->device)
+      return HXQ_EINVAL;
+  }
+  hxq_group* g = new (std::nothrow) hxq_group();
+  if (!g) return HXQ_ENOMEM;
+  g->n = n_layers;
+  for (int i = 0; i < n_layers; ++i) g->h[i] = layers[i];
+  g->device = layers[0]->device;
+  g->num_sms = layers[0]->num_sms;
+  for (int& c : g->gemv_cluster) c = -1;
+  *out = g;
+  return HXQ_OK;
+}
+
+int hxq_group_forward(hxq_group_t g, const void* x_bf16, const float* const* bias, void* const* y, int out_dtype,
+                      int M, void* stream) {
+  if (!g || !x_bf16 || !y || M < 1) return HXQ_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) != 0) return HXQ_EINVAL;
+  if (out_dtype != HXQ_OUT_F32 && out_dtype != HXQ_OUT_BF16) return HXQ_EINVAL;
+  hxq::Out outs[hxq::kMaxGroup];
+  for (int i = 0; i < g->n; ++i) {
+    if (!y[i]) return HXQ_EINVAL;
+    outs[i] = hxq::Out{y[i], bias ? bias[i] : nullptr, out_dtype == HXQ_OUT_BF16 ? 1 : 0};
+  }
+  if (M <= 4 && hxq::gemv_supports(*g->h[0], M)) {
+    const cudaError_t e = hxq::launch_gemv_group(*g, static_cast<const uint16_t*>(x_bf16), outs, M,
+                                                 static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return e == cudaErrorInvalidValue ? HXQ_EINVAL : HXQ_ECUDA;
+    }
+    return HXQ_OK;
+  }
+  for (int i = 0; i < g->n; ++i) {
+    const int rc = forward_impl(g->h[i], x_bf16, outs[i], M, HXQ_KERNEL_AUTO, 0, stream);
+    if (rc != HXQ_OK) return rc;
+  }
+  return HXQ_OK;
+}
+
+void hxq_group_destroy(hxq_group_t g) { delete g; }
 
 int hxq_decode(hxq_linear_t h, float* W_out, void* stream) {
   if (!h || !W_out) return HXQ_EINVAL;

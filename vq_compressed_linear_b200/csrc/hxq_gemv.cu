@@ -229,8 +229,8 @@ struct Segments {
 // from the workspace (a batch of contributors' loads in flight per sum).
 template <int MT>
 __device__ __forceinline__ void finish_tile(const Layer& L, const Out& out, const float* __restrict__ work,
-                                            const float* own, int M, int t, int c_first, int c_last, int W, int G,
-                                            int n_st, int tid, int nthreads) {
+                                            const float* own, int M, int t, int c_first, int c_last, int b, int W,
+                                            int G, int n_st, int tid, int nthreads) {
   const int rows = min(kTileRows, L.N - t * kTileRows);
   for (int i = tid; i < MT * kTileRows; i += nthreads) {
     const int m = i / kTileRows, r = i % kTileRows;
@@ -246,16 +246,19 @@ __device__ __forceinline__ void finish_tile(const Layer& L, const Out& out, cons
       }
 #pragma unroll
       for (int e = 0; e < 16; ++e)
-        if (c0 + e <= c_last) v += c0 + e == (int)blockIdx.x ? own[i] : q[e];
+        if (c0 + e <= c_last) v += c0 + e == b ? own[i] : q[e];
     }
     store_out(out, (size_t)m * L.N + t * kTileRows + r, t * kTileRows + r, v);
   }
 }
 
+// One CTA's work on layer L: CTA b of the G that share the layer's W stages
+// (stream-K, cs == 0), or of its tiles' clusters of cs CTAs.
 template <int MT, bool XF32, int MODE>
-__global__ void __launch_bounds__(kGemvBlock, 1)
-gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int R, int cs,
-            float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
+__device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __restrict__ x, const Out& out, int M,
+                                          int W, int R, int cs, float* __restrict__ work,
+                                          int* __restrict__ counters, int* __restrict__ status, const int b,
+                                          const int G) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int TB = table_bytes<MODE>();
   constexpr int NP = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per row and stage
@@ -275,17 +278,16 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_st = n_stages(L);
-  const int G = gridDim.x;
   // Stage range: stream-K (cs == 0), or with cs > 0 rank r of cluster t
   // takes stages [r n_st / cs, (r + 1) n_st / cs) of tile t.
   int rw0, rw1;
   if (cs > 0) {
-    const int t = blockIdx.x / cs, r = blockIdx.x - t * cs;
+    const int t = b / cs, r = b - t * cs;
     rw0 = t * n_st + (r * n_st) / cs;
     rw1 = t * n_st + ((r + 1) * n_st) / cs;
   } else {
-    rw0 = (blockIdx.x * W) / G;
-    rw1 = ((blockIdx.x + 1) * W) / G;
+    rw0 = (b * W) / G;
+    rw1 = ((b + 1) * W) / G;
   }
   const Segments S(rw0, rw1, n_st);
   volatile int* abrt = &abort_sh;
@@ -353,7 +355,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int 
       const int t = S.tile(k), slot = S.slot(k);
       mbar_wait(&bar_handoff[slot], 0, &never, 64);
       const int c_first = cta_of(t * n_st, W, G), c_last = cta_of((t + 1) * n_st - 1, W, G);
-      float* part = work + (size_t)(blockIdx.x * 2 + slot) * TS;
+      float* part = work + (size_t)(b * 2 + slot) * TS;
       for (int i = lane; i < TS; i += 32) part[i] = pbuf[slot * TS + i];
       __threadfence();
       __syncwarp();
@@ -361,7 +363,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int 
       prev = __shfl_sync(0xffffffffu, prev, 0);
       if (prev == c_last - c_first) {
         __threadfence();  // the other contributors' sums are visible past their count
-        finish_tile<MT>(L, out, work, pbuf + slot * TS, M, t, c_first, c_last, W, G, n_st, lane, 32);
+        finish_tile<MT>(L, out, work, pbuf + slot * TS, M, t, c_first, c_last, b, W, G, n_st, lane, 32);
         if (lane == 0) counters[t] = 0;
       }
     }
@@ -569,7 +571,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int 
       if (!split) {
         if (m < M && rr < rows) store_out(out, (size_t)m * L.N + t * kTileRows + rr, t * kTileRows + rr, v);
       } else if (cs > 0) {
-        st_cluster_f32(map_to_rank(smem_u32(cbuf + (blockIdx.x % cs) * TS + i), 0), v);
+        st_cluster_f32(map_to_rank(smem_u32(cbuf + (b % cs) * TS + i), 0), v);
       } else {
         pbuf[slot * TS + i] = v;
       }
@@ -580,7 +582,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int 
       // rank 0 adds them in rank order and writes y.
       cluster_arrive_release();
       cluster_wait();
-      if (blockIdx.x % cs == 0) {
+      if (b % cs == 0) {
         for (int i = threadIdx.x; i < TS; i += kGemvThreads) {
           const int m = i / kTileRows;
           float v = 0.f;
@@ -605,7 +607,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int 
       bool last = flag_sh;
       const float* own = pbuf + slot * TS;
       if (!last) {
-        float* part = work + (size_t)(blockIdx.x * 2 + slot) * TS;
+        float* part = work + (size_t)(b * 2 + slot) * TS;
         for (int i = threadIdx.x; i < TS; i += kGemvThreads) part[i] = own[i];
         __threadfence();
         consumer_sync();
@@ -615,7 +617,7 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int 
       }
       if (last) {
         __threadfence();  // the other contributors' sums are visible past their count
-        finish_tile<MT>(L, out, work, own, M, t, c_first, c_last, W, G, n_st, threadIdx.x, kGemvThreads);
+        finish_tile<MT>(L, out, work, own, M, t, c_first, c_last, b, W, G, n_st, threadIdx.x, kGemvThreads);
         if (threadIdx.x == 0) counters[t] = 0;
       }
     }
@@ -625,23 +627,56 @@ gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int 
   __syncthreads();
 }
 
+template <int MT, bool XF32, int MODE>
+__global__ void __launch_bounds__(kGemvBlock, 1)
+gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int R, int cs,
+            float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
+  gemv_body<MT, XF32, MODE>(L, x, out, M, W, R, cs, work, counters, status, (int)blockIdx.x, (int)gridDim.x);
+}
+
+// Several layers that read the same activations (same K and mode), in one
+// launch: layer i owns CTAs [first[i], first[i + 1]) of the grid and runs on
+// them exactly as a launch of its own would (its own codebook, sidecar,
+// output, workspace and counters). Under the cluster split every first[i] is
+// a multiple of the cluster size, so no cluster spans two layers.
+struct GemvGroup {
+  Layer L[kMaxGroup];
+  Out out[kMaxGroup];
+  float* work[kMaxGroup];
+  int* counters[kMaxGroup];
+  int* status[kMaxGroup];
+  int W[kMaxGroup];             // stages of each layer
+  int first[kMaxGroup + 1];     // first CTA of each layer; first[n] = grid size
+  int n;
+};
+
+template <int MT, bool XF32, int MODE>
+__global__ void __launch_bounds__(kGemvBlock, 1)
+gemv_group_kernel(const __grid_constant__ GemvGroup g, const uint16_t* __restrict__ x, int M, int R, int cs) {
+  int li = 0;
+#pragma unroll
+  for (int i = 1; i < kMaxGroup; ++i)
+    if (i < g.n && (int)blockIdx.x >= g.first[i]) li = i;
+  gemv_body<MT, XF32, MODE>(g.L[li], x, g.out[li], M, g.W[li], R, cs, g.work[li], g.counters[li], g.status[li],
+                            (int)blockIdx.x - g.first[li], g.first[li + 1] - g.first[li]);
+}
+
 // Cluster split (no global-memory reduction): each tile gets a cluster of
 // cs CTAs (2..8) that split its K, for the largest cs whose grid (tiles x cs)
 // fills at least 70 % of the SMs without exceeding them and whose clusters
-// all fit on the GPU at once. 0 = the stream-K decomposition.
-template <int MT, bool XF32, int MODE>
-int pick_cluster(const hxq_linear& h) {
-  int& cached = h.gemv_cluster[(XF32 ? 4 : 0) + (MT <= 1 ? 0 : MT <= 2 ? 1 : MT <= 4 ? 2 : 3)];
+// all fit on the GPU at once. 0 = the stream-K decomposition. `cached` keeps
+// the answer for the next launch of the same shape.
+template <int MT, bool XF32, int MODE, typename Kern>
+int pick_cluster_for(Kern kern, int n_tiles, int Kp, int num_sms, int& cached) {
   if (cached >= 0) return cached;
   cached = 0;
   if (MT > 4) return 0;
-  auto kern = gemv_kernel<MT, XF32, MODE>;
-  const int n_st = h.L.Kp / kStageK;
+  const int n_st = Kp / kStageK;
   for (int cs = 8; cs >= 2; --cs) {
-    const int g = h.L.n_tiles * cs;
-    if (g > h.num_sms || 100 * g < 70 * h.num_sms || n_st < cs) continue;
-    if (ring_slots(MODE, MT, h.L.Kp, XF32, cs) < kMinRing) continue;
-    const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32, cs);
+    const int g = n_tiles * cs;
+    if (g > num_sms || 100 * g < 70 * num_sms || n_st < cs) continue;
+    if (ring_slots(MODE, MT, Kp, XF32, cs) < kMinRing) continue;
+    const size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
       cudaGetLastError();
       continue;
@@ -658,13 +693,24 @@ int pick_cluster(const hxq_linear& h) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n_clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&n_clusters, kern, &cfg) == cudaSuccess && n_clusters >= h.L.n_tiles) {
+    if (cudaOccupancyMaxActiveClusters(&n_clusters, kern, &cfg) == cudaSuccess && n_clusters >= n_tiles) {
       cached = cs;
       return cs;
     }
     cudaGetLastError();
   }
   return 0;
+}
+
+// Index of a launch shape's cached cluster size: (activation staging, token
+// count class).
+template <int MT, bool XF32>
+constexpr int cluster_slot() { return (XF32 ? 4 : 0) + (MT <= 1 ? 0 : MT <= 2 ? 1 : MT <= 4 ? 2 : 3); }
+
+template <int MT, bool XF32, int MODE>
+int pick_cluster(const hxq_linear& h) {
+  return pick_cluster_for<MT, XF32, MODE>(gemv_kernel<MT, XF32, MODE>, h.L.n_tiles, h.L.Kp, h.num_sms,
+                                          h.gemv_cluster[cluster_slot<MT, XF32>()]);
 }
 
 template <int MT, bool XF32, int MODE>
@@ -708,6 +754,97 @@ cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, const Out& out, 
 
 int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
+// Stream-K shares of a group's grid: G CTAs, layer i getting about
+// G W[i] / sum W of them, at least 1 and at most W[i]; the CTAs left over
+// (or taken back) go to (come from) the layers with the most (fewest)
+// stages per CTA.
+void group_shares(const int64_t* W, int n, int G, int* Gl) {
+  int64_t Wt = 0;
+  for (int i = 0; i < n; ++i) Wt += W[i];
+  int sum = 0;
+  for (int i = 0; i < n; ++i) {
+    Gl[i] = (int)std::max<int64_t>(1, std::min<int64_t>(W[i], (int64_t)G * W[i] / Wt));
+    sum += Gl[i];
+  }
+  while (sum < G) {  // W[i] / Gl[i] largest among the layers that can take one more
+    int best = -1;
+    for (int i = 0; i < n; ++i)
+      if (Gl[i] < W[i] && (best < 0 || W[i] * Gl[best] > W[best] * Gl[i])) best = i;
+    if (best < 0) break;
+    ++Gl[best];
+    ++sum;
+  }
+  while (sum > G) {  // W[i] / Gl[i] smallest among the layers that can give one up
+    int best = -1;
+    for (int i = 0; i < n; ++i)
+      if (Gl[i] > 1 && (best < 0 || W[i] * Gl[best] < W[best] * Gl[i])) best = i;
+    if (best < 0) break;
+    --Gl[best];
+    --sum;
+  }
+}
+
+template <int MT, bool XF32, int MODE>
+cudaError_t launch_group_cfg(const hxq_group& g, const uint16_t* x, const Out* outs, int M, cudaStream_t s) {
+  auto kern = gemv_group_kernel<MT, XF32, MODE>;
+  const int Kp = g.h[0]->L.Kp, n_st = Kp / kStageK;
+  GemvGroup p = {};
+  p.n = g.n;
+  int n_tiles = 0;
+  int64_t W[kMaxGroup];
+  for (int i = 0; i < g.n; ++i) {
+    const hxq_linear& h = *g.h[i];
+    p.L[i] = h.L;
+    p.out[i] = outs[i];
+    p.work[i] = h.d_work;
+    p.counters[i] = h.d_counters;
+    p.status[i] = h.d_status;
+    W[i] = (int64_t)h.L.n_tiles * n_st;
+    p.W[i] = (int)W[i];
+    n_tiles += h.L.n_tiles;
+  }
+  const int cs = pick_cluster_for<MT, XF32, MODE>(kern, n_tiles, Kp, g.num_sms,
+                                                  g.gemv_cluster[cluster_slot<MT, XF32>()]);
+  p.first[0] = 0;
+  if (cs > 0) {
+    for (int i = 0; i < g.n; ++i) p.first[i + 1] = p.first[i] + g.h[i]->L.n_tiles * cs;
+  } else {
+    int64_t Wt = 0;
+    for (int i = 0; i < g.n; ++i) Wt += W[i];
+    const int G = (int)std::max<int64_t>(g.n, std::min<int64_t>(g.num_sms, Wt));
+    int Gl[kMaxGroup];
+    group_shares(W, g.n, G, Gl);
+    for (int i = 0; i < g.n; ++i) {
+      if (W[i] * Gl[i] >= INT_MAX) return cudaErrorInvalidValue;  // item arithmetic is 32-bit
+      // every CTA writes at most two partial tiles of MT x 128 floats
+      if ((size_t)Gl[i] * 2 * MT * kTileRows > g.h[i]->work_floats) return cudaErrorInvalidValue;
+      p.first[i + 1] = p.first[i] + Gl[i];
+    }
+  }
+  for (int i = g.n + 1; i <= kMaxGroup; ++i) p.first[i] = p.first[g.n];
+  const int grid = p.first[g.n];
+  const int R = ring_slots(MODE, MT, Kp, XF32, cs);
+  if (R < kMinRing) return cudaErrorInvalidValue;
+  const size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (cs > 0) return launch_pdl_cluster(kern, grid, kGemvBlock, smem, cs, s, p, x, M, R, cs);
+  return launch_pdl(kern, grid, kGemvBlock, smem, s, p, x, M, R, 0);
+}
+
+template <int MT, int MODE>
+cudaError_t launch_group_mt(const hxq_group& g, const uint16_t* x, const Out* outs, int M, cudaStream_t s) {
+  if (ring_slots(MODE, MT, g.h[0]->L.Kp, true) >= kMinRing) return launch_group_cfg<MT, true, MODE>(g, x, outs, M, s);
+  return launch_group_cfg<MT, false, MODE>(g, x, outs, M, s);
+}
+
+template <int MODE>
+cudaError_t launch_group_mode(const hxq_group& g, const uint16_t* x, const Out* outs, int M, cudaStream_t s) {
+  if (M <= 1) return launch_group_mt<1, MODE>(g, x, outs, M, s);
+  if (M <= 2) return launch_group_mt<2, MODE>(g, x, outs, M, s);
+  return launch_group_mt<4, MODE>(g, x, outs, M, s);
+}
+
 }  // namespace
 
 bool gemv_supports(const hxq_linear& h, int M) {
@@ -723,6 +860,14 @@ int gemv_grid(const hxq_linear& h, int split) {
   grid = std::max<int64_t>(1, std::min<int64_t>({grid, (int64_t)h.num_sms, W}));
   if (W * grid >= INT_MAX) return 0;  // item arithmetic is 32-bit
   return (int)grid;
+}
+
+cudaError_t launch_gemv_group(const hxq_group& g, const uint16_t* x, const Out* outs, int M, cudaStream_t s) {
+  if (g.n < 1 || g.n > kMaxGroup || M < 1 || M > 4) return cudaErrorInvalidValue;
+  for (int i = 0; i < g.n; ++i)
+    if (!gemv_supports(*g.h[i], M)) return cudaErrorInvalidValue;
+  if (g.h[0]->L.mode == HXQ_MODE_SCALAR8) return launch_group_mode<HXQ_MODE_SCALAR8>(g, x, outs, M, s);
+  return launch_group_mode<HXQ_MODE_VQ2D12>(g, x, outs, M, s);
 }
 
 cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split, cudaStream_t s) {

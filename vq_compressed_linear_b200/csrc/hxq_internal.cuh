@@ -32,6 +32,7 @@ namespace hxq {
 constexpr int kTileRows = 128;
 constexpr int kStageK = 64;           // weights per row per pipeline stage
 constexpr int kMaxSplitK = 64;
+constexpr int kMaxGroup = HXQ_MAX_GROUP;  // layers in one grouped launch
 
 struct Layer {
   int mode;          // HXQ_MODE_*
@@ -96,6 +97,17 @@ struct hxq_linear {
   mutable int gemv_cluster[8];
 };
 
+// Layers that share their activations (same mode and K, one device); the
+// handles are borrowed.
+struct hxq_group {
+  int n;
+  hxq_linear* h[hxq::kMaxGroup];
+  int device;
+  int num_sms;
+  // cluster size of the grouped GEMV, as hxq_linear::gemv_cluster
+  mutable int gemv_cluster[8];
+};
+
 namespace hxq {
 
 // Launchers (each returns a cudaError_t from the launch).
@@ -104,6 +116,8 @@ cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, const Out& out, 
                         cudaStream_t s);
 cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split,
                       cudaStream_t s);
+// One launch of the GEMV over every layer of g (outs[i] for layer i).
+cudaError_t launch_gemv_group(const hxq_group& g, const uint16_t* x, const Out* outs, int M, cudaStream_t s);
 bool gemv_supports(const hxq_linear& h, int M);
 int gemv_grid(const hxq_linear& h, int split);
 size_t tc_workspace_floats(int num_sms);
