@@ -1,2 +1,3 @@
-"""CPU oracle for the HXQ HelixLinear forward: test infrastructure only."""
+"""CPU oracle for the HXQ HelixLinear forward and encoder: test infrastructure only."""
+from .hxq_encoder_oracle import *  # noqa: F401,F403
 from .hxq_oracle import *  # noqa: F401,F403

@@ -1,0 +1,151 @@
+"""CPU oracle for the HXQ encoder side -- TEST INFRASTRUCTURE.
+
+Only the tests use this module; the CUDA library never imports, links or
+calls it, and the two share no code.
+
+The HXQ whitepaper (method section) compresses each weight tensor on its
+own, in this order:
+
+1. "Per-tensor k-means": k-means on the weight values (k = 256 entries of
+   one weight for scalar VQ, k = 4096 entries of an adjacent pair for 2D VQ)
+   gives the codebook; no calibration data is used.
+2. "Index assignment": each weight, or pair, gets the index of its nearest
+   codebook entry.
+3. "Sidecar outlier correction": weights whose reconstruction error exceeds
+   a threshold are stored apart, exactly.
+4. "12-bit index packing" (2D): two 12-bit indices per 3 bytes, the layout
+   the decoder reads (oracle.pack12).
+
+k-means is Lloyd's algorithm: assign every point to its nearest centroid,
+move every centroid to the mean of its points, repeat.
+
+Readings where the pages are silent (each is listed in the design notes):
+* The initial centroids are an input (the pages name no initialisation; a
+  random draw is the caller's, passed in), and the number of Lloyd rounds is
+  fixed by the caller: no convergence test, so both sides take the same
+  steps.
+* Distances are decided in fp32, the precision of the weights and of the
+  kernels: for one dimension d = |p - c| (one rounded subtraction); for
+  pairs d = dx*dx + dy*dy, each product and the sum rounded to fp32 in that
+  order, with no fused multiply-add. Equal distances go to the lowest index.
+* A centroid moves to the mean of its points, formed in float64 and rounded
+  to fp32 (nearest even); a centroid with no points stays where it is.
+* The sidecar threshold is on |w - w_hat| per weight, in fp32, and strict
+  (an error equal to the threshold is not stored). An entry stores the
+  weight itself, the replacement form the decoder takes (the whitepaper's
+  "(row, col, delta)" wording read as a value that restores w exactly),
+  at flat position n*K + k, in ascending order. On a 2D pair each of the
+  two weights is tested and stored on its own.
+
+Pins (tests/test_encoder_oracle.py): pure-Python brute force on tiny sets,
+the midpoint rule for sorted 1D centroids, scikit-learn's Lloyd k-means
+from the same start, the non-increasing objective, weights drawn exactly
+from a codebook, planted outliers at dyadic values, and planted mistakes.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .hxq_oracle import MODE_SCALAR8, MODE_VQ2D12, SCALAR_ENTRIES, VQ2D_ENTRIES, pack12
+
+_CHUNK_CELLS = 1 << 22  # points x centroids per block of the distance table
+
+
+def _as_points(a) -> np.ndarray:
+    p = np.asarray(a, dtype=np.float32)
+    return p.reshape(-1, 1) if p.ndim == 1 else p
+
+
+def distances_f32(points, centroids) -> np.ndarray:
+    """fp32 distance table [n][k] as the readings define it."""
+    p = _as_points(points)
+    c = _as_points(centroids)
+    if p.shape[1] != c.shape[1] or p.shape[1] not in (1, 2):
+        raise ValueError("points and centroids need the same dimension, 1 or 2")
+    if p.shape[1] == 1:
+        return np.abs(p[:, 0][:, None] - c[:, 0][None, :])  # float32 throughout
+    dx = p[:, 0][:, None] - c[:, 0][None, :]
+    dy = p[:, 1][:, None] - c[:, 1][None, :]
+    return dx * dx + dy * dy  # numpy rounds each float32 operation; nothing is fused
+
+
+def assign(points, centroids) -> np.ndarray:
+    """Index assignment: the nearest centroid of each point (int64), fp32
+    distances, lowest index on ties (argmin returns the first minimum)."""
+    p = _as_points(points)
+    c = _as_points(centroids)
+    out = np.empty(p.shape[0], dtype=np.int64)
+    step = max(1, _CHUNK_CELLS // max(1, c.shape[0]))
+    for i in range(0, p.shape[0], step):
+        out[i:i + step] = np.argmin(distances_f32(p[i:i + step], c), axis=1)
+    return out
+
+
+def kmeans_update(points, labels, centroids) -> np.ndarray:
+    """Each centroid moves to the mean of its points (float64 sum / count,
+    rounded to fp32); one without points keeps its position."""
+    p = _as_points(points).astype(np.float64)
+    c = _as_points(centroids)
+    k, dim = c.shape
+    labels = np.asarray(labels, dtype=np.int64)
+    count = np.bincount(labels, minlength=k)
+    new = c.copy()
+    for d in range(dim):
+        s = np.bincount(labels, weights=p[:, d], minlength=k)
+        has = count > 0
+        new[has, d] = (s[has] / count[has]).astype(np.float32)
+    return new
+
+
+def kmeans(points, init, iters: int) -> tuple[np.ndarray, np.ndarray]:
+    """Lloyd's k-means from `init` for `iters` rounds; returns the centroids
+    (fp32, shaped like init) and the assignment to them."""
+    c = _as_points(init).copy()
+    p = _as_points(points)
+    for _ in range(int(iters)):
+        c = kmeans_update(p, assign(p, c), c)
+    labels = assign(p, c)
+    return c.reshape(np.shape(init)), labels
+
+
+def inertia(points, centroids, labels) -> float:
+    """Sum of squared distances to the assigned centroids, in float64."""
+    p = _as_points(points).astype(np.float64)
+    c = _as_points(centroids).astype(np.float64)
+    return float(np.sum((p - c[np.asarray(labels, dtype=np.int64)]) ** 2))
+
+
+def sidecar_select(W, W_hat, threshold: float) -> tuple[np.ndarray, np.ndarray]:
+    """Sidecar outlier correction: flat positions (ascending, int64) where
+    |w - w_hat| > threshold in fp32, and the weights there (the values that
+    replace the decoded ones)."""
+    w = np.asarray(W, dtype=np.float32).reshape(-1)
+    wh = np.asarray(W_hat, dtype=np.float32).reshape(-1)
+    err = np.abs(w - wh)
+    pos = np.nonzero(err > np.float32(threshold))[0].astype(np.int64)
+    return pos, w[pos].copy()
+
+
+def encode(W, mode: int, codebook, threshold: float):
+    """Steps 2-4 for a trained codebook: W fp32 [N][K] -> (index bytes in the
+    decoder's layout, sidecar positions, sidecar values)."""
+    W = np.asarray(W, dtype=np.float32)
+    N, K = W.shape
+    cb = np.asarray(codebook, dtype=np.float32).reshape(-1)
+    if mode == MODE_SCALAR8:
+        if cb.size != SCALAR_ENTRIES:
+            raise ValueError("scalar mode needs 256 codebook entries")
+        lab = assign(W.reshape(-1), cb)
+        indices = lab.astype(np.uint8)
+        W_hat = cb[lab].reshape(N, K)
+    elif mode == MODE_VQ2D12:
+        if K % 4 or cb.size != 2 * VQ2D_ENTRIES:
+            raise ValueError("2D mode needs K % 4 == 0 and 4096 pairs")
+        pairs = cb.reshape(VQ2D_ENTRIES, 2)
+        lab = assign(W.reshape(-1, 2), pairs)
+        indices = pack12(lab)
+        W_hat = pairs[lab].reshape(N, K)
+    else:
+        raise ValueError(f"unknown mode {mode}")
+    pos, val = sidecar_select(W, W_hat, threshold)
+    return indices, pos, val

@@ -1,0 +1,245 @@
+"""Pins of the encoder oracle (CPU): k-means, index assignment, sidecar
+selection and the full encode, each checked against something other than
+its own formula -- exact integer brute force on dyadic inputs, the midpoint
+rule, scikit-learn's Lloyd k-means, Lloyd's monotone objective, weights drawn
+exactly from a codebook -- and planted mistakes that those pins must catch.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+
+enc = oracle.hxq_encoder_oracle
+
+
+def _dyadic(rng, shape, lo=-64, hi=64, scale=2.0 ** -6):
+    """Small multiples of 2^-6: fp32 differences, squares and sums of two
+    squares of these are exact, so fp32 decisions equal exact ones."""
+    return (rng.integers(lo, hi, size=shape) * scale).astype(np.float32)
+
+
+def _exact_nearest(points_int, cents_int):
+    """Nearest centroid with Python integers (the dyadic grid scaled to
+    integers); ties to the lowest index."""
+    out = []
+    for p in points_int:
+        best, bi = None, -1
+        for i, c in enumerate(cents_int):
+            d = sum((a - b) * (a - b) for a, b in zip(p, c))
+            if best is None or d < best:
+                best, bi = d, i
+        out.append(bi)
+    return np.array(out, dtype=np.int64)
+
+
+@pytest.mark.parametrize("dim", [1, 2])
+def test_assign_exact_integer_bruteforce(dim):
+    rng = np.random.default_rng(3 + dim)
+    pts = _dyadic(rng, (300, dim))
+    # few distinct centroid values, some repeated: exact ties must go to the lowest index
+    cents = _dyadic(rng, (12, dim), -16, 16, 2.0 ** -4)
+    cents[7] = cents[2]
+    cents[11] = cents[5]
+    got = enc.assign(pts if dim == 2 else pts[:, 0], cents if dim == 2 else cents[:, 0])
+    to_int = lambda a: [tuple(int(v) for v in row) for row in np.rint(a.astype(np.float64) * 64)]
+    want = _exact_nearest(to_int(pts), to_int(cents))
+    assert np.array_equal(got, want)
+    assert not np.isin(got, [7, 11]).any()  # the later copy of a tie never wins
+
+
+def test_assign_midpoint_rule_1d():
+    """Sorted distinct centroids in 1D: the nearest is found by comparing
+    with the midpoints between neighbours (a point on a midpoint goes left,
+    to the lower index)."""
+    rng = np.random.default_rng(5)
+    cents = np.unique(_dyadic(rng, 40, -512, 512, 2.0 ** -7))
+    pts = _dyadic(rng, 5000, -600, 600, 2.0 ** -8)
+    mids = (cents[:-1].astype(np.float64) + cents[1:]) / 2
+    want = np.searchsorted(mids, pts.astype(np.float64), side="left")
+    assert np.array_equal(enc.assign(pts, cents), want)
+
+
+def _blobs(rng, centers, per, sigma):
+    c = np.asarray(centers, np.float64)
+    pts = np.repeat(c, per, axis=0) + rng.normal(0, sigma, size=(c.shape[0] * per, c.shape[1]))
+    return pts[rng.permutation(pts.shape[0])].astype(np.float32)
+
+
+@pytest.mark.parametrize("dim", [1, 2])
+def test_kmeans_matches_sklearn_lloyd(dim):
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(11 + dim)
+    k = 6
+    centers = rng.uniform(-1, 1, size=(k, dim)) * 4
+    pts = _blobs(rng, centers, 400, 0.25)
+    init = pts[rng.choice(pts.shape[0], k, replace=False)]
+    for iters in (1, 3, 20):
+        c, lab = enc.kmeans(pts, init, iters)
+        km = KMeans(n_clusters=k, init=init.astype(np.float64), n_init=1, max_iter=iters, tol=0.0,
+                    algorithm="lloyd").fit(pts.astype(np.float64))
+        assert np.array_equal(lab, km.labels_), f"iters {iters}"
+        assert np.allclose(c, km.cluster_centers_, rtol=0, atol=1e-6), f"iters {iters}"
+
+
+@pytest.mark.parametrize("dim", [1, 2])
+def test_kmeans_objective_never_increases(dim):
+    rng = np.random.default_rng(21 + dim)
+    pts = rng.normal(0, 0.02, size=(4000, dim)).astype(np.float32)
+    c = pts[rng.choice(pts.shape[0], 64, replace=False)].copy()
+    prev = enc.inertia(pts, c, enc.assign(pts, c))
+    for _ in range(8):
+        c = enc.kmeans_update(pts, enc.assign(pts, c), c)
+        cur = enc.inertia(pts, c, enc.assign(pts, c))
+        assert cur <= prev * (1 + 1e-9)
+        prev = cur
+
+
+def test_kmeans_recovers_separated_clusters_and_stays_there():
+    rng = np.random.default_rng(31)
+    centers = np.array([[-3.0, 1.0], [0.0, -2.0], [2.5, 2.5], [4.0, -4.0]])
+    pts = _blobs(rng, centers, 500, 0.05)
+    c, lab = enc.kmeans(pts, centers + 0.7, 10)
+    assert np.allclose(c, centers, atol=0.02)
+    assert np.array_equal(np.bincount(lab, minlength=4), [500] * 4)
+    c2, lab2 = enc.kmeans(pts, c, 3)  # a fixed point of Lloyd's rounds
+    assert np.array_equal(c2, c) and np.array_equal(lab2, lab)
+
+
+def test_kmeans_update_empty_cluster_keeps_position():
+    pts = np.array([[0.0], [0.25], [4.0], [4.5]], np.float32)
+    c = np.array([[0.0], [4.0], [100.0]], np.float32)
+    new = enc.kmeans_update(pts, enc.assign(pts, c), c)
+    assert np.array_equal(new[:, 0], np.array([0.125, 4.25, 100.0], np.float32))
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_encode_recovers_weights_drawn_from_the_codebook(mode):
+    rng = np.random.default_rng(41 + mode)
+    N, K = 24, 40
+    if mode == 0:
+        cb = np.sort(rng.normal(0, 0.02, 256)).astype(np.float32)
+        idx = rng.integers(0, 256, size=N * K)
+        W = cb[idx].reshape(N, K)
+    else:
+        cb = rng.normal(0, 0.02, 8192).astype(np.float32)
+        idx = rng.integers(0, 4096, size=N * K // 2)
+        W = cb.reshape(4096, 2)[idx].reshape(N, K)
+    indices, pos, val = enc.encode(W, mode, cb, 0.0)
+    want = idx.astype(np.uint8) if mode == 0 else oracle.pack12(idx)
+    assert np.array_equal(indices, want)
+    assert pos.size == 0 and val.size == 0
+    assert np.array_equal(oracle.decode(mode, cb, indices, pos, val, N, K), W)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_sidecar_planted_outliers_dyadic(mode):
+    """Codebook on a coarse dyadic grid, weights on it plus planted offsets:
+    an error exactly at the threshold stays out, one above it goes in."""
+    rng = np.random.default_rng(51 + mode)
+    N, K = 8, 32
+    tau = np.float32(2.0 ** -5)
+    if mode == 0:
+        cb = (np.arange(256) - 128).astype(np.float32) * 2.0 ** -3
+        idx = rng.integers(0, 256, size=N * K)
+        W_hat = cb[idx].reshape(N, K)
+    else:
+        g = (np.arange(64) - 32).astype(np.float32) * 2.0 ** -3
+        cb = np.stack(np.meshgrid(g, g, indexing="ij"), -1).reshape(-1).astype(np.float32)  # 64 x 64 grid
+        idx = rng.integers(0, 4096, size=N * K // 2)
+        W_hat = cb.reshape(4096, 2)[idx].reshape(N, K)
+    W = W_hat.copy()
+    flat = W.reshape(-1)
+    at_tau = np.array([3, 77, 130])
+    above = np.array([5, 64, 200, 255])
+    small = np.array([9, 100])
+    flat[at_tau] += tau               # exactly the threshold: not stored
+    flat[above] -= np.float32(3 * 2.0 ** -6)  # 0.046875 > tau, still nearest to its own entry
+    flat[small] += np.float32(2.0 ** -7)
+    indices, pos, val = enc.encode(W, mode, cb, float(tau))
+    assert np.array_equal(pos, np.sort(above))
+    assert np.array_equal(val, flat[np.sort(above)])
+    W_rec = oracle.decode(mode, cb, indices, pos, val, N, K)
+    assert np.max(np.abs(W_rec - W)) <= tau
+    assert np.array_equal(W_rec.reshape(-1)[pos], flat[pos])
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_encode_decode_roundtrip_within_threshold(mode):
+    rng = np.random.default_rng(61 + mode)
+    N, K = 16, 64
+    W = rng.normal(0, 0.02, size=(N, K)).astype(np.float32)
+    pts = W.reshape(-1, 1 if mode == 0 else 2)
+    k = 256 if mode == 0 else 4096
+    init = pts[rng.choice(pts.shape[0], min(k, pts.shape[0]), replace=False)]
+    if init.shape[0] < k:  # 2D with fewer pairs than entries: pad with far points that stay empty
+        init = np.concatenate([init, np.full((k - init.shape[0], 2), 1e3, np.float32)])
+    cb, _ = enc.kmeans(pts, init, 4)
+    tau = 0.004
+    indices, pos, val = enc.encode(W, mode, cb.reshape(-1), tau)
+    W_rec = oracle.decode(mode, cb.reshape(-1), indices, pos, val, N, K)
+    assert np.all(np.abs(W_rec - W) <= np.float32(tau))
+    assert np.array_equal(W_rec.reshape(-1)[pos], W.reshape(-1)[pos])
+
+
+# ----------------------------------------------------------------- planted mistakes
+
+def _pins_pass():
+    try:
+        for dim in (1, 2):
+            test_assign_exact_integer_bruteforce(dim)
+            test_kmeans_matches_sklearn_lloyd(dim)
+        test_assign_midpoint_rule_1d()
+        test_kmeans_update_empty_cluster_keeps_position()
+        for mode in (0, 1):
+            test_encode_recovers_weights_drawn_from_the_codebook(mode)
+            test_sidecar_planted_outliers_dyadic(mode)
+    except AssertionError:
+        return False
+    return True
+
+
+@pytest.mark.parametrize("mutant", ["ties_last", "swap_pair_components", "update_skips_last_point",
+                                    "empty_to_zero", "threshold_inclusive", "sidecar_stores_delta",
+                                    "sidecar_colmajor"])
+def test_encoder_planted_mistakes_are_caught(monkeypatch, mutant):
+    assert _pins_pass()
+    orig_dist, orig_update, orig_select = enc.distances_f32, enc.kmeans_update, enc.sidecar_select
+    if mutant == "ties_last":
+        def assign_last(points, centroids):
+            d = orig_dist(points, centroids)
+            return d.shape[1] - 1 - np.argmin(d[:, ::-1], axis=1)
+        monkeypatch.setattr(enc, "assign", assign_last)
+    elif mutant == "swap_pair_components":
+        def dist_swapped(points, centroids):
+            c = enc._as_points(centroids)
+            return orig_dist(points, c[:, ::-1] if c.shape[1] == 2 else c)
+        monkeypatch.setattr(enc, "distances_f32", dist_swapped)
+    elif mutant == "update_skips_last_point":
+        monkeypatch.setattr(enc, "kmeans_update",
+                            lambda p, lab, c: orig_update(enc._as_points(p)[:-1], np.asarray(lab)[:-1], c))
+    elif mutant == "empty_to_zero":
+        def update_zero(p, lab, c):
+            new = orig_update(p, lab, c)
+            new[np.bincount(np.asarray(lab), minlength=len(new)) == 0] = 0
+            return new
+        monkeypatch.setattr(enc, "kmeans_update", update_zero)
+    elif mutant == "threshold_inclusive":
+        def select_ge(W, W_hat, t):
+            w, wh = np.asarray(W, np.float32).reshape(-1), np.asarray(W_hat, np.float32).reshape(-1)
+            pos = np.nonzero(np.abs(w - wh) >= np.float32(t))[0].astype(np.int64)
+            return pos, w[pos]
+        monkeypatch.setattr(enc, "sidecar_select", select_ge)
+    elif mutant == "sidecar_stores_delta":
+        def select_delta(W, W_hat, t):
+            pos, _ = orig_select(W, W_hat, t)
+            return pos, (np.asarray(W, np.float32).reshape(-1) - np.asarray(W_hat, np.float32).reshape(-1))[pos]
+        monkeypatch.setattr(enc, "sidecar_select", select_delta)
+    elif mutant == "sidecar_colmajor":
+        def select_colmajor(W, W_hat, t):
+            Wa = np.asarray(W, np.float32)
+            pos, val = orig_select(Wa.T, np.asarray(W_hat, np.float32).T, t)
+            return pos, val
+        monkeypatch.setattr(enc, "sidecar_select", select_colmajor)
+    assert not _pins_pass(), f"planted mistake {mutant} was not caught"
