@@ -407,6 +407,71 @@ def profile_run(hxq, torch, items, steps, warmup):
     return 0
 
 
+# ----------------------------------------------------------------------------- encoder
+
+ENCODER_ROUNDS = 10
+# fp32 instructions per point-centroid comparison in the assignment loop
+# (subtract, compare, two selects; pairs: two subtracts, two multiplies, add,
+# compare, two selects) -- the count the ALU roofline below rests on
+ENCODER_OPS = {1: 4, 2: 8}
+
+
+def encoder_run(hxq, torch, args):
+    """One step = ENCODER_ROUNDS k-means rounds on one layer's weights plus
+    its encode (indices + sidecar); metric: weights per second."""
+    mode, N, K, k = (0, 8512, 2048, 256) if args.encoder == "scalar" else (1, 11008, 4096, 4096)
+    dim = 1 if mode == 0 else 2
+    rng = np.random.default_rng(0)
+    W = torch.from_numpy(rng.normal(0, 0.02, size=(N, K)).astype(np.float32)).cuda()
+    pts = W.view(-1, dim) if dim == 2 else W.view(-1)
+    n = pts.shape[0]
+    init = pts[torch.from_numpy(rng.choice(n, k, replace=False)).cuda()].clone()
+    cent = torch.empty_like(init)
+    labels = torch.empty(n, dtype=torch.int16, device="cuda")
+    idx = torch.empty(N * K if mode == 0 else 3 * N * K // 4, dtype=torch.uint8, device="cuda")
+    cap = N * K // 50
+    pos = torch.empty(cap, dtype=torch.int64, device="cuda")
+    val = torch.empty(cap, dtype=torch.float32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
+    tau = 0.002 if mode == 0 else 0.006
+    stream = torch.cuda.Stream()
+
+    def step():
+        cent.copy_(init)
+        hxq.hxq_kmeans(pts, n, dim, k, ENCODER_ROUNDS, cent, labels, stream)
+        hxq.hxq_encode(W, mode, N, K, cent.view(-1), tau, idx, pos, val, cap, cnt, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        e1.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    # comparisons per step: (rounds + final assignment + encode) x n x k
+    evals = (ENCODER_ROUNDS + 2) * n * k
+    props = torch.cuda.get_device_properties(0)
+    clock_ghz = 1.965  # clocks.max.sm of this part
+    peak = props.multi_processor_count * 128 * clock_ghz * 1e9 / ENCODER_OPS[dim]
+    achieved = evals / (ms * 1e-3)
+    line = {"metric": "HXQ encoder weights/s", "value": N * K / (ms * 1e-3), "unit": "weights/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": f"encode {N}x{K} mode {mode}, k={k}, {ENCODER_ROUNDS} k-means rounds, "
+                                   f"threshold {tau}", "sidecar_entries": int(cnt.item())},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "comparisons/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_kind": f"derived: SMs x 128 fp32 lanes x {clock_ghz} GHz / {ENCODER_OPS[dim]} "
+                                      "instructions per comparison"}}
+    print(json.dumps(line))
+    return 0
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -421,6 +486,9 @@ def main():
     ap.add_argument("--grouped", action="store_true",
                     help="run the layers that share their input as one grouped forward each")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--encoder", choices=["scalar", "vq2d"], default=None,
+                    help="time the GPU encoder instead (k-means rounds + encode of one layer): "
+                         "scalar = in_proj 8512x2048, k=256; vq2d = 11008x4096 pairs, k=4096")
     ap.add_argument("--ncu", action="store_true",
                     help="minimal run for profilers: enough layer replicas to exceed L2, then "
                          "W + K eager steps; prints nothing")
@@ -463,6 +531,8 @@ def main():
 
     if args.ncu:
         return profile_run(hxq, torch, items, args.steps, args.warmup)
+    if args.encoder:
+        return encoder_run(hxq, torch, args)
 
     if world > 1:
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")

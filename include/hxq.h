@@ -200,6 +200,66 @@ int hxq_group_forward(hxq_group_t g, const void* x_bf16, const float* const* bia
 void hxq_group_destroy(hxq_group_t g);
 
 /*
+ * ---- Encoder: the codec's other side (HXQ whitepaper, method section, the
+ * per-tensor pipeline: "Per-tensor k-means", "Index assignment", "Sidecar
+ * outlier correction", "12-bit index packing"). All pointers are device
+ * pointers; every call is asynchronous on `stream` and writes only its
+ * outputs (scratch comes from the stream-ordered allocator).
+ *
+ * Points are fp32 [n][dim]: dim 1 for scalar VQ (one weight per point, the
+ * weight matrix read flat), dim 2 for 2D VQ (adjacent pairs (k, k+1), k
+ * even, of a row: the row-major [N][K] weight matrix read as [N*K/2][2]).
+ * Points and centroids must be finite. Distances are decided in fp32 with
+ * each operation rounded (no fused multiply-add): |p - c| for dim 1,
+ * dx*dx + dy*dy for dim 2; equal distances go to the lowest index.
+ */
+
+/*
+ * Index assignment: labels[i] = index of the nearest of the k centroids
+ * ([k][dim] fp32) to point i. 1 <= k <= 4096, 1 <= n < 2^31, dim 1 or 2.
+ * Returns HXQ_EINVAL for NULL pointers or sizes out of range; HXQ_ECUDA if
+ * a launch fails.
+ */
+int hxq_assign(const float* points, int64_t n, int dim, const float* centroids, int k,
+               uint16_t* labels, void* stream);
+
+/*
+ * Per-tensor k-means: `iters` rounds of Lloyd's algorithm on the n points,
+ * starting from the k centroids in `centroids` ([k][dim] fp32, overwritten
+ * with the result). The pages name no initialisation and no stopping rule:
+ * the caller supplies the start (for instance a seeded random sample of the
+ * points) and the number of rounds. Each round assigns every point as
+ * hxq_assign does and moves every centroid with points to their mean,
+ * rounded to fp32; a centroid without points stays. The means are formed
+ * from exact fixed-point sums, so the result is bitwise repeatable and
+ * within one fp32 rounding of the float64 mean. labels (NULL allowed)
+ * receives the assignment to the final centroids. iters >= 0; other limits
+ * and errors as hxq_assign, plus HXQ_ENOMEM if scratch cannot be allocated.
+ */
+int hxq_kmeans(const float* points, int64_t n, int dim, int k, int iters, float* centroids,
+               uint16_t* labels, void* stream);
+
+/*
+ * Encode a weight matrix W (fp32 [N][K], row-major) with a trained codebook
+ * into what hxq_linear_create reads: `indices` in the layout above (scalar:
+ * N*K bytes; 2D: 3*N*K/4 bytes) from the nearest entry of each weight or
+ * pair, and the sidecar: every weight with |w - w_hat| > threshold (fp32,
+ * strict), as flat position n*K + k (ascending) and the weight itself, which
+ * replaces the decoded value. `codebook` holds 256 floats (scalar) or 4096
+ * fp32 pairs (2D). *n_sidecar (device int64) receives the number of such
+ * weights; only the first min(*n_sidecar, max_sidecar) are written, so a
+ * caller that finds *n_sidecar > max_sidecar can retry with more room.
+ * Shape limits as hxq_linear_create (K >= 8, K % 8 == 0), N*K < 2^31.
+ * Returns HXQ_EINVAL for NULL W/codebook/indices/n_sidecar, NULL sidecar
+ * arrays with max_sidecar > 0, max_sidecar < 0, a negative or NaN
+ * threshold, an unknown mode or a bad shape; HXQ_ENOMEM / HXQ_ECUDA on
+ * scratch or launch failures.
+ */
+int hxq_encode(const float* W, int mode, int N, int K, const float* codebook, float threshold,
+               uint8_t* indices, int64_t* sidecar_pos, float* sidecar_val, int64_t max_sidecar,
+               int64_t* n_sidecar, void* stream);
+
+/*
  * Test helper: write the decoded fp32 weights W[N][K] (sidecar applied) to
  * the device buffer W_out on `stream`. Bit-exact with the definition above.
  * Returns HXQ_EINVAL for a NULL handle or W_out, HXQ_ECUDA on launch failure.

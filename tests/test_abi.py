@@ -105,6 +105,23 @@ def test_group_entry_points_reject_null_arguments():
     m.lib.hxq_group_destroy(None)  # ignored
 
 
+def test_encoder_entry_points_reject_null_arguments():
+    import vq_compressed_linear_b200 as m
+    p = np.zeros(64, np.float32)
+    lab = np.zeros(64, np.uint16)
+    assert m.lib.hxq_assign(None, 64, 1, m._ptr(p), 8, m._ptr(lab), None) == m.HXQ_EINVAL
+    assert m.lib.hxq_assign(m._ptr(p), 64, 1, None, 8, m._ptr(lab), None) == m.HXQ_EINVAL
+    assert m.lib.hxq_assign(m._ptr(p), 64, 1, m._ptr(p), 8, None, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_kmeans(None, 64, 1, 8, 1, m._ptr(p), None, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_kmeans(m._ptr(p), 64, 1, 8, 1, None, None, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_kmeans(m._ptr(p), 64, 1, 0, 1, m._ptr(p), None, None) == m.HXQ_EINVAL
+    cnt = np.zeros(1, np.int64)
+    assert m.lib.hxq_encode(None, 0, 8, 8, m._ptr(p), 0.1, m._ptr(lab), None, None, 0, m._ptr(cnt),
+                            None) == m.HXQ_EINVAL
+    assert m.lib.hxq_encode(m._ptr(p), 0, 8, 8, m._ptr(p), 0.1, m._ptr(lab), None, None, 0, None,
+                            None) == m.HXQ_EINVAL
+
+
 def test_create_without_device_reports_unsupported():
     import torch
     if torch.cuda.is_available():

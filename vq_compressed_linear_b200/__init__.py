@@ -62,13 +62,19 @@ lib.hxq_group_forward.argtypes = [_vp, _vp, ctypes.POINTER(_vp), ctypes.POINTER(
 lib.hxq_group_forward.restype = _i
 lib.hxq_group_destroy.argtypes = [_vp]
 lib.hxq_group_destroy.restype = None
+lib.hxq_assign.argtypes = [_vp, _i64, _i, _vp, _i, _vp, _vp]
+lib.hxq_assign.restype = _i
+lib.hxq_kmeans.argtypes = [_vp, _i64, _i, _i, _i, _vp, _vp, _vp]
+lib.hxq_kmeans.restype = _i
+lib.hxq_encode.argtypes = [_vp, _i, _i, _i, _vp, ctypes.c_float, _vp, _vp, _vp, _i64, _vp, _vp]
+lib.hxq_encode.restype = _i
 lib.hxq_linear_destroy.argtypes = [_vp]
 lib.hxq_linear_destroy.restype = None
 lib.hxq_strerror.argtypes = [_i]
 lib.hxq_strerror.restype = ctypes.c_char_p
 
 EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_linear_forward_out",
-            "hxq_linear_forward_noalloc", "hxq_group_create", "hxq_group_forward", "hxq_group_destroy", "hxq_decode",
+            "hxq_linear_forward_noalloc", "hxq_group_create", "hxq_group_forward", "hxq_group_destroy", "hxq_assign", "hxq_kmeans", "hxq_encode", "hxq_decode",
             "hxq_linear_check", "hxq_linear_info", "hxq_linear_destroy", "hxq_strerror")
 
 
@@ -155,6 +161,23 @@ def hxq_group_forward(g, x, biases, ys, out_dtype, M, stream=None) -> None:
 
 def hxq_group_destroy(g) -> None:
     lib.hxq_group_destroy(g)
+
+
+def hxq_assign(points, n, dim, centroids, k, labels, stream=None) -> None:
+    _check(lib.hxq_assign(_ptr(points), int(n), int(dim), _ptr(centroids), int(k), _ptr(labels), _stream(stream)),
+           "hxq_assign")
+
+
+def hxq_kmeans(points, n, dim, k, iters, centroids, labels, stream=None) -> None:
+    _check(lib.hxq_kmeans(_ptr(points), int(n), int(dim), int(k), int(iters), _ptr(centroids), _ptr(labels),
+                          _stream(stream)), "hxq_kmeans")
+
+
+def hxq_encode(W, mode, N, K, codebook, threshold, indices, sidecar_pos, sidecar_val, max_sidecar, n_sidecar,
+               stream=None) -> None:
+    _check(lib.hxq_encode(_ptr(W), int(mode), int(N), int(K), _ptr(codebook), float(threshold), _ptr(indices),
+                          _ptr(sidecar_pos), _ptr(sidecar_val), int(max_sidecar), _ptr(n_sidecar),
+                          _stream(stream)), "hxq_encode")
 
 
 def hxq_decode(h, W_out, stream=None) -> None:
@@ -285,3 +308,41 @@ class HelixGroup:
             self.close()
         except Exception:
             pass
+
+
+# ---- encoder convenience ------------------------------------------------------
+
+def kmeans(points, init, iters, stream=None):
+    """Lloyd k-means on the GPU: points float32 CUDA [n] or [n, 2], init
+    [k] or [k, 2]. Returns (centroids like init, labels int16 bits of the
+    uint16 indices as an int32 tensor)."""
+    import torch
+    dim = 1 if points.dim() == 1 else int(points.shape[1])
+    n, k = int(points.shape[0]), int(init.shape[0])
+    cent = init.detach().to(device=points.device, dtype=torch.float32).contiguous().clone()
+    lab = torch.empty(n, dtype=torch.int16, device=points.device)
+    hxq_kmeans(points.contiguous(), n, dim, k, iters, cent, lab, stream)
+    return cent, lab.to(torch.int32) & 0xFFFF
+
+
+def encode(W, mode, codebook, threshold, max_sidecar=None, stream=None):
+    """Indices and sidecar of W (float32 CUDA [N, K]) for a trained codebook,
+    in the layout HelixLinear takes. Returns (indices uint8, sidecar_pos
+    int64, sidecar_val float32), all CUDA tensors."""
+    import torch
+    N, K = int(W.shape[0]), int(W.shape[1])
+    W = W.contiguous()
+    cb = codebook.to(device=W.device, dtype=torch.float32).contiguous()
+    nbytes = N * K if mode == HXQ_MODE_SCALAR8 else 3 * N * K // 4
+    idx = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    count = torch.zeros(1, dtype=torch.int64, device=W.device)
+    cap = max(1024, N * K // 100) if max_sidecar is None else int(max_sidecar)
+    while True:
+        pos = torch.empty(max(cap, 1), dtype=torch.int64, device=W.device)
+        val = torch.empty(max(cap, 1), dtype=torch.float32, device=W.device)
+        hxq_encode(W, mode, N, K, cb, threshold, idx, pos, val, cap, count, stream)
+        n = int(count.item())
+        if n <= cap or max_sidecar is not None:
+            m = min(n, cap)
+            return idx, pos[:m], val[:m]
+        cap = n
