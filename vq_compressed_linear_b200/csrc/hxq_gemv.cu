@@ -56,6 +56,7 @@
 #include <type_traits>
 
 #include "hxq_internal.cuh"
+#include "hxq_plan.h"
 
 namespace hxq {
 namespace {
@@ -753,36 +754,6 @@ cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, const Out& out, 
 }
 
 int mt_of(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
-
-// Stream-K shares of a group's grid: G CTAs, layer i getting about
-// G W[i] / sum W of them, at least 1 and at most W[i]; the CTAs left over
-// (or taken back) go to (come from) the layers with the most (fewest)
-// stages per CTA.
-void group_shares(const int64_t* W, int n, int G, int* Gl) {
-  int64_t Wt = 0;
-  for (int i = 0; i < n; ++i) Wt += W[i];
-  int sum = 0;
-  for (int i = 0; i < n; ++i) {
-    Gl[i] = (int)std::max<int64_t>(1, std::min<int64_t>(W[i], (int64_t)G * W[i] / Wt));
-    sum += Gl[i];
-  }
-  while (sum < G) {  // W[i] / Gl[i] largest among the layers that can take one more
-    int best = -1;
-    for (int i = 0; i < n; ++i)
-      if (Gl[i] < W[i] && (best < 0 || W[i] * Gl[best] > W[best] * Gl[i])) best = i;
-    if (best < 0) break;
-    ++Gl[best];
-    ++sum;
-  }
-  while (sum > G) {  // W[i] / Gl[i] smallest among the layers that can give one up
-    int best = -1;
-    for (int i = 0; i < n; ++i)
-      if (Gl[i] > 1 && (best < 0 || W[i] * Gl[best] < W[best] * Gl[i])) best = i;
-    if (best < 0) break;
-    --Gl[best];
-    --sum;
-  }
-}
 
 template <int MT, bool XF32, int MODE>
 cudaError_t launch_group_cfg(const hxq_group& g, const uint16_t* x, const Out* outs, int M, cudaStream_t s) {
