@@ -106,9 +106,10 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode,
 /*
  * y[M][N] = x[M][K] . W^T on `stream` (a cudaStream_t; NULL = legacy default
  * stream). x (bf16 bits) and y (float) are device pointers; x must be 16-byte
- * aligned. Asynchronous: returns after the launch. M >= 1.
- * Returns HXQ_EINVAL for a NULL handle/x/y, M < 1 or a misaligned x;
- * HXQ_ECUDA if a launch fails.
+ * aligned. Asynchronous: returns after the launch. M >= 1. The handle's
+ * device must be the current one (as for every call that takes a handle).
+ * Returns HXQ_EINVAL for a NULL handle/x/y, M < 1, a misaligned x or
+ * another device current; HXQ_ECUDA if a launch fails.
  */
 int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M,
                        void* stream);

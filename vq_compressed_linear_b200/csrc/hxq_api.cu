@@ -265,12 +265,24 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
 }
 
 namespace {
+// The handle's device must be current: a launch on another device would
+// hand its kernels pointers they cannot use. 0 if it is, else a status.
+int check_device(int device) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_ECUDA;
+  }
+  return dev == device ? HXQ_OK : HXQ_EINVAL;
+}
+
 int forward_impl(hxq_linear_t h, const void* x_bf16, const hxq::Out& out, int M, int kernel, int split_k,
                  void* stream) {
   if (!h || !x_bf16 || !out.y || M < 1) return HXQ_EINVAL;
   if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) != 0) return HXQ_EINVAL;
   if (kernel < HXQ_KERNEL_AUTO || kernel > HXQ_KERNEL_TC) return HXQ_EINVAL;
   if (split_k < 0 || split_k > hxq::kMaxSplitK) return HXQ_EINVAL;
+  if (const int rc = check_device(h->device)) return rc;
   if (kernel == HXQ_KERNEL_AUTO) kernel = (M <= 4 && hxq::gemv_supports(*h, M)) ? HXQ_KERNEL_GEMV : HXQ_KERNEL_TC;
   if (kernel == HXQ_KERNEL_GEMV && !hxq::gemv_supports(*h, M)) return HXQ_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -333,6 +345,7 @@ int hxq_group_forward(hxq_group_t g, const void* x_bf16, const float* const* bia
   if (!g || !x_bf16 || !y || M < 1) return HXQ_EINVAL;
   if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) != 0) return HXQ_EINVAL;
   if (out_dtype != HXQ_OUT_F32 && out_dtype != HXQ_OUT_BF16) return HXQ_EINVAL;
+  if (const int rc = check_device(g->device)) return rc;
   hxq::Out outs[hxq::kMaxGroup];
   for (int i = 0; i < g->n; ++i) {
     if (!y[i]) return HXQ_EINVAL;
@@ -358,6 +371,7 @@ void hxq_group_destroy(hxq_group_t g) { delete g; }
 
 int hxq_decode(hxq_linear_t h, float* W_out, void* stream) {
   if (!h || !W_out) return HXQ_EINVAL;
+  if (const int rc = check_device(h->device)) return rc;
   cudaError_t e = hxq::launch_decode(*h, W_out, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
