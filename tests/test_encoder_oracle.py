@@ -2,10 +2,9 @@
 selection and the full encode, each checked against something other than
 its own formula -- exact integer brute force on dyadic inputs, the midpoint
 rule, scikit-learn's Lloyd k-means, Lloyd's monotone objective, weights drawn
-exactly from a codebook -- and planted mistakes that those pins must catch.
+exactly from a codebook, hand-worked cases in tests/golden/tiny_kmeans.txt --
+and planted mistakes that those pins must catch.
 """
-import itertools
-
 import numpy as np
 import pytest
 
@@ -195,6 +194,7 @@ def _pins_pass():
         for mode in (0, 1):
             test_encode_recovers_weights_drawn_from_the_codebook(mode)
             test_sidecar_planted_outliers_dyadic(mode)
+        test_hand_worked_encoder_cases()
     except AssertionError:
         return False
     return True
@@ -243,3 +243,45 @@ def test_encoder_planted_mistakes_are_caught(monkeypatch, mutant):
             return pos, val
         monkeypatch.setattr(enc, "sidecar_select", select_colmajor)
     assert not _pins_pass(), f"planted mistake {mutant} was not caught"
+
+
+# ----------------------------------------------------------------- hand-worked fixtures
+
+def _golden_cases():
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_kmeans.txt")
+    cases = []
+    for raw in open(path):
+        line = raw.split("#", 1)[0].strip()
+        if not line:
+            continue
+        kind, rest = line.split(":", 1)
+        cases.append((kind.strip(), [f.split() for f in rest.split("|")]))
+    return cases
+
+
+def _arr(tokens, dim=1):
+    a = np.array([float(t) for t in tokens], np.float32)
+    return a.reshape(-1, dim) if dim == 2 else a
+
+
+def test_hand_worked_encoder_cases():
+    cases = _golden_cases()
+    assert {k for k, _ in cases} == {"kmeans", "assign", "sidecar"}
+    for kind, f in cases:
+        name = f[0][0]
+        if kind == "kmeans":
+            dim = int(f[1][0])
+            c, lab = enc.kmeans(_arr(f[2], dim), _arr(f[3], dim), int(f[4][0]))
+            assert np.array_equal(c, _arr(f[5], dim)), name
+            assert np.array_equal(lab, [int(t) for t in f[6]]), name
+        elif kind == "assign":
+            dim = int(f[1][0])
+            assert np.array_equal(enc.assign(_arr(f[2], dim), _arr(f[3], dim)), [int(t) for t in f[4]]), name
+        else:
+            cb, w, t = _arr(f[1]), _arr(f[2]), float(f[3][0])
+            lab = enc.assign(w, cb)
+            assert np.array_equal(lab, [int(v) for v in f[4]]), name
+            pos, val = enc.sidecar_select(w, cb[lab], t)
+            assert np.array_equal(pos, [int(v) for v in f[5]]), name
+            assert np.array_equal(val, _arr(f[6])), name
