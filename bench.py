@@ -416,16 +416,63 @@ ENCODER_ROUNDS = 10
 ENCODER_OPS = {1: 4, 2: 8}
 
 
+# (mode, N, K, codebook entries, sidecar threshold)
+ENCODER_SHAPES = {"scalar": (0, 8512, 2048, 256, 0.002), "vq2d": (1, 11008, 4096, 4096, 0.006),
+                  "tiny": (0, 256, 256, 256, 0.002)}
+
+
+def encoder_layer(name):
+    """The encoder workload: W ~ N(0, 0.02) fp32 [N][K] and k start centroids
+    drawn from its points (seeded), the same for both arms."""
+    mode, N, K, k, tau = ENCODER_SHAPES[name]
+    dim = 1 if mode == 0 else 2
+    rng = np.random.default_rng(0)
+    W = rng.normal(0, 0.02, size=(N, K)).astype(np.float32)
+    pts = W.reshape(-1, dim)
+    init = pts[rng.choice(pts.shape[0], k, replace=False)].copy()
+    return mode, N, K, k, tau, dim, W, init
+
+
+def encoder_workload_name(name):
+    mode, N, K, k, tau = ENCODER_SHAPES[name]
+    return f"encode {N}x{K} mode {mode}, k={k}, {ENCODER_ROUNDS} k-means rounds, threshold {tau}"
+
+
+def oracle_encoder_arm(name, steps, warmup, budget_s=60.0):
+    """--impl reference --encoder: the oracle's k-means rounds and encode on
+    the first rows of the same layer, sized so that W + K steps take about
+    budget_s. Returns (weights/s, description, threads, seconds)."""
+    import oracle
+    enc = oracle.hxq_encoder_oracle
+    mode, N, K, k, tau, dim, W, init = encoder_layer(name)
+    est_s = (ENCODER_ROUNDS + 2) * (W.size // dim) * k * 3e-9  # ~3 ns per point-centroid cell
+    rows = max(1, min(N, int(N * budget_s / max(1, steps + warmup) / max(est_s, 1e-9))))
+    Ws = W[:rows]
+    pts = Ws.reshape(-1, dim)
+    start = init if dim == 2 else init[:, 0]
+
+    def step():
+        c, _ = enc.kmeans(pts, start, ENCODER_ROUNDS)
+        enc.encode(Ws, mode, c.reshape(-1), tau)
+
+    for _ in range(warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    tt = time.perf_counter() - t0
+    desc = f"{steps} oracle steps on the first {rows} of {N} rows"
+    return rows * K * steps / tt, desc, _oracle_threads(), tt
+
+
 def encoder_run(hxq, torch, args):
     """One step = ENCODER_ROUNDS k-means rounds on one layer's weights plus
     its encode (indices + sidecar); metric: weights per second."""
-    mode, N, K, k = (0, 8512, 2048, 256) if args.encoder == "scalar" else (1, 11008, 4096, 4096)
-    dim = 1 if mode == 0 else 2
-    rng = np.random.default_rng(0)
-    W = torch.from_numpy(rng.normal(0, 0.02, size=(N, K)).astype(np.float32)).cuda()
+    mode, N, K, k, tau, dim, W_h, init_h = encoder_layer(args.encoder)
+    W = torch.from_numpy(W_h).cuda()
     pts = W.view(-1, dim) if dim == 2 else W.view(-1)
     n = pts.shape[0]
-    init = pts[torch.from_numpy(rng.choice(n, k, replace=False)).cuda()].clone()
+    init = torch.from_numpy(init_h if dim == 2 else init_h[:, 0].copy()).cuda()
     cent = torch.empty_like(init)
     labels = torch.empty(n, dtype=torch.int16, device="cuda")
     idx = torch.empty(N * K if mode == 0 else 3 * N * K // 4, dtype=torch.uint8, device="cuda")
@@ -433,7 +480,6 @@ def encoder_run(hxq, torch, args):
     pos = torch.empty(cap, dtype=torch.int64, device="cuda")
     val = torch.empty(cap, dtype=torch.float32, device="cuda")
     cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
-    tau = 0.002 if mode == 0 else 0.006
     stream = torch.cuda.Stream()
 
     def step():
@@ -462,8 +508,7 @@ def encoder_run(hxq, torch, args):
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": f"encode {N}x{K} mode {mode}, k={k}, {ENCODER_ROUNDS} k-means rounds, "
-                                   f"threshold {tau}", "sidecar_entries": int(cnt.item())},
+            "config": {"workload": encoder_workload_name(args.encoder), "sidecar_entries": int(cnt.item())},
             "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "comparisons/s",
                          "frac": achieved / peak, "traffic": None,
                          "peak_kind": f"derived: SMs x 128 fp32 lanes x {clock_ghz} GHz / {ENCODER_OPS[dim]} "
@@ -486,9 +531,10 @@ def main():
     ap.add_argument("--grouped", action="store_true",
                     help="run the layers that share their input as one grouped forward each")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--encoder", choices=["scalar", "vq2d"], default=None,
-                    help="time the GPU encoder instead (k-means rounds + encode of one layer): "
-                         "scalar = in_proj 8512x2048, k=256; vq2d = 11008x4096 pairs, k=4096")
+    ap.add_argument("--encoder", choices=sorted(ENCODER_SHAPES), default=None,
+                    help="time the encoder instead (k-means rounds + encode of one layer): "
+                         "scalar = in_proj 8512x2048, k=256; vq2d = 11008x4096 pairs, k=4096; "
+                         "tiny = 256x256, k=256")
     ap.add_argument("--ncu", action="store_true",
                     help="minimal run for profilers: enough layer replicas to exceed L2, then "
                          "W + K eager steps; prints nothing")
@@ -511,6 +557,17 @@ def main():
 
     if args.impl == "reference":
         if rank != 0:
+            return 0
+        if args.encoder:
+            v, sample, threads, secs = oracle_encoder_arm(args.encoder, args.steps, args.warmup)
+            print(json.dumps({
+                "impl": "reference", "metric": "HXQ encoder weights/s", "value": v, "unit": "weights/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": encoder_workload_name(args.encoder)},
+                "cpu_baseline": {"value": v, "unit": "weights/s", "cores": threads, "kind": "oracle",
+                                 "sample": sample + f" ({secs:.1f} s)"},
+                "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
             return 0
         gbs, tfs, sample, threads, secs = oracle_reference_arm(items, args.steps, args.warmup)
         v = tfs if is_prefill else gbs

@@ -111,3 +111,19 @@ def test_item_groups_pick_layers_sharing_input():
     assert bench.item_groups("mamba2", [("in_proj/M=1", None, 1), ("out_proj/M=1", None, 1)]) == []
     # a group with one member left is no group
     assert bench.item_groups("qwen25_3b", [("q/M=1", None, 1), ("o/M=1", None, 1)]) == []
+
+
+def test_reference_arm_encoder_line():
+    """--impl reference --encoder: the oracle's k-means rounds and encode,
+    one JSON line with the encoder metric and the reference fields."""
+    env = dict(os.environ, RANK="0", LOCAL_RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--encoder", "tiny", "--steps", "3", "--warmup", "3"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == "HXQ encoder weights/s" and d["unit"] == "weights/s"
+    assert d["config"]["workload"].startswith("encode 256x256 mode 0, k=256")
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["value"] > 0
