@@ -94,7 +94,7 @@ enum {
  * independent.
  *
  * Returns HXQ_EINVAL for: NULL codebook/indices/out, NULL sidecar arrays with
- * n_sidecar > 0, n_sidecar < 0 or > N*K, N < 1, K < 8, K % 8 != 0, unknown
+ * n_sidecar > 0, n_sidecar < 0, > N*K or >= 2^31, N < 1, K < 8, K % 8 != 0, unknown
  * mode, a sidecar position outside [0, N*K) or repeated. HXQ_EUNSUPPORTED if
  * the current device is not compute capability 10.0. HXQ_ENOMEM / HXQ_ECUDA
  * on allocation / copy failures (nothing is leaked).

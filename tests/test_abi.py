@@ -135,3 +135,36 @@ def test_create_without_device_reports_unsupported():
 def test_build_flags_target_sm100a():
     import __graft_entry__
     assert __graft_entry__._builder().ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_create_argument_rules_fuzzed():
+    """hxq_linear_create's documented argument rules, over random shapes,
+    modes, sidecar counts and NULL pointers: every violation returns
+    HXQ_EINVAL before any CUDA call; arguments that pass reach the device
+    check (HXQ_EUNSUPPORTED here, without a GPU)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    from hypothesis import given, settings, strategies as st
+    import vq_compressed_linear_b200 as m
+
+    cb = np.zeros(8192, np.float32)
+    idx = np.zeros(64, np.uint8)
+    pos = np.zeros(4, np.int64)
+    val = np.zeros(4, np.float32)
+
+    @settings(max_examples=400, deadline=None, derandomize=True)
+    @given(mode=st.integers(-1, 3), N=st.integers(-2, 1 << 20), K=st.integers(-16, 1 << 16),
+           ns=st.one_of(st.integers(-3, 8), st.sampled_from([(1 << 31) - 1, 1 << 31, 1 << 40])),
+           null_cb=st.booleans(), null_idx=st.booleans(), null_side=st.booleans(), null_out=st.booleans())
+    def check(mode, N, K, ns, null_cb, null_idx, null_side, null_out):
+        invalid = (null_cb or null_idx or null_out or mode not in (0, 1) or N < 1 or K < 8 or K % 8
+                   or ns < 0 or ns > N * K or (ns > 0 and null_side) or ns >= (1 << 31))
+        h = ctypes.c_void_p()
+        rc = m.lib.hxq_linear_create(None if null_cb else m._ptr(cb), None if null_idx else m._ptr(idx), mode,
+                                     None if null_side else m._ptr(pos), None if null_side else m._ptr(val),
+                                     ns, N, K, None if null_out else ctypes.byref(h))
+        assert rc == (m.HXQ_EINVAL if invalid else m.HXQ_EUNSUPPORTED), (mode, N, K, ns)
+        assert h.value is None
+
+    check()
