@@ -168,3 +168,50 @@ def test_create_argument_rules_fuzzed():
         assert h.value is None
 
     check()
+
+
+def test_encoder_argument_rules_fuzzed():
+    """hxq_assign / hxq_kmeans / hxq_encode: every documented argument error
+    returns HXQ_EINVAL before any CUDA call; arguments that pass go on to
+    the launch, which fails here without a GPU (HXQ_ECUDA), except a
+    k-means call with nothing to do (no rounds, no labels): HXQ_OK."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    from hypothesis import given, settings, strategies as st
+    import vq_compressed_linear_b200 as m
+
+    buf = np.zeros(64, np.float32)
+    lab = np.zeros(64, np.uint16)
+    cnt = np.zeros(1, np.int64)
+    P = lambda null: None if null else m._ptr(buf)
+    big = st.sampled_from([(1 << 31) - 1, 1 << 31, 1 << 40])
+
+    @settings(max_examples=300, deadline=None, derandomize=True)
+    @given(n=st.one_of(st.integers(-2, 100), big), dim=st.integers(0, 3), k=st.integers(-1, 4100),
+           iters=st.integers(-2, 3), nulls=st.lists(st.booleans(), min_size=3, max_size=3))
+    def check_assign_kmeans(n, dim, k, iters, nulls):
+        shape_bad = n < 1 or n >= (1 << 31) or dim not in (1, 2) or k < 1 or k > 4096
+        rc = m.lib.hxq_assign(P(nulls[0]), n, dim, P(nulls[1]), k, None if nulls[2] else m._ptr(lab), None)
+        assert rc == (m.HXQ_EINVAL if shape_bad or any(nulls) else m.HXQ_ECUDA), ("assign", n, dim, k, nulls)
+        rc = m.lib.hxq_kmeans(P(nulls[0]), n, dim, k, iters, P(nulls[1]), None if nulls[2] else m._ptr(lab), None)
+        if shape_bad or nulls[0] or nulls[1] or iters < 0:
+            want = m.HXQ_EINVAL
+        else:
+            want = m.HXQ_OK if iters == 0 and nulls[2] else m.HXQ_ECUDA
+        assert rc == want, ("kmeans", n, dim, k, iters, nulls)
+
+    @settings(max_examples=300, deadline=None, derandomize=True)
+    @given(mode=st.integers(-1, 2), N=st.integers(-1, 1 << 20), K=st.integers(-8, 1 << 14),
+           t=st.sampled_from([0.0, 0.5, -1e-9, float("nan"), float("inf")]), cap=st.integers(-2, 5),
+           nulls=st.lists(st.booleans(), min_size=5, max_size=5))
+    def check_encode(mode, N, K, t, cap, nulls):
+        bad = (nulls[0] or nulls[1] or nulls[2] or nulls[3] or mode not in (0, 1) or N < 1 or K < 8 or K % 8
+               or N * K >= (1 << 31) or not (t >= 0) or cap < 0 or (cap > 0 and nulls[4]))
+        side = None if nulls[4] else m._ptr(buf)
+        rc = m.lib.hxq_encode(P(nulls[0]), mode, N, K, P(nulls[1]), t, P(nulls[2]), side, side, cap,
+                              None if nulls[3] else m._ptr(cnt), None)
+        assert rc == (m.HXQ_EINVAL if bad else m.HXQ_ECUDA), (mode, N, K, t, cap, nulls)
+
+    check_assign_kmeans()
+    check_encode()
