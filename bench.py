@@ -407,6 +407,16 @@ def profile_run(hxq, torch, items, steps, warmup):
     return 0
 
 
+def run_env(torch, device):
+    """What the numbers were taken on: GPU, SM count, torch and CUDA versions."""
+    try:
+        props = torch.cuda.get_device_properties(device)
+        return {"gpu": props.name, "sms": props.multi_processor_count, "torch": torch.__version__,
+                "cuda": torch.version.cuda}
+    except Exception as e:  # the record must not cost the measurement
+        return {"error": type(e).__name__}
+
+
 # ----------------------------------------------------------------------------- encoder
 
 ENCODER_ROUNDS = 10
@@ -651,7 +661,8 @@ def main():
             "roofline": roof,
             "e2e": {"value": e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * launches,
-            "clocks": clocks}
+            "clocks": clocks,
+            "env": run_env(torch, local_rank)}
 
     if not args.no_secondary and world == 1:
         sec = []

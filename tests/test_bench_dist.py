@@ -127,3 +127,11 @@ def test_reference_arm_encoder_line():
     assert d["impl"] == "reference" and d["metric"] == "HXQ encoder weights/s" and d["unit"] == "weights/s"
     assert d["config"]["workload"].startswith("encode 256x256 mode 0, k=256")
     assert d["cpu_baseline"]["kind"] == "oracle" and d["value"] > 0
+
+
+def test_run_env_never_raises():
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    env = bench.run_env(torch, 0)
+    assert ("gpu" in env and "torch" in env) or "error" in env
