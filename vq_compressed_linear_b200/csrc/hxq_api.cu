@@ -108,8 +108,8 @@ const char* hxq_strerror(int code) {
   }
 }
 
-int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, const int64_t* sidecar_pos,
-                      const float* sidecar_val, int64_t n_sidecar, int N, int K, hxq_linear_t* out) {
+static int create_impl(const float* codebook, const uint8_t* indices, int mode, const int64_t* sidecar_pos,
+                       const float* sidecar_val, int64_t n_sidecar, int N, int K, hxq_linear_t* out) {
   // ---- pure argument checks: no CUDA call before these pass
   if (!out) return HXQ_EINVAL;
   *out = nullptr;
@@ -262,6 +262,18 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, c
   }
   *out = h;
   return HXQ_OK;
+}
+
+// No C++ exception may cross the C boundary: a host allocation that fails
+// (sidecar lists of absurd size) reports HXQ_ENOMEM instead.
+int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode, const int64_t* sidecar_pos,
+                      const float* sidecar_val, int64_t n_sidecar, int N, int K, hxq_linear_t* out) {
+  try {
+    return create_impl(codebook, indices, mode, sidecar_pos, sidecar_val, n_sidecar, N, K, out);
+  } catch (const std::bad_alloc&) {
+    cudaGetLastError();
+    return HXQ_ENOMEM;
+  }
 }
 
 namespace {
