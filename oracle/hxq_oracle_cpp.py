@@ -1,0 +1,72 @@
+"""ctypes wrapper of the plain C++ oracle (oracle/hxq_oracle_ref.cpp) --
+TEST INFRASTRUCTURE, used only by the tests to check it against the numpy
+oracle. build() compiles it with the host C++ compiler next to its source;
+the CUDA library never loads it."""
+from __future__ import annotations
+
+import ctypes
+import os
+import shutil
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "hxq_oracle_ref.cpp")
+LIB = os.path.join(HERE, "libhxq_oracle_ref.so")
+_lib = None
+
+
+def build() -> str:
+    """Compile the oracle (no fused multiply-add contraction, so every
+    product and sum is rounded as written)."""
+    cxx = os.environ.get("CXX") or shutil.which("g++") or shutil.which("c++")
+    if not cxx:
+        raise RuntimeError("no host C++ compiler")
+    tmp = LIB + ".tmp"
+    subprocess.run([cxx, "-O2", "-std=c++17", "-ffp-contract=off", "-fPIC", "-shared", SRC, "-o", tmp],
+                   check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+            build()
+        lib = ctypes.CDLL(LIB)
+        vp, i, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        lib.oracle_decode.argtypes = [i, vp, vp, vp, vp, i64, i, i, vp]
+        lib.oracle_decode.restype = i
+        lib.oracle_forward.argtypes = [vp, vp, i, i, i, vp, vp]
+        lib.oracle_forward.restype = None
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def decode(mode, codebook, indices, sidecar_pos, sidecar_val, N, K) -> np.ndarray:
+    cb = np.ascontiguousarray(codebook, dtype=np.float32)
+    idx = np.ascontiguousarray(indices, dtype=np.uint8)
+    pos = np.ascontiguousarray(sidecar_pos, dtype=np.int64).reshape(-1)
+    val = np.ascontiguousarray(sidecar_val, dtype=np.float32).reshape(-1)
+    W = np.empty((N, K), dtype=np.float32)
+    rc = _load().oracle_decode(int(mode), _p(cb), _p(idx), _p(pos), _p(val), int(pos.size), int(N), int(K), _p(W))
+    if rc != 0:
+        raise ValueError("invalid layer")
+    return W
+
+
+def forward(x_bits, W) -> tuple[np.ndarray, np.ndarray]:
+    x = np.ascontiguousarray(np.atleast_2d(x_bits), dtype=np.uint16)
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    M, K = x.shape
+    N = W.shape[0]
+    y = np.empty((M, N), np.float64)
+    s = np.empty((M, N), np.float64)
+    _load().oracle_forward(_p(x), _p(W), int(M), int(N), int(K), _p(y), _p(s))
+    return y, s

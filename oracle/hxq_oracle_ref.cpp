@@ -1,0 +1,89 @@
+// Plain C++ oracle of the HXQ HelixLinear forward -- TEST INFRASTRUCTURE.
+//
+// A second, independently written CPU oracle beside oracle/hxq_oracle.py
+// (numpy): the tests check that the two agree, decode bit for bit and the
+// forward to float64 rounding. Only the tests load it; the CUDA library
+// never includes, links or calls it, and the two share no code.
+//
+// What it computes, as plain loops in the definition's order:
+//  * scalar mode: W[n][k] = codebook[indices[n*K + k]] (Zamba2-1.2B-HXQ model
+//    card, "What is HelixCode?": 256-entry fp32 codebook, one uint8 index per
+//    weight);
+//  * 2D mode: pair g = n*K/2 + k/2 of the row-major pair stream has a 12-bit
+//    index; group g/2 of the index bytes is the little-endian 24-bit word
+//    b0 | b1<<8 | b2<<16 whose low 12 bits index the even pair and high 12
+//    bits the odd one; W[n][k] = codebook[2*index + (k & 1)] (HXQ whitepaper,
+//    method section: 2D VQ paragraph and "12-bit index packing");
+//  * sidecar: W[p / K][p % K] = value for every (p, value) (HXQ whitepaper,
+//    method section, "Sidecar outlier correction", read as replacement);
+//  * y[m][n] = sum over k, in k order, of double(x[m][k]) * double(W[n][k]),
+//    x widened exactly from its bf16 bits; s[m][n] the same sum of absolute
+//    values (the tolerance scale).
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+namespace {
+
+double bf16_to_double(uint16_t bits) {
+  const uint32_t u = (uint32_t)bits << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+}  // namespace
+
+extern "C" {
+
+// Decoded weights W [N][K] (fp32). Returns 0, or -1 for an unknown mode, a
+// bad shape, or a sidecar position out of range or repeated.
+int oracle_decode(int mode, const float* codebook, const uint8_t* indices, const int64_t* sidecar_pos,
+                  const float* sidecar_val, int64_t n_sidecar, int N, int K, float* W) {
+  if (N < 1 || K < 1) return -1;
+  const int64_t NK = (int64_t)N * K;
+  if (mode == 0) {
+    for (int64_t p = 0; p < NK; ++p) W[p] = codebook[indices[p]];
+  } else if (mode == 1) {
+    if (K % 4 != 0) return -1;
+    for (int n = 0; n < N; ++n) {
+      for (int k = 0; k < K; ++k) {
+        const int64_t g = (int64_t)n * (K / 2) + k / 2;  // pair
+        const int64_t grp = g / 2;                        // 3-byte group
+        const uint32_t word = (uint32_t)indices[3 * grp] | ((uint32_t)indices[3 * grp + 1] << 8) |
+                              ((uint32_t)indices[3 * grp + 2] << 16);
+        const uint32_t e = (g % 2 == 0) ? (word & 0xFFFu) : (word >> 12);
+        W[(int64_t)n * K + k] = codebook[2 * e + (k % 2)];
+      }
+    }
+  } else {
+    return -1;
+  }
+  std::vector<char> seen(n_sidecar > 0 ? (size_t)NK : 0, 0);
+  for (int64_t i = 0; i < n_sidecar; ++i) {
+    const int64_t p = sidecar_pos[i];
+    if (p < 0 || p >= NK || seen[(size_t)p]) return -1;
+    seen[(size_t)p] = 1;
+    W[p] = sidecar_val[i];
+  }
+  return 0;
+}
+
+// y[m][n] and s[m][n] (float64) for x [M][K] given as bf16 bits.
+void oracle_forward(const uint16_t* x_bits, const float* W, int M, int N, int K, double* y, double* s) {
+  for (int m = 0; m < M; ++m) {
+    for (int n = 0; n < N; ++n) {
+      double acc = 0.0, mag = 0.0;
+      for (int k = 0; k < K; ++k) {
+        const double xv = bf16_to_double(x_bits[(int64_t)m * K + k]);
+        const double wv = (double)W[(int64_t)n * K + k];
+        acc += xv * wv;
+        mag += (xv < 0 ? -xv : xv) * (wv < 0 ? -wv : wv);
+      }
+      y[(int64_t)m * N + n] = acc;
+      s[(int64_t)m * N + n] = mag;
+    }
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+"""The plain C++ oracle (oracle/hxq_oracle_ref.cpp) against the hand-worked
+golden layers and against the numpy oracle: two independently written CPU
+oracles of the same definition must decode identically, bit for bit, and
+agree on the forward to float64 rounding (their sums run in different
+orders); on dyadic layers with integer activations both are exact, so they
+agree exactly."""
+import numpy as np
+import pytest
+
+import golden_io
+import oracle
+import synthetic
+from oracle import hxq_oracle_cpp as cpp
+
+
+@pytest.mark.parametrize("name", ["tiny_scalar.txt", "tiny_vq2d.txt"])
+def test_cpp_oracle_golden_layers(name):
+    layer, x, W, y, s = golden_io.tiny_layer(name)
+    Wc = cpp.decode(layer["mode"], layer["codebook"], layer["indices"], layer["sidecar_pos"],
+                    layer["sidecar_val"], layer["N"], layer["K"])
+    assert np.array_equal(Wc, W.astype(np.float32))
+    bits = synthetic.f32_to_bf16_bits(x.astype(np.float32))
+    yc, sc = cpp.forward(bits, Wc)
+    assert np.array_equal(yc, y) and np.array_equal(sc, s)
+
+
+@pytest.mark.parametrize("mode,N,K,ns", [(0, 130, 72, 40), (0, 3, 8, 0), (1, 129, 136, 60), (1, 7, 64, 7)])
+@pytest.mark.parametrize("M", [1, 5])
+def test_cpp_oracle_matches_numpy_oracle(mode, N, K, ns, M):
+    layer = synthetic.make_layer(mode, N, K, 900 + N, sidecar_count=ns)
+    x = synthetic.activations(M, K, 901)
+    args = (mode, layer["codebook"], layer["indices"], layer["sidecar_pos"], layer["sidecar_val"], N, K)
+    Wn = oracle.decode(*args)
+    Wc = cpp.decode(*args)
+    assert np.array_equal(Wc, Wn)
+    yn, sn = oracle.forward(x, Wn), oracle.abs_scale(x, Wn)
+    yc, sc = cpp.forward(x, Wc)
+    tol = 1e-12 * sn
+    assert np.all(np.abs(yc - yn) <= tol) and np.all(np.abs(sc - sn) <= tol)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_cpp_oracle_dyadic_exact_agreement(mode):
+    rng = np.random.default_rng(910 + mode)
+    N, K, M = 40, 64, 3
+    if mode == 0:
+        cb = (rng.integers(-64, 64, 256) * 2.0 ** -6).astype(np.float32)
+        idx = rng.integers(0, 256, N * K).astype(np.uint8)
+    else:
+        cb = (rng.integers(-64, 64, 8192) * 2.0 ** -6).astype(np.float32)
+        idx = oracle.pack12(rng.integers(0, 4096, N * K // 2))
+    pos = rng.choice(N * K, 30, replace=False).astype(np.int64)
+    val = (rng.integers(-32, 32, 30) * 2.0 ** -3).astype(np.float32)
+    x = synthetic.f32_to_bf16_bits(rng.integers(-8, 8, (M, K)).astype(np.float32))
+    Wn = oracle.decode(mode, cb, idx, pos, val, N, K)
+    Wc = cpp.decode(mode, cb, idx, pos, val, N, K)
+    assert np.array_equal(Wc, Wn)
+    yc, sc = cpp.forward(x, Wc)
+    assert np.array_equal(yc, oracle.forward(x, Wn)) and np.array_equal(sc, oracle.abs_scale(x, Wn))
+
+
+def test_cpp_oracle_rejects_bad_layers():
+    cb = np.zeros(8192, np.float32)
+    idx = np.zeros(64, np.uint8)
+    with pytest.raises(ValueError):
+        cpp.decode(0, cb, idx, [3, 3], [1.0, 2.0], 8, 8)       # repeated position
+    with pytest.raises(ValueError):
+        cpp.decode(0, cb, idx, [64], [1.0], 8, 8)              # out of range
+    with pytest.raises(ValueError):
+        cpp.decode(2, cb, idx, [], [], 8, 8)                   # unknown mode
+    with pytest.raises(ValueError):
+        cpp.decode(1, cb, idx, [], [], 2, 6)                   # 2D needs K % 4 == 0
