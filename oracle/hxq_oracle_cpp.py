@@ -41,6 +41,12 @@ def _load():
         lib.oracle_decode.restype = i
         lib.oracle_forward.argtypes = [vp, vp, i, i, i, vp, vp]
         lib.oracle_forward.restype = None
+        lib.oracle_assign.argtypes = [vp, i64, i, vp, i, vp]
+        lib.oracle_assign.restype = None
+        lib.oracle_kmeans_update.argtypes = [vp, i64, i, vp, i, vp]
+        lib.oracle_kmeans_update.restype = None
+        lib.oracle_sidecar_select.argtypes = [vp, vp, i64, ctypes.c_float, vp, vp, i64]
+        lib.oracle_sidecar_select.restype = i64
         _lib = lib
     return _lib
 
@@ -70,3 +76,38 @@ def forward(x_bits, W) -> tuple[np.ndarray, np.ndarray]:
     s = np.empty((M, N), np.float64)
     _load().oracle_forward(_p(x), _p(W), int(M), int(N), int(K), _p(y), _p(s))
     return y, s
+
+
+def _pts(a):
+    p = np.ascontiguousarray(a, dtype=np.float32)
+    return p.reshape(-1, 1) if p.ndim == 1 else p
+
+
+def assign(points, centroids) -> np.ndarray:
+    p, c = _pts(points), _pts(centroids)
+    lab = np.empty(p.shape[0], np.int32)
+    _load().oracle_assign(_p(p), int(p.shape[0]), int(p.shape[1]), _p(c), int(c.shape[0]), _p(lab))
+    return lab.astype(np.int64)
+
+
+def kmeans_update(points, labels, centroids) -> np.ndarray:
+    p, c = _pts(points), _pts(centroids).copy()
+    lab = np.ascontiguousarray(labels, dtype=np.int32)
+    _load().oracle_kmeans_update(_p(p), int(p.shape[0]), int(p.shape[1]), _p(lab), int(c.shape[0]), _p(c))
+    return c
+
+
+def kmeans(points, init, iters):
+    c = _pts(init).copy()
+    for _ in range(int(iters)):
+        c = kmeans_update(points, assign(points, c), c)
+    return c.reshape(np.shape(init)), assign(points, c)
+
+
+def sidecar_select(W, W_hat, threshold):
+    w = np.ascontiguousarray(W, dtype=np.float32).reshape(-1)
+    wh = np.ascontiguousarray(W_hat, dtype=np.float32).reshape(-1)
+    pos = np.empty(w.size, np.int64)
+    val = np.empty(w.size, np.float32)
+    n = _load().oracle_sidecar_select(_p(w), _p(wh), int(w.size), float(threshold), _p(pos), _p(val), int(w.size))
+    return pos[:n].copy(), val[:n].copy()

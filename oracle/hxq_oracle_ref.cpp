@@ -19,6 +19,10 @@
 //  * y[m][n] = sum over k, in k order, of double(x[m][k]) * double(W[n][k]),
 //    x widened exactly from its bf16 bits; s[m][n] the same sum of absolute
 //    values (the tolerance scale).
+// The encoder functions below follow the same readings as the numpy encoder
+// oracle: fp32 distance decisions with ties to the lowest index, float64
+// means rounded to fp32 with empty clusters kept, a strict threshold on
+// |w - w_hat| that stores the weight itself.
 #include <cstdint>
 #include <cstring>
 #include <vector>
@@ -84,6 +88,74 @@ void oracle_forward(const uint16_t* x_bits, const float* W, int M, int N, int K,
       s[(int64_t)m * N + n] = mag;
     }
   }
+}
+
+// ---- encoder side (HXQ whitepaper, method section: "Per-tensor k-means",
+// "Index assignment", "Sidecar outlier correction"), as plain loops.
+
+// Nearest of k centroids [k][dim] for each of n points [n][dim]: fp32
+// distance |p - c| (dim 1) or dx*dx + dy*dy (dim 2), every operation rounded
+// to fp32 as written (compiled without contraction); a strictly smaller
+// distance wins, so ties keep the lowest index.
+void oracle_assign(const float* points, int64_t n, int dim, const float* centroids, int k, int32_t* labels) {
+  for (int64_t i = 0; i < n; ++i) {
+    float best = 0.f;
+    int bi = -1;
+    for (int e = 0; e < k; ++e) {
+      float d;
+      if (dim == 1) {
+        const float diff = points[i] - centroids[e];
+        d = diff < 0.f ? -diff : diff;
+      } else {
+        const float dx = points[2 * i] - centroids[2 * e];
+        const float dy = points[2 * i + 1] - centroids[2 * e + 1];
+        const float xx = dx * dx;
+        const float yy = dy * dy;
+        d = xx + yy;
+      }
+      if (bi < 0 || d < best) {
+        best = d;
+        bi = e;
+      }
+    }
+    labels[i] = bi;
+  }
+}
+
+// One Lloyd update: each centroid with points moves to their mean (float64
+// sum in point order, divided by the count, rounded to fp32); the others stay.
+void oracle_kmeans_update(const float* points, int64_t n, int dim, const int32_t* labels, int k,
+                          float* centroids) {
+  std::vector<double> sum((size_t)k * dim, 0.0);
+  std::vector<int64_t> count((size_t)k, 0);
+  for (int64_t i = 0; i < n; ++i) {
+    const int e = labels[i];
+    ++count[(size_t)e];
+    for (int d = 0; d < dim; ++d) sum[(size_t)e * dim + d] += (double)points[i * dim + d];
+  }
+  for (int e = 0; e < k; ++e)
+    if (count[(size_t)e] > 0)
+      for (int d = 0; d < dim; ++d)
+        centroids[(size_t)e * dim + d] = (float)(sum[(size_t)e * dim + d] / (double)count[(size_t)e]);
+}
+
+// Flat positions (ascending) where |w - w_hat| > t in fp32, and the weights
+// there; returns their number (at most cap are written).
+int64_t oracle_sidecar_select(const float* W, const float* W_hat, int64_t nw, float t, int64_t* pos, float* val,
+                              int64_t cap) {
+  int64_t c = 0;
+  for (int64_t p = 0; p < nw; ++p) {
+    const float diff = W[p] - W_hat[p];
+    const float err = diff < 0.f ? -diff : diff;
+    if (err > t) {
+      if (c < cap) {
+        pos[c] = p;
+        val[c] = W[p];
+      }
+      ++c;
+    }
+  }
+  return c;
 }
 
 }  // extern "C"

@@ -3,7 +3,9 @@ golden layers and against the numpy oracle: two independently written CPU
 oracles of the same definition must decode identically, bit for bit, and
 agree on the forward to float64 rounding (their sums run in different
 orders); on dyadic layers with integer activations both are exact, so they
-agree exactly."""
+agree exactly. Their encoder sides (assignment, Lloyd rounds, sidecar
+selection) take the same fp32 decisions and sum the means in the same
+order, so they agree bit for bit."""
 import numpy as np
 import pytest
 
@@ -70,3 +72,45 @@ def test_cpp_oracle_rejects_bad_layers():
         cpp.decode(2, cb, idx, [], [], 8, 8)                   # unknown mode
     with pytest.raises(ValueError):
         cpp.decode(1, cb, idx, [], [], 2, 6)                   # 2D needs K % 4 == 0
+
+
+# ----------------------------------------------------------------- encoder side
+
+enc = oracle.hxq_encoder_oracle
+
+
+@pytest.mark.parametrize("dim,k,n", [(1, 256, 20000), (2, 512, 8000), (2, 4096, 6000)])
+def test_cpp_encoder_matches_numpy_encoder(dim, k, n):
+    rng = np.random.default_rng(920 + dim + k)
+    pts = rng.normal(0, 0.02, size=(n, dim)).astype(np.float32)
+    init = pts[rng.choice(n, k, replace=False)].copy()
+    init[k // 3] = init[1]  # an exact tie
+    assert np.array_equal(cpp.assign(pts, init), enc.assign(pts, init))
+    # float64 means in the same (point) order: the same fp32 centroids, bit for bit
+    c_c, lab_c = cpp.kmeans(pts, init, 4)
+    c_n, lab_n = enc.kmeans(pts, init, 4)
+    assert np.array_equal(c_c, c_n) and np.array_equal(lab_c, lab_n)
+
+
+def test_cpp_sidecar_select_matches_numpy():
+    rng = np.random.default_rng(930)
+    W = rng.normal(0, 0.02, size=(64, 96)).astype(np.float32)
+    W_hat = (np.rint(W * 256) / 256).astype(np.float32)
+    for t in (0.0, 0.0005, 0.001, 0.00195312):
+        pc, vc = cpp.sidecar_select(W, W_hat, t)
+        pn, vn = enc.sidecar_select(W, W_hat, t)
+        assert np.array_equal(pc, pn) and np.array_equal(vc, vn)
+
+
+def test_cpp_encoder_hand_worked_cases():
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_kmeans.txt")
+    for raw in open(path):
+        line = raw.split("#", 1)[0].strip()
+        if not line.startswith("kmeans:"):
+            continue
+        f = [x.split() for x in line.split(":", 1)[1].split("|")]
+        dim = int(f[1][0])
+        arr = lambda t: np.array([float(v) for v in t], np.float32).reshape(-1, dim)
+        c, lab = cpp.kmeans(arr(f[2]), arr(f[3]), int(f[4][0]))
+        assert np.array_equal(c, arr(f[5])) and np.array_equal(lab, [int(v) for v in f[6]]), f[0]
