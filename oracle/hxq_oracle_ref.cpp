@@ -23,8 +23,11 @@
 // oracle: fp32 distance decisions with ties to the lowest index, float64
 // means rounded to fp32 with empty clusters kept, a strict threshold on
 // |w - w_hat| that stores the weight itself.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <numeric>
+#include <thread>
 #include <vector>
 
 namespace {
@@ -36,6 +39,17 @@ double bf16_to_double(uint16_t bits) {
   return (double)f;
 }
 
+// Decoded weight W[n][k] before the sidecar (fp32).
+float decode_one(int mode, const float* codebook, const uint8_t* indices, int K, int n, int k) {
+  if (mode == 0) return codebook[indices[(int64_t)n * K + k]];
+  const int64_t g = (int64_t)n * (K / 2) + k / 2;  // pair
+  const int64_t grp = g / 2;                        // 3-byte group
+  const uint32_t word = (uint32_t)indices[3 * grp] | ((uint32_t)indices[3 * grp + 1] << 8) |
+                        ((uint32_t)indices[3 * grp + 2] << 16);
+  const uint32_t e = (g % 2 == 0) ? (word & 0xFFFu) : (word >> 12);
+  return codebook[2 * e + (k % 2)];
+}
+
 }  // namespace
 
 extern "C" {
@@ -45,24 +59,11 @@ extern "C" {
 int oracle_decode(int mode, const float* codebook, const uint8_t* indices, const int64_t* sidecar_pos,
                   const float* sidecar_val, int64_t n_sidecar, int N, int K, float* W) {
   if (N < 1 || K < 1) return -1;
+  if (mode != 0 && mode != 1) return -1;
+  if (mode == 1 && K % 4 != 0) return -1;
   const int64_t NK = (int64_t)N * K;
-  if (mode == 0) {
-    for (int64_t p = 0; p < NK; ++p) W[p] = codebook[indices[p]];
-  } else if (mode == 1) {
-    if (K % 4 != 0) return -1;
-    for (int n = 0; n < N; ++n) {
-      for (int k = 0; k < K; ++k) {
-        const int64_t g = (int64_t)n * (K / 2) + k / 2;  // pair
-        const int64_t grp = g / 2;                        // 3-byte group
-        const uint32_t word = (uint32_t)indices[3 * grp] | ((uint32_t)indices[3 * grp + 1] << 8) |
-                              ((uint32_t)indices[3 * grp + 2] << 16);
-        const uint32_t e = (g % 2 == 0) ? (word & 0xFFFu) : (word >> 12);
-        W[(int64_t)n * K + k] = codebook[2 * e + (k % 2)];
-      }
-    }
-  } else {
-    return -1;
-  }
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) W[(int64_t)n * K + k] = decode_one(mode, codebook, indices, K, n, k);
   std::vector<char> seen(n_sidecar > 0 ? (size_t)NK : 0, 0);
   for (int64_t i = 0; i < n_sidecar; ++i) {
     const int64_t p = sidecar_pos[i];
@@ -88,6 +89,50 @@ void oracle_forward(const uint16_t* x_bits, const float* W, int M, int N, int K,
       s[(int64_t)m * N + n] = mag;
     }
   }
+}
+
+// The whole path for output rows [r0, r1) of a layer, for timing the oracle
+// on the host's cores: each row is decoded (sidecar entries of the row
+// replace their weights), then y[m][n - r0] = sum over k, in k order, of
+// double(x[m][k]) * double(W[n][k]) -- the arithmetic of oracle_decode and
+// oracle_forward, row by row. `threads` std::threads split the rows in
+// contiguous blocks. Returns 0, or -1 for a bad argument (positions are not
+// checked for repeats here).
+int oracle_forward_rows(int mode, const float* codebook, const uint8_t* indices, const int64_t* sidecar_pos,
+                        const float* sidecar_val, int64_t n_sidecar, int N, int K, const uint16_t* x_bits, int M,
+                        int r0, int r1, int threads, double* y) {
+  if (N < 1 || K < 1 || M < 1 || r0 < 0 || r1 > N || r0 >= r1 || threads < 1) return -1;
+  if (mode != 0 && mode != 1) return -1;
+  if (mode == 1 && K % 4 != 0) return -1;
+  // sidecar entries in position order, so that a row finds its own
+  std::vector<int64_t> order((size_t)n_sidecar);
+  std::iota(order.begin(), order.end(), (int64_t)0);
+  std::sort(order.begin(), order.end(), [&](int64_t a, int64_t b) { return sidecar_pos[a] < sidecar_pos[b]; });
+  const int64_t NK = (int64_t)N * K;
+  for (int64_t i = 0; i < n_sidecar; ++i)
+    if (sidecar_pos[i] < 0 || sidecar_pos[i] >= NK) return -1;
+  const int R = r1 - r0;
+  auto work = [&](int a, int b) {
+    std::vector<double> w((size_t)K);
+    for (int n = a; n < b; ++n) {
+      for (int k = 0; k < K; ++k) w[(size_t)k] = (double)decode_one(mode, codebook, indices, K, n, k);
+      auto it = std::lower_bound(order.begin(), order.end(), (int64_t)n * K,
+                                 [&](int64_t e, int64_t v) { return sidecar_pos[e] < v; });
+      for (; it != order.end() && sidecar_pos[*it] < (int64_t)(n + 1) * K; ++it)
+        w[(size_t)(sidecar_pos[*it] - (int64_t)n * K)] = (double)sidecar_val[*it];
+      for (int m = 0; m < M; ++m) {
+        double acc = 0.0;
+        for (int k = 0; k < K; ++k) acc += bf16_to_double(x_bits[(int64_t)m * K + k]) * w[(size_t)k];
+        y[(int64_t)m * R + (n - r0)] = acc;
+      }
+    }
+  };
+  const int T = std::min(threads, R);
+  std::vector<std::thread> pool;
+  for (int t = 1; t < T; ++t) pool.emplace_back(work, r0 + (int)((int64_t)R * t / T), r0 + (int)((int64_t)R * (t + 1) / T));
+  work(r0, r0 + R / T);
+  for (auto& th : pool) th.join();
+  return 0;
 }
 
 // ---- encoder side (HXQ whitepaper, method section: "Per-tensor k-means",

@@ -245,10 +245,11 @@ def test_full_size_prefill_sampled_rows(hxq, name, M):
 
 
 def _cluster_shapes(num_sms):
-    """Layer heights whose tile counts select each cluster size (2, 4, 8):
-    tiles x size between 85 % and 100 % of the SMs, last tile partial."""
+    """Layer heights whose tile counts select each cluster size (2, 4, 8, and
+    the non-portable 12 and 16 where the device allows them): tiles x size
+    between 85 % and 100 % of the SMs, last tile partial."""
     out = []
-    for cs in (2, 4, 8):
+    for cs in (2, 4, 8, 12, 16):
         tiles = num_sms // cs
         if 100 * tiles * cs >= 85 * num_sms:
             out.append((cs, tiles * 128 - 37))

@@ -13,11 +13,19 @@
 //   length, one per CTA of a persistent grid (one CTA per SM), so every CTA
 //   streams the same number of index bytes whatever the layer shape.
 //
-// Inside a CTA a producer warp streams the range in chunks of up to 4 stages
-// of one tile (32 KB of scalar indices, contiguous in the tiled layout) with
-// TMA bulk copies into a ring of shared-memory slots; it starts before the
-// previous kernel has finished, since the indices do not depend on it. The
-// 16 consumer warps share every chunk: warp q takes the q-th 16-weight piece
+// Two launches share an SM. A CTA keeps its shared memory to about half of
+// the SM's (a 32 KB codebook table, the activations, a ring of 16 KB slots)
+// and its registers to half of the register file, so that while one launch
+// drains, the next launch in the stream (programmatic dependent launch)
+// already has a CTA on every SM: it builds its table, asks the TMA engine to
+// bring its whole index range into L2 (bulk prefetch) and fills its ring,
+// and only its activation load waits for the previous launch to finish. HBM
+// therefore keeps streaming across launch boundaries.
+//
+// Inside a CTA a producer warp streams the range in chunks of up to 2 stages
+// of one tile (16 KB of scalar indices, contiguous in the tiled layout) with
+// TMA bulk copies into the ring; the bulk L2 prefetch runs ahead of it. The
+// 8 consumer warps share every chunk: warp q takes the q-th 16-weight piece
 // of the chunk (stage q / 4, quarter q % 4) for all 128 rows, lane l for rows
 // l, l + 32, l + 64, l + 96. So each activation a warp loads from shared
 // memory serves four rows: the decode is bound by the shared-memory pipe, and
@@ -35,7 +43,8 @@
 // Scalar codebook in shared memory: replicated once per lane with entry e of
 // lane l at byte e*256 + l*4, so the 32 lanes of a lookup always hit 32
 // different banks. The byte address is one PRMT away from the index word:
-// {0, 0, index byte, l*4}.
+// {0, 0, index byte, l*4}. The table uses the first half of each 256-byte
+// row; the other halves hold the activations and the reduction buffers.
 //
 // 2D codebook: the 4096 fp32 pairs (32 KB) are kept once; random pair
 // lookups can conflict on banks (a per-lane replica would need 1 MB).
@@ -47,7 +56,7 @@
 // "Sidecar outlier correction"): replacing w = c by v adds (v - c) x to the
 // dot product, so each entry carries delta = v - c (fp32, computed once when
 // the handle is built). The main loop decodes with the codebook alone. When a
-// segment starts, the four threads that finish row n load up to four each of
+// segment starts, the two threads that finish row n load up to four each of
 // the row's entries in the segment's columns (found through a per-stage
 // lower-bound table, the bounds fetched one segment ahead); at the segment
 // end they add delta * x[m][k] to the row's sum.
@@ -61,42 +70,84 @@
 namespace hxq {
 namespace {
 
-constexpr int kGemvThreads = 512;                  // consumers; then a producer and a fixup warp
-constexpr int kConsumerWarps = kGemvThreads / 32;  // 16: one 16-weight piece of a chunk each
+constexpr int kGemvThreads = 256;                  // consumers; then a producer and a fixup warp
+constexpr int kConsumerWarps = kGemvThreads / 32;  // 8: one 16-weight piece of a chunk each
 constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kFixupWarp = kConsumerWarps + 1;
 constexpr int kGemvBlock = kGemvThreads + 64;
 constexpr int kBarConsumers = 1;                   // named barrier of the consumers
-constexpr int kChunkStages = 4;                    // stages per ring slot (16 pieces per row)
-constexpr int kMaxRing = 6;                        // ring slots
+constexpr int kChunkStages = 2;                    // stages per ring slot (8 pieces per row)
+constexpr int kMaxRing = 8;                        // ring slots
 constexpr int kGemvMaxM = 8;                       // tokens
-constexpr int kSideGroups = kGemvThreads / kTileRows;  // 4 threads per row share its patch entries
+constexpr int kSideGroups = kGemvThreads / kTileRows;  // 2 threads per row share its patch entries
 constexpr int kPE = 4;                             // patch entries per thread and segment in registers
 constexpr size_t kSmemLimit = 226 * 1024;          // dynamic shared memory per CTA (static kept apart)
+// At most this much dynamic shared memory per CTA lets two CTAs share an SM:
+// 2 x (dynamic + static (under 512 bytes) + 1 KB reserved) <= 228 KB.
+constexpr size_t kSmemShared = 113 * 1024 - 512;
+constexpr uint32_t kPrefetchAhead = 256 * 1024;    // bulk L2 prefetch distance ahead of the ring
+constexpr int kScalarTable = 256 * 256;            // bytes: 256 rows of 32 lanes x fp32, then a 128-byte hole
+constexpr uint32_t kHoleBytes = 256 * 128;         // the rows' second halves, used as scratch
+constexpr int kPairTable = 4096 * 8;               // bytes: 4096 fp32 pairs
 
-// Dynamic shared memory of one CTA: codebook table, activations (fp32 or
-// bf16), the warps' partial sums and the split-tile sum handed to the fixup
-// warp, then the index ring.
+// Scratch of one CTA (bytes): activations (fp32 or bf16), the warps'
+// partial sums, the split-tile sums handed to the fixup warp, the sidecar
+// corrections and, for a cluster, the cluster's sums of its tile.
+inline size_t gemv_scratch(int MT, int Kp, bool xf32, int cs) {
+  return (size_t)MT * Kp * (xf32 ? 4 : 2) + (size_t)(kConsumerWarps + 2 + kSideGroups + cs) * MT * kTileRows * sizeof(float);
+}
+// Dynamic shared memory before the index ring: the codebook table and the
+// scratch (in scalar mode partly inside the table's holes).
 inline size_t gemv_smem_fixed(int mode, int MT, int Kp, bool xf32, int cs = 0) {
-  return (size_t)(mode == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8) + (size_t)MT * Kp * (xf32 ? 4 : 2) +
-         (size_t)(kConsumerWarps + 2 + kSideGroups + cs) * MT * kTileRows * sizeof(float);
+  const size_t sc = gemv_scratch(MT, Kp, xf32, cs);
+  if (mode == HXQ_MODE_SCALAR8) return (size_t)kScalarTable + (sc > kHoleBytes ? sc - kHoleBytes : 0);
+  return (size_t)kPairTable + sc;
 }
 inline int slot_bytes(int mode) { return kChunkStages * (mode == HXQ_MODE_SCALAR8 ? 4 : 3) * kTileRows * 16; }
-// Ring slots that fit next to the fixed part (0 if none fits; a single slot
-// -- no overlap of copies and decoding -- only happens for 8 tokens).
-constexpr int kMinRing = 1;
+// Ring slots: as many as fit (up to kMaxRing) while two CTAs still share an
+// SM; failing that, as many as fit in one CTA per SM; 0 if not even
+// kMinRing fit.
+constexpr int kMinRing = 2;
+constexpr int kMaxCluster = 16;                    // CTAs sharing one tile's K in the cluster split
 inline int ring_slots(int mode, int MT, int Kp, bool xf32, int cs = 0) {
-  const size_t fixed = gemv_smem_fixed(mode, MT, Kp, xf32, cs);
-  if (fixed + 128 > kSmemLimit) return 0;
-  const int fit = std::min(kMaxRing, (int)((kSmemLimit - fixed - 128) / slot_bytes(mode)));
-  return fit >= kMinRing ? fit : 0;
+  const size_t fixed = gemv_smem_fixed(mode, MT, Kp, xf32, cs) + 128;
+  for (size_t cap : {kSmemShared, kSmemLimit}) {
+    if (fixed + (size_t)kMinRing * slot_bytes(mode) > cap) continue;
+    return std::min(kMaxRing, (int)((cap - fixed) / slot_bytes(mode)));
+  }
+  return 0;
 }
 inline size_t gemv_smem(int mode, int MT, int Kp, bool xf32, int cs = 0) {
   return gemv_smem_fixed(mode, MT, Kp, xf32, cs) + 128 + (size_t)ring_slots(mode, MT, Kp, xf32, cs) * slot_bytes(mode);
 }
+// Activations staged as fp32 (no conversion in the inner loop) unless only
+// bf16 staging lets two CTAs share an SM, or fp32 does not fit at all.
+inline bool stage_x_f32(int mode, int MT, int Kp) {
+  auto shared = [&](bool f32) {
+    return gemv_smem_fixed(mode, MT, Kp, f32) + 128 + (size_t)kMinRing * slot_bytes(mode) <= kSmemShared;
+  };
+  if (shared(true)) return true;
+  if (shared(false)) return false;
+  return ring_slots(mode, MT, Kp, true) >= kMinRing;
+}
 
 template <int MODE>
-constexpr int table_bytes() { return MODE == HXQ_MODE_SCALAR8 ? 256 * 256 : 4096 * 8; }
+constexpr int table_bytes() { return MODE == HXQ_MODE_SCALAR8 ? kScalarTable : kPairTable; }
+
+// The CTA's scratch in shared memory, addressed by a logical byte offset: in
+// scalar mode the first kHoleBytes lie in the table's holes (the second
+// half of each 256-byte row) and the rest follows the table; in 2D mode the
+// scratch follows the pair table.
+template <int MODE>
+struct Scratch {
+  uint8_t* smem;
+  __device__ __forceinline__ uint8_t* at(uint32_t o) const {
+    if (MODE == HXQ_MODE_SCALAR8)
+      return smem + (o < kHoleBytes ? ((o >> 7) << 8) + 128 + (o & 127) : kScalarTable + (o - kHoleBytes));
+    return smem + kPairTable + o;
+  }
+  __device__ __forceinline__ float& f(uint32_t o) const { return *reinterpret_cast<float*>(at(o)); }
+};
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -109,18 +160,20 @@ __device__ __forceinline__ int cta_of(int w, int W, int G) {
   return b;
 }
 
-// 16 activations x[m][k0 .. k0+16) from shared memory as fp32.
-template <bool XF32>
-__device__ __forceinline__ void x16(const uint8_t* xs, int Kp, int m, int k0, float (&f)[16]) {
+// 16 activations x[m][k0 .. k0+16) from shared memory as fp32 (the staged
+// activations start at scratch offset 0; k0 is a multiple of 16, so the 64
+// or 32 bytes never cross a hole).
+template <bool XF32, int MODE>
+__device__ __forceinline__ void x16(const Scratch<MODE>& sc, int Kp, int m, int k0, float (&f)[16]) {
   if (XF32) {
-    const float4* p = reinterpret_cast<const float4*>(xs + ((size_t)m * Kp + k0) * 4);
+    const float4* p = reinterpret_cast<const float4*>(sc.at((uint32_t)(m * Kp + k0) * 4));
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float4 v = p[i];
       f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
     }
   } else {
-    const uint4* p = reinterpret_cast<const uint4*>(xs + ((size_t)m * Kp + k0) * 2);
+    const uint4* p = reinterpret_cast<const uint4*>(sc.at((uint32_t)(m * Kp + k0) * 2));
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const uint4 v = p[i];
@@ -148,12 +201,14 @@ __device__ __forceinline__ float acc_sum(float a) { return a; }
 __device__ __forceinline__ void acc_zero(float2& a) { a = make_float2(0.f, 0.f); }
 __device__ __forceinline__ void acc_zero(float& a) { a = 0.f; }
 
-__device__ __forceinline__ float x_at(const uint8_t* xs, int Kp, int m, int k, bool xf32) {
-  return xf32 ? *reinterpret_cast<const float*>(xs + ((size_t)m * Kp + k) * 4)
-              : bf16lo(*reinterpret_cast<const uint16_t*>(xs + ((size_t)m * Kp + k) * 2));
+template <int MODE>
+__device__ __forceinline__ float x_at(const Scratch<MODE>& sc, int Kp, int m, int k, bool xf32) {
+  return xf32 ? *reinterpret_cast<const float*>(sc.at((uint32_t)(m * Kp + k) * 4))
+              : bf16lo(*reinterpret_cast<const uint16_t*>(sc.at((uint32_t)(m * Kp + k) * 2)));
 }
 
 // The 16 weights of one row's piece: scalar indices (one 16-byte piece).
+// lane4 = 4 * lane (scalar table addressing).
 template <int MODE>
 __device__ __forceinline__ void decode16(const uint8_t* smem, const uint8_t* piece, int rows, int quarter,
                                          uint32_t lane4, float (&wv)[16]) {
@@ -226,12 +281,13 @@ struct Segments {
 };
 
 // y rows of tile t from the sums of its contributors c_first..c_last, added
-// in CTA order: this CTA's own sum from `own` (shared memory), the others'
-// from the workspace (a batch of contributors' loads in flight per sum).
-template <int MT>
+// in CTA order: this CTA's own sum from the scratch at offset `own`, the
+// others' from the workspace (a batch of contributors' loads in flight per
+// sum).
+template <int MT, int MODE>
 __device__ __forceinline__ void finish_tile(const Layer& L, const Out& out, const float* __restrict__ work,
-                                            const float* own, int M, int t, int c_first, int c_last, int b, int W,
-                                            int G, int n_st, int tid, int nthreads) {
+                                            const Scratch<MODE>& sc, uint32_t own, int M, int t, int c_first,
+                                            int c_last, int b, int W, int G, int n_st, int tid, int nthreads) {
   const int rows = min(kTileRows, L.N - t * kTileRows);
   for (int i = tid; i < MT * kTileRows; i += nthreads) {
     const int m = i / kTileRows, r = i % kTileRows;
@@ -247,7 +303,7 @@ __device__ __forceinline__ void finish_tile(const Layer& L, const Out& out, cons
       }
 #pragma unroll
       for (int e = 0; e < 16; ++e)
-        if (c0 + e <= c_last) v += c0 + e == b ? own[i] : q[e];
+        if (c0 + e <= c_last) v += c0 + e == b ? sc.f(own + 4 * i) : q[e];
     }
     store_out(out, (size_t)m * L.N + t * kTileRows + r, t * kTileRows + r, v);
   }
@@ -264,14 +320,19 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
   constexpr int TB = table_bytes<MODE>();
   constexpr int NP = MODE == HXQ_MODE_SCALAR8 ? 4 : 3;  // 16-byte pieces per row and stage
   constexpr int TS = MT * kTileRows;                    // sums per tile
-  uint8_t* xs = smem + TB;
-  // per-warp partial sums [kConsumerWarps][MT][kTileRows], after the activations
-  float* red = reinterpret_cast<float*>(xs + (size_t)MT * L.Kp * (XF32 ? 4 : 2));
-  float* pbuf = red + kConsumerWarps * TS;  // [2][TS] this CTA's sums of its split tiles (by slot)
-  float* side = pbuf + 2 * TS;              // [kSideGroups][TS] sidecar corrections
-  float* cbuf = side + kSideGroups * TS;    // [cs][TS] the cluster's sums of its tile (rank 0's copy)
-  uint8_t* ring = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(cbuf + cs * TS) + 127) & ~(uintptr_t)127);
+  const Scratch<MODE> sc{smem};
+  // scratch offsets (bytes): activations at 0, then the per-warp partial
+  // sums [kConsumerWarps][MT][kTileRows], this CTA's sums of its split tiles
+  // [2][TS] (by slot), the sidecar corrections [kSideGroups][TS] and the
+  // cluster's sums of its tile [cs][TS] (rank 0's copy)
+  const uint32_t red = (uint32_t)MT * L.Kp * (XF32 ? 4 : 2);
+  const uint32_t pbuf = red + kConsumerWarps * TS * 4;
+  const uint32_t side = pbuf + 2 * TS * 4;
+  const uint32_t cbuf = side + kSideGroups * TS * 4;
+  const uint32_t sc_end = cbuf + cs * TS * 4;
+  const uint32_t fixed =
+      MODE == HXQ_MODE_SCALAR8 ? TB + (sc_end > kHoleBytes ? sc_end - kHoleBytes : 0) : TB + sc_end;
+  uint8_t* ring = smem + ((fixed + 127) & ~127u);
   constexpr int SLOT = kChunkStages * NP * kTileRows * 16;
   __shared__ uint64_t bar_full[kMaxRing], bar_empty[kMaxRing];
   __shared__ uint64_t bar_handoff[2];  // a split tile's sums (by slot) are in pbuf: consumers -> fixup warp
@@ -308,8 +369,25 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
   pdl_launch_dependents();  // the next kernel in the stream may start its prologue
 
   if (warp == kProducerWarp) {
-    // ---------------- producer: the segments' chunks, in processing order
+    // ---------------- producer: the segments' chunks, in processing order,
+    // with a bulk L2 prefetch of the range running kPrefetchAhead bytes
+    // ahead of the ring (the indices do not depend on the previous kernel)
     if (lane == 0) {
+      const size_t tile_bytes = (size_t)kTileRows * L.KC * 16 * L.P;
+      int pf_k = 0, pf_w = S.n > 0 ? S.begin(0) : 0;  // prefetch cursor: segment, stage
+      size_t pf_bytes = 0, ring_bytes = 0;
+      auto prefetch_to = [&](size_t limit) {
+        while (pf_k < S.n && pf_bytes < limit) {
+          const int t = S.tile(pf_k), seg1 = S.end(pf_k);
+          const int rows = min(kTileRows, L.N - t * kTileRows);
+          const int we = min(pf_w + 4, seg1);
+          const uint32_t bytes = (uint32_t)((we - pf_w) * NP * rows * 16);
+          prefetch_l2_bulk(L.idx + (size_t)t * tile_bytes + (size_t)(pf_w - t * n_st) * NP * rows * 16, bytes);
+          pf_bytes += bytes;
+          pf_w = we;
+          if (pf_w >= seg1 && ++pf_k < S.n) pf_w = S.begin(pf_k);
+        }
+      };
       int issued = 0, s = 0;
       uint32_t ph = 0;
       for (int k = 0; k < S.n && !*abrt; ++k) {
@@ -321,10 +399,11 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
           if (!mbar_wait(&bar_empty[s], ph ^ 1, abrt)) break;
           const uint32_t bytes = (uint32_t)((we - w) * NP * rows * 16);
           mbar_arrive_expect_tx(&bar_full[s], bytes);
-          bulk_load(ring + (size_t)s * SLOT,
-                    L.idx + (size_t)t * kTileRows * L.KC * 16 * L.P + (size_t)st * NP * rows * 16, bytes,
+          bulk_load(ring + (size_t)s * SLOT, L.idx + (size_t)t * tile_bytes + (size_t)st * NP * rows * 16, bytes,
                     &bar_full[s]);
           ++issued;
+          ring_bytes += bytes;
+          prefetch_to(ring_bytes + kPrefetchAhead);
           if (++s == R) s = 0, ph ^= 1;
           w = we;
         }
@@ -357,14 +436,14 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
       mbar_wait(&bar_handoff[slot], 0, &never, 64);
       const int c_first = cta_of(t * n_st, W, G), c_last = cta_of((t + 1) * n_st - 1, W, G);
       float* part = work + (size_t)(b * 2 + slot) * TS;
-      for (int i = lane; i < TS; i += 32) part[i] = pbuf[slot * TS + i];
+      for (int i = lane; i < TS; i += 32) part[i] = sc.f(pbuf + 4 * (slot * TS + i));
       __threadfence();
       __syncwarp();
       int prev = lane == 0 ? atomicAdd(counters + t, 1) : 0;
       prev = __shfl_sync(0xffffffffu, prev, 0);
       if (prev == c_last - c_first) {
         __threadfence();  // the other contributors' sums are visible past their count
-        finish_tile<MT>(L, out, work, pbuf + slot * TS, M, t, c_first, c_last, b, W, G, n_st, lane, 32);
+        finish_tile<MT>(L, out, work, sc, pbuf + 4 * slot * TS, M, t, c_first, c_last, b, W, G, n_st, lane, 32);
         if (lane == 0) counters[t] = 0;
       }
     }
@@ -397,6 +476,7 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
   // shared-memory codebook (compile-time trip counts: a thread's codebook
   // loads are all in flight together)
   if (MODE == HXQ_MODE_SCALAR8) {
+    // lane (i % 32)'s copy of entry i / 32 at word (i / 32) * 64 + i % 32
     constexpr int PER = 256 * 32 / kGemvThreads;
     float cv[PER];
 #pragma unroll
@@ -436,11 +516,11 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
         if (i >= n8) break;
         const int m = i / (L.Kp / 8), k = (i % (L.Kp / 8)) * 8;
         if (XF32) {
-          float4* d = reinterpret_cast<float4*>(xs + ((size_t)m * L.Kp + k) * 4);
+          float4* d = reinterpret_cast<float4*>(sc.at((uint32_t)(m * L.Kp + k) * 4));
           d[0] = make_float4(bf16lo(q[u].x), bf16hi(q[u].x), bf16lo(q[u].y), bf16hi(q[u].y));
           d[1] = make_float4(bf16lo(q[u].z), bf16hi(q[u].z), bf16lo(q[u].w), bf16hi(q[u].w));
         } else {
-          *reinterpret_cast<uint4*>(xs + ((size_t)m * L.Kp + k) * 2) = q[u];
+          *reinterpret_cast<uint4*>(sc.at((uint32_t)(m * L.Kp + k) * 2)) = q[u];
         }
       }
     }
@@ -496,7 +576,7 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
         // their sums are never stored.
         if (MT == 1) {
           float xv[16];
-          x16<XF32>(xs, L.Kp, 0, k0, xv);
+          x16<XF32>(sc, L.Kp, 0, k0, xv);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float wv[16];
@@ -516,7 +596,7 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
             for (int m = 0; m < MT; ++m) {
               if (MT >= 4) asm volatile("" ::: "memory");  // one token's activations live at a time
               float xv[16];
-              x16<XF32>(xs, L.Kp, m, k0, xv);
+              x16<XF32>(sc, L.Kp, m, k0, xv);
               fma16(acc[2 * jp][m], wv0, xv);
               fma16(acc[2 * jp + 1][m], wv1, xv);
             }
@@ -541,7 +621,7 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
       for (int j = 0; j < kPE; ++j)
         if (j < n_mine) {
 #pragma unroll
-          for (int m = 0; m < MT; ++m) sp[m] = fmaf(ed[j], x_at(xs, L.Kp, m, ek[j], XF32), sp[m]);
+          for (int m = 0; m < MT; ++m) sp[m] = fmaf(ed[j], x_at(sc, L.Kp, m, ek[j], XF32), sp[m]);
         }
       if (sg == kSideGroups - 1) {
 #pragma unroll 1
@@ -549,16 +629,16 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
           const int kk = __ldg(L.pk + p);
           const float d = __ldg(L.pd + p);
 #pragma unroll
-          for (int m = 0; m < MT; ++m) sp[m] = fmaf(d, x_at(xs, L.Kp, m, kk, XF32), sp[m]);
+          for (int m = 0; m < MT; ++m) sp[m] = fmaf(d, x_at(sc, L.Kp, m, kk, XF32), sp[m]);
         }
       }
 #pragma unroll
-      for (int m = 0; m < MT; ++m) side[(sg * MT + m) * kTileRows + rr] = sp[m];
+      for (int m = 0; m < MT; ++m) sc.f(side + 4 * ((sg * MT + m) * kTileRows + rr)) = sp[m];
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int m = 0; m < MT; ++m) red[(q * MT + m) * kTileRows + lane + 32 * j] = acc_sum(acc[j][m]);
+      for (int m = 0; m < MT; ++m) sc.f(red + 4 * ((q * MT + m) * kTileRows + lane + 32 * j)) = acc_sum(acc[j][m]);
     consumer_sync();
     const int slot = S.slot(k);
     if (cs > 0) cluster_wait();  // every CTA of the cluster has started: rank 0's memory may be written
@@ -566,15 +646,15 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
       const int m = i / kTileRows;
       float v = 0.f;
 #pragma unroll
-      for (int qq = 0; qq < kConsumerWarps; ++qq) v += red[(qq * MT + m) * kTileRows + rr];
+      for (int qq = 0; qq < kConsumerWarps; ++qq) v += sc.f(red + 4 * ((qq * MT + m) * kTileRows + rr));
 #pragma unroll
-      for (int g = 0; g < kSideGroups; ++g) v += side[(g * MT + m) * kTileRows + rr];
+      for (int g = 0; g < kSideGroups; ++g) v += sc.f(side + 4 * ((g * MT + m) * kTileRows + rr));
       if (!split) {
         if (m < M && rr < rows) store_out(out, (size_t)m * L.N + t * kTileRows + rr, t * kTileRows + rr, v);
       } else if (cs > 0) {
-        st_cluster_f32(map_to_rank(smem_u32(cbuf + (b % cs) * TS + i), 0), v);
+        st_cluster_f32(map_to_rank(smem_u32(sc.at(cbuf + 4 * ((b % cs) * TS + i))), 0), v);
       } else {
-        pbuf[slot * TS + i] = v;
+        sc.f(pbuf + 4 * (slot * TS + i)) = v;
       }
     }
     if (cs > 0) {
@@ -587,7 +667,7 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
         for (int i = threadIdx.x; i < TS; i += kGemvThreads) {
           const int m = i / kTileRows;
           float v = 0.f;
-          for (int r = 0; r < cs; ++r) v += cbuf[r * TS + i];
+          for (int r = 0; r < cs; ++r) v += sc.f(cbuf + 4 * (r * TS + i));
           if (m < M && rr < rows) store_out(out, (size_t)m * L.N + t * kTileRows + rr, t * kTileRows + rr, v);
         }
       }
@@ -606,10 +686,10 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
       if (threadIdx.x == 0) flag_sh = ld_acquire_gpu(counters + t) == others;
       consumer_sync();
       bool last = flag_sh;
-      const float* own = pbuf + slot * TS;
+      const uint32_t own = pbuf + 4 * slot * TS;
       if (!last) {
         float* part = work + (size_t)(b * 2 + slot) * TS;
-        for (int i = threadIdx.x; i < TS; i += kGemvThreads) part[i] = own[i];
+        for (int i = threadIdx.x; i < TS; i += kGemvThreads) part[i] = sc.f(own + 4 * i);
         __threadfence();
         consumer_sync();
         if (threadIdx.x == 0) flag_sh = atomicAdd(counters + t, 1) == others;
@@ -618,7 +698,7 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
       }
       if (last) {
         __threadfence();  // the other contributors' sums are visible past their count
-        finish_tile<MT>(L, out, work, own, M, t, c_first, c_last, b, W, G, n_st, threadIdx.x, kGemvThreads);
+        finish_tile<MT>(L, out, work, sc, own, M, t, c_first, c_last, b, W, G, n_st, threadIdx.x, kGemvThreads);
         if (threadIdx.x == 0) counters[t] = 0;
       }
     }
@@ -629,7 +709,7 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
 }
 
 template <int MT, bool XF32, int MODE>
-__global__ void __launch_bounds__(kGemvBlock, 1)
+__global__ void __launch_bounds__(kGemvBlock, 2)
 gemv_kernel(Layer L, const uint16_t* __restrict__ x, Out out, int M, int W, int R, int cs,
             float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
   gemv_body<MT, XF32, MODE>(L, x, out, M, W, R, cs, work, counters, status, (int)blockIdx.x, (int)gridDim.x);
@@ -652,7 +732,7 @@ struct GemvGroup {
 };
 
 template <int MT, bool XF32, int MODE>
-__global__ void __launch_bounds__(kGemvBlock, 1)
+__global__ void __launch_bounds__(kGemvBlock, 2)
 gemv_group_kernel(const __grid_constant__ GemvGroup g, const uint16_t* __restrict__ x, int M, int R, int cs) {
   int li = 0;
 #pragma unroll
@@ -662,23 +742,35 @@ gemv_group_kernel(const __grid_constant__ GemvGroup g, const uint16_t* __restric
                             (int)blockIdx.x - g.first[li], g.first[li + 1] - g.first[li]);
 }
 
+// Sets the kernel's dynamic shared memory size and asks for the largest
+// shared-memory carveout, so that two CTAs of up to kSmemShared bytes each
+// (this launch's and the next one's) can be resident on one SM.
+template <typename Kern>
+cudaError_t set_smem(Kern kern, size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
 // Cluster split (no global-memory reduction): each tile gets a cluster of
-// cs CTAs (2..8) that split its K, for the largest cs whose grid (tiles x cs)
-// fills at least 70 % of the SMs without exceeding them and whose clusters
-// all fit on the GPU at once. 0 = the stream-K decomposition. `cached` keeps
-// the answer for the next launch of the same shape.
+// cs CTAs (2..16; above 8 where the device allows such clusters) that split
+// its K, for the largest cs whose grid (tiles x cs) fills at least 70 % of
+// the SMs without exceeding them and whose clusters all fit on the GPU at
+// once. 0 = the stream-K decomposition. `cached` keeps the answer for the
+// next launch of the same shape.
 template <int MT, bool XF32, int MODE, typename Kern>
 int pick_cluster_for(Kern kern, int n_tiles, int Kp, int num_sms, int& cached) {
   if (cached >= 0) return cached;
   cached = 0;
   if (MT > 4) return 0;
   const int n_st = Kp / kStageK;
-  for (int cs = 8; cs >= 2; --cs) {
+  for (int cs = kMaxCluster; cs >= 2; --cs) {
     const int g = n_tiles * cs;
     if (g > num_sms || 100 * g < 70 * num_sms || n_st < cs) continue;
     if (ring_slots(MODE, MT, Kp, XF32, cs) < kMinRing) continue;
     const size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+    if (set_smem(kern, smem) != cudaSuccess ||
+        (cs > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
       cudaGetLastError();
       continue;
     }
@@ -723,7 +815,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
   if (cs > 0) {
     const int Rc = ring_slots(MODE, MT, h.L.Kp, XF32, cs);
     const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32, cs);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl_cluster(kern, h.L.n_tiles * cs, kGemvBlock, smem, cs, s, h.L, x, out, M, W, Rc, cs, work, counters,
                               h.d_status);
@@ -731,7 +823,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
   const int R = ring_slots(MODE, MT, h.L.Kp, XF32);
   if (R < kMinRing) return cudaErrorInvalidValue;
   const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, grid, kGemvBlock, smem, s, h.L, x, out, M, W, R, 0, work, counters, h.d_status);
 }
@@ -739,7 +831,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
 template <int MT, int MODE>
 cudaError_t launch_mt(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, float* work, int* counters,
                       bool allow_cluster, cudaStream_t s) {
-  if (ring_slots(MODE, MT, h.L.Kp, true) >= kMinRing)
+  if (stage_x_f32(MODE, MT, h.L.Kp))
     return launch_cfg<MT, true, MODE>(h, x, out, M, grid, work, counters, allow_cluster, s);
   return launch_cfg<MT, false, MODE>(h, x, out, M, grid, work, counters, allow_cluster, s);
 }
@@ -797,7 +889,7 @@ cudaError_t launch_group_cfg(const hxq_group& g, const uint16_t* x, const Out* o
   const int R = ring_slots(MODE, MT, Kp, XF32, cs);
   if (R < kMinRing) return cudaErrorInvalidValue;
   const size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   if (cs > 0) return launch_pdl_cluster(kern, grid, kGemvBlock, smem, cs, s, p, x, M, R, cs);
   return launch_pdl(kern, grid, kGemvBlock, smem, s, p, x, M, R, 0);
@@ -805,7 +897,7 @@ cudaError_t launch_group_cfg(const hxq_group& g, const uint16_t* x, const Out* o
 
 template <int MT, int MODE>
 cudaError_t launch_group_mt(const hxq_group& g, const uint16_t* x, const Out* outs, int M, cudaStream_t s) {
-  if (ring_slots(MODE, MT, g.h[0]->L.Kp, true) >= kMinRing) return launch_group_cfg<MT, true, MODE>(g, x, outs, M, s);
+  if (stage_x_f32(MODE, MT, g.h[0]->L.Kp)) return launch_group_cfg<MT, true, MODE>(g, x, outs, M, s);
   return launch_group_cfg<MT, false, MODE>(g, x, outs, M, s);
 }
 

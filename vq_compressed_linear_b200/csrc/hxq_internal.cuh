@@ -141,7 +141,8 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, si
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
-// As launch_pdl, with the grid in clusters of `cluster` CTAs (1 = none).
+// As launch_pdl, with the grid in clusters of `cluster` CTAs (1 = none),
+// each cluster's CTAs spread over distinct SMs.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, unsigned cluster,
                                cudaStream_t s, Args... args) {
@@ -150,15 +151,17 @@ cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), unsigned grid, unsigned b
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
   attr[1].val.clusterDim.x = cluster;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
+  attr[2].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+  attr[2].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicySpread;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 3;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
