@@ -300,14 +300,6 @@ def e2e_workload(hxq, torch, items, steps, warmup, stream, groups=()):
 
 # ----------------------------------------------------------------------------- CPU oracle arm
 
-def _oracle_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        return os.cpu_count() or 1
-
-
 _X_CACHE = {}
 
 
@@ -318,73 +310,112 @@ def _x_for(layer, M):
     return _X_CACHE[key]
 
 
-def _oracle_pass(items, frac, offset=0):
-    """One pass of the fp64 oracle over the workload, on `frac` of each
-    layer's output rows (a contiguous, rotating slice). Returns (bytes, flops)
-    credited, scaled by the fraction of rows done."""
-    import oracle
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _timing_oracle():
+    """The plain C++ oracle compiled for this host (-O3 -march=native, no
+    fused multiply-add), in a temporary directory."""
+    import tempfile
+    from oracle import hxq_oracle_cpp
+    return hxq_oracle_cpp, hxq_oracle_cpp.load_timing_build(tempfile.mkdtemp(prefix="hxq_oracle_"))
+
+
+def _oracle_pass(cpp, lib, items, frac, threads, offset=0):
+    """One pass of the C++ oracle (decode with the sidecar, float64 dot
+    products) over `frac` of each layer's output rows (a contiguous slice
+    that rotates with `offset`). Returns the (bytes, flops) credited, scaled
+    by the fraction of rows done."""
     b = f = 0.0
     for _, layer, M in items:
-        x = _x_for(layer, M)
         N = layer["N"]
-        nr = max(1, int(round(frac * N)))
-        if nr >= N:
-            oracle.forward_layer(layer, x)
-            nr = N
-        else:
-            rows = (offset * nr + np.arange(nr)) % N
-            oracle.forward_rows(layer, x, rows)
-        b += layer_bytes(layer, M) * nr / N
-        f += layer_flops(layer, M) * nr / N
+        nr = max(1, min(N, int(round(frac * N))))
+        r0 = (offset * nr) % N if nr < N else 0
+        r1 = min(N, r0 + nr)
+        cpp.forward_rows(layer, _x_for(layer, M), r0, r1, threads, lib)
+        b += layer_bytes(layer, M) * (r1 - r0) / N
+        f += layer_flops(layer, M) * (r1 - r0) / N
     return b, f
 
 
-def oracle_sample(items, budget_s=12.0):
-    """cpu_baseline: repeat oracle passes over the workload until about
-    budget_s of CPU time is spent (a row slice per pass when a whole pass would
-    take longer). Returns (GB/s, TFLOP/s, description, threads, seconds)."""
+def oracle_rate(items, threads, budget_s, cpp=None, lib=None):
+    """The C++ oracle's rate on `threads` host threads: repeated passes over
+    the workload (a row slice per pass, sized so that one pass takes about
+    budget_s / 20) until budget_s of wall time. Returns (GB/s, TFLOP/s,
+    passes, fraction of rows per pass, seconds)."""
+    if lib is None:
+        cpp, lib = _timing_oracle()
     for _, layer, M in items:
         _x_for(layer, M)
+    frac = 1.0
     t0 = time.perf_counter()
-    b, f = _oracle_pass(items, 1.0 if _est_pass_s(items) < budget_s / 4 else 0.05)
-    first = time.perf_counter() - t0
-    frac = 1.0 if first < budget_s / 4 and _est_pass_s(items) < budget_s / 4 else 0.05
-    passes, tb, tf, tt = 1, b, f, first
+    _oracle_pass(cpp, lib, items, 0.01, threads)  # size the slice on 1 % of the rows
+    one = max(1e-6, (time.perf_counter() - t0) / 0.01)
+    frac = min(1.0, budget_s / 20 / one)
+    passes, tb, tf, tt = 0, 0.0, 0.0, 0.0
     while tt < budget_s:
         t1 = time.perf_counter()
-        b, f = _oracle_pass(items, frac, passes)
+        b, f = _oracle_pass(cpp, lib, items, frac, threads, passes)
         tt += time.perf_counter() - t1
-        tb += b
-        tf += f
-        passes += 1
-    desc = f"{passes} oracle passes over " + ", ".join(lbl for lbl, _, _ in items) + \
-        ("" if frac == 1.0 else f" ({frac:.0%} of output rows per pass after the first)")
-    return tb / tt / 1e9, tf / tt / 1e12, desc, _oracle_threads(), tt
+        tb, tf, passes = tb + b, tf + f, passes + 1
+    return tb / tt / 1e9, tf / tt / 1e12, passes, frac, tt
 
 
-def _est_pass_s(items):
-    # fp64 oracle: decode ~ 20 ns per weight, product ~ 1 ns per multiply-add
-    return sum(20e-9 * l["N"] * l["K"] + 1e-9 * M * l["N"] * l["K"] for _, l, M in items)
+def oracle_sample(items, budget_s=6.0):
+    """cpu_baseline: the plain C++ oracle timed on one host thread and on
+    all host threads, each for about budget_s."""
+    cpp, lib = _timing_oracle()
+    n_all = os.cpu_count() or 1
+    r1 = oracle_rate(items, 1, budget_s, cpp, lib)
+    ra = oracle_rate(items, n_all, budget_s, cpp, lib)
+    names = ", ".join(lbl for lbl, _, _ in items)
+    desc = (f"plain C++ oracle (decode with sidecar + fp64 dot, -O3 -march=native) over {names}: "
+            f"1 thread {r1[2]} passes of {r1[3]:.1%} of the rows ({r1[4]:.1f} s); "
+            f"{n_all} threads {ra[2]} passes of {ra[3]:.1%} of the rows ({ra[4]:.1f} s)")
+    return r1, ra, n_all, desc
 
 
 def oracle_reference_arm(items, steps, warmup, budget_s=60.0):
-    """--impl reference: W warm-up passes, then K timed passes, each on a row
-    slice sized so that the K passes take about budget_s in total."""
-    frac = min(1.0, budget_s / max(1, steps) / max(1e-6, _est_pass_s(items)))
+    """--impl reference: the plain C++ oracle on all host threads; W warm-up
+    passes, then K timed passes, each on a row slice sized so that the K
+    passes take about budget_s in total."""
+    cpp, lib = _timing_oracle()
+    n_all = os.cpu_count() or 1
     for _, layer, M in items:
         _x_for(layer, M)
+    t0 = time.perf_counter()
+    _oracle_pass(cpp, lib, items, 0.01, n_all)
+    one = max(1e-6, (time.perf_counter() - t0) / 0.01)
+    frac = min(1.0, budget_s / max(1, steps) / one)
     for i in range(warmup):
-        _oracle_pass(items, frac, i)
+        _oracle_pass(cpp, lib, items, frac, n_all, i)
     t0 = time.perf_counter()
     tb = tf = 0.0
     for i in range(steps):
-        b, f = _oracle_pass(items, frac, warmup + i)
+        b, f = _oracle_pass(cpp, lib, items, frac, n_all, warmup + i)
         tb += b
         tf += f
     tt = time.perf_counter() - t0
-    desc = f"{steps} oracle passes over " + ", ".join(lbl for lbl, _, _ in items) + \
-        f", {min(frac, 1.0):.2%} of output rows per pass"
-    return tb / tt / 1e9, tf / tt / 1e12, desc, _oracle_threads(), tt
+    desc = (f"plain C++ oracle (-O3 -march=native), {steps} passes over " + ", ".join(lbl for lbl, _, _ in items) +
+            f", {frac:.2%} of output rows per pass, {n_all} threads, {cpu_model()}")
+    return tb / tt / 1e9, tf / tt / 1e12, desc, n_all, tt
+
+
+def _oracle_threads():
+    """Threads the numpy oracle's BLAS uses (encoder reference arm)."""
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
 
 
 def profile_run(hxq, torch, items, steps, warmup):
@@ -586,7 +617,7 @@ def main():
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": wl_name},
                 "cpu_baseline": {"value": v, "unit": unit, "cores": threads, "kind": "oracle",
-                                 "sample": sample + f" ({secs:.1f} s)"},
+                                 "sample": sample + f" ({secs:.1f} s)", "cpu_model": cpu_model()},
                 "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return 0
@@ -685,9 +716,11 @@ def main():
         line["secondary"] = sec
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs_c, tfs_c, sample, threads, secs = oracle_sample(items)
-        line["cpu_baseline"] = {"value": tfs_c if is_prefill else gbs_c, "unit": unit, "cores": threads,
-                                "kind": "oracle", "sample": sample + f" ({secs:.1f} s)"}
+        r1, ra, n_all, sample = oracle_sample(items)
+        pick = (lambda r: r[1]) if is_prefill else (lambda r: r[0])
+        line["cpu_baseline"] = {"value": pick(ra), "unit": unit, "cores": n_all, "kind": "oracle",
+                                "sample": sample, "cores_1": pick(r1), "cores_all": pick(ra),
+                                "cpu_model": cpu_model()}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -24,7 +24,7 @@ def build() -> str:
     if not cxx:
         raise RuntimeError("no host C++ compiler")
     tmp = LIB + ".tmp"
-    subprocess.run([cxx, "-O2", "-std=c++17", "-ffp-contract=off", "-fPIC", "-shared", SRC, "-o", tmp],
+    subprocess.run([cxx, "-O2", "-std=c++17", "-ffp-contract=off", "-fPIC", "-shared", "-pthread", SRC, "-o", tmp],
                    check=True)
     os.replace(tmp, LIB)
     return LIB
@@ -47,8 +47,31 @@ def _load():
         lib.oracle_kmeans_update.restype = None
         lib.oracle_sidecar_select.argtypes = [vp, vp, i64, ctypes.c_float, vp, vp, i64]
         lib.oracle_sidecar_select.restype = i64
+        _declare_rows(lib)
         _lib = lib
     return _lib
+
+
+def _declare_rows(lib):
+    vp, i, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    lib.oracle_forward_rows.argtypes = [i, vp, vp, vp, vp, i64, i, i, vp, i, i, i, i, vp]
+    lib.oracle_forward_rows.restype = i
+
+
+def load_timing_build(out_dir):
+    """The same oracle compiled for timing on this host (-O3 -march=native,
+    still without fused multiply-add) into out_dir; returns the loaded
+    library. Used by bench.py's CPU baseline leg only."""
+    cxx = os.environ.get("CXX") or shutil.which("g++") or shutil.which("c++")
+    if not cxx:
+        raise RuntimeError("no host C++ compiler")
+    os.makedirs(out_dir, exist_ok=True)
+    path = os.path.join(out_dir, "libhxq_oracle_timing.so")
+    subprocess.run([cxx, "-O3", "-march=native", "-std=c++17", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
+                    SRC, "-o", path], check=True)
+    lib = ctypes.CDLL(path)
+    _declare_rows(lib)
+    return lib
 
 
 def _p(a):
@@ -111,3 +134,22 @@ def sidecar_select(W, W_hat, threshold):
     val = np.empty(w.size, np.float32)
     n = _load().oracle_sidecar_select(_p(w), _p(wh), int(w.size), float(threshold), _p(pos), _p(val), int(w.size))
     return pos[:n].copy(), val[:n].copy()
+
+
+def forward_rows(layer, x_bits, r0, r1, threads=1, lib=None):
+    """y[:, r0:r1] of the layer's forward (decode with the sidecar, then the
+    float64 dot products), computed by oracle_forward_rows on `threads`
+    host threads."""
+    L = lib or _load()
+    x = np.ascontiguousarray(np.atleast_2d(x_bits), dtype=np.uint16)
+    cb = np.ascontiguousarray(layer["codebook"], dtype=np.float32)
+    idx = np.ascontiguousarray(layer["indices"], dtype=np.uint8)
+    pos = np.ascontiguousarray(layer["sidecar_pos"], dtype=np.int64).reshape(-1)
+    val = np.ascontiguousarray(layer["sidecar_val"], dtype=np.float32).reshape(-1)
+    M = x.shape[0]
+    y = np.empty((M, r1 - r0), np.float64)
+    rc = L.oracle_forward_rows(int(layer["mode"]), _p(cb), _p(idx), _p(pos), _p(val), int(pos.size), int(layer["N"]),
+                               int(layer["K"]), _p(x), int(M), int(r0), int(r1), int(threads), _p(y))
+    if rc != 0:
+        raise ValueError("invalid layer or rows")
+    return y

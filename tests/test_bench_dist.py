@@ -135,3 +135,15 @@ def test_run_env_never_raises():
     import bench
     env = bench.run_env(torch, 0)
     assert ("gpu" in env and "torch" in env) or "error" in env
+
+
+def test_cpu_baseline_times_cpp_oracle_on_one_and_all_threads():
+    """The CPU baseline times the plain C++ oracle (compiled for the host) on
+    one thread and on every host thread, on the bench's own workload."""
+    sys.path.insert(0, ROOT)
+    import bench
+    items = bench.workload("tiny", 0, 1)
+    r1, ra, n_all, desc = bench.oracle_sample(items, budget_s=0.3)
+    assert n_all == (os.cpu_count() or 1)
+    assert r1[0] > 0 and ra[0] > 0 and r1[2] >= 1 and ra[2] >= 1
+    assert "C++ oracle" in desc and bench.cpu_model()

@@ -114,3 +114,20 @@ def test_cpp_encoder_hand_worked_cases():
         arr = lambda t: np.array([float(v) for v in t], np.float32).reshape(-1, dim)
         c, lab = cpp.kmeans(arr(f[2]), arr(f[3]), int(f[4][0]))
         assert np.array_equal(c, arr(f[5])) and np.array_equal(lab, [int(v) for v in f[6]]), f[0]
+
+
+@pytest.mark.parametrize("mode,N,K,ns", [(0, 130, 72, 40), (1, 129, 136, 60), (0, 300, 64, 300)])
+@pytest.mark.parametrize("threads", [1, 3])
+def test_cpp_forward_rows_equals_forward(mode, N, K, ns, threads):
+    """The row-range forward used to time the oracle on the host cores takes
+    the same steps as decode + forward (the same k-order float64 sums), so
+    any row range, on any number of threads, matches them exactly."""
+    layer = synthetic.make_layer(mode, N, K, 70 + N, sidecar_count=ns)
+    x = synthetic.activations(2, K, 71)
+    W = cpp.decode(mode, layer["codebook"], layer["indices"], layer["sidecar_pos"], layer["sidecar_val"], N, K)
+    y, _ = cpp.forward(x, W)
+    for r0, r1 in [(0, N), (1, N - 1), (N // 2, N // 2 + 1)]:
+        got = cpp.forward_rows(layer, x, r0, r1, threads)
+        assert np.array_equal(got, y[:, r0:r1])
+    with pytest.raises(ValueError):
+        cpp.forward_rows(layer, x, 3, 2)
