@@ -64,7 +64,7 @@ constexpr int kEpiWarp0 = 4;                            // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;                            // warps 8..: decoders
 constexpr int kTmemCols = 512;
 constexpr int kMaxTokBlocks = 64;                       // token blocks per launch (counter space)
-constexpr int kMaxContrib = 4;                          // CTAs sharing one tile's K at most
+constexpr int kMaxContrib = 16;                         // CTAs sharing one tile's K at most
 constexpr int kPrefetchItems = 16;                      // index bytes streamed into L2 this far ahead
 
 // Decoding warps: 4 groups of 4 (one warp per TMEM lane quadrant). Every
@@ -292,7 +292,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
         const int T = w / n_st, st = w - T * n_st;
         const int tb = T / L.n_tiles;
         if (i + kIS + kPrefetchItems < n_items) prefetch_item(i + kIS + kPrefetchItems);
-        if (!mbar_wait(&bar_empty[b], ph ^ 1, abrt)) break;
+        // (the producers run slots ahead: they poll with short sleeps, so that
+        // their warps leave issue slots to the decoders)
+        if (!mbar_wait(&bar_empty[b], ph ^ 1, abrt, 64)) break;
         mbar_arrive_expect_tx(&bar_x[b], XSLOT);
         tma_load_2d(xs + b * XSLOT, &tmx, &bar_x[b], st * kStageK, tok0 + tb * BN);
         ++issued;
@@ -349,7 +351,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
       int issued = 0, s = 0;
       uint32_t ph = 0;
       for (int i = 0; i < n_items; ++i) {
-        if (!mbar_wait(&bar_ifree[s], ph ^ 1, abrt)) break;
+        if (!mbar_wait(&bar_ifree[s], ph ^ 1, abrt, 64)) break;
         const int w = w0 + i, T = w / n_st, st = w - T * n_st, t = T % L.n_tiles;
         const int rows = min(kTileRows, L.N - t * kTileRows);
         const uint32_t bytes = (uint32_t)(NPC * rows * 16);
@@ -387,20 +389,24 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
       const int slot = (T == w0 / n_st) ? 0 : 1;
       float* part = work + ((size_t)(blockIdx.x * 2 + slot) * BN) * kTileRows + r;
       const uint32_t dcol = lane_base + (seg % NACC) * BN;
+      // 32 columns per wait: two loads in flight before their stores
 #pragma unroll 1
-      for (int cc = 0; cc < BN; cc += 16) {
-        uint32_t v[16];
-        tmem_ld16(dcol + cc, v);
+      for (int cc = 0; cc < BN; cc += 32) {
+        uint32_t v[32];
+        tmem_ld16(dcol + cc, *reinterpret_cast<uint32_t(*)[16]>(v));
+        if (BN > 16) tmem_ld16(dcol + cc + 16, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
         tmem_wait_ld();
+        constexpr int CW = BN > 16 ? 32 : 16;
         if (full) {
           if (r < rows) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
+            for (int j = 0; j < CW; ++j)
               if (cc + j < ntok) store_out(out, (size_t)(tok_b + cc + j) * L.N + n, n, __uint_as_float(v[j]));
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) part[(size_t)(cc + j) * kTileRows] = __uint_as_float(v[j]);
+          for (int j = 0; j < CW; ++j)
+            if (cc + j < BN) part[(size_t)(cc + j) * kTileRows] = __uint_as_float(v[j]);
         }
       }
       tc_fence_before();
@@ -465,11 +471,13 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
     int b = 0, is = 0;         // A / x slot and index slot of the next item
     uint32_t bph = 0, iph = 0;  // their phase parities
 
-    for (int i = 0; i < n_items; ++i) {
+    // Item i's index words (the index slot goes back to the producer), the
+    // sidecar cursor moved to it, and its decoded words: hi (and mid), two
+    // weights per 32-bit TMEM cell. false if a wait gave up.
+    auto fetch_decode = [&](int i, uint32_t (&hi)[8], uint32_t (&mid)[8]) -> bool {
       const int w = w0 + i, T = w / n_st, st = w - T * n_st, t = T % L.n_tiles;
       const int rows = min(kTileRows, L.N - t * kTileRows);
-      // this quarter's index bytes, then the slot goes back to the producer
-      if (!mbar_wait(&bar_ifull[is], iph, abrt)) break;
+      if (!mbar_wait(&bar_ifull[is], iph, abrt)) return false;
       const uint8_t* src = ring + (size_t)is * ISLOT + r * 16;
       uint32_t wd[4] = {0, 0, 0, 0};
       if (r < rows) {
@@ -500,10 +508,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
         }
       }
       while (pkn < k0) step();  // entries in other quarters
-      if (!mbar_wait(&bar_empty[b], bph ^ 1, abrt)) break;
-      tc_fence_after();
-      const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS + g * 8;
-      uint32_t hi[8], mid[8];
       if (MODE == HXQ_MODE_SCALAR8) {
         uint32_t v[16];
 #pragma unroll
@@ -546,13 +550,31 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
           step();
         }
       }
+      return true;
+    };
+
+    // Software pipeline: item i's TMEM stores drain while item i + 1 is
+    // fetched and decoded; then the stores are waited for and the MMA
+    // thread is told that slot b holds item i.
+    uint32_t hi[8], mid[8], nhi[8], nmid[8];
+    bool ok = n_items > 0 && fetch_decode(0, hi, mid);
+    for (int i = 0; ok && i < n_items; ++i) {
+      if (!mbar_wait(&bar_empty[b], bph ^ 1, abrt)) break;
+      tc_fence_after();
+      const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS + g * 8;
       tmem_st8(acol, hi);
       if (TERMS == 2) tmem_st8(acol + 32, mid);
+      if (i + 1 < n_items) ok = fetch_decode(i + 1, nhi, nmid);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_a[b]);
       if (++b == kSlots) b = 0, bph ^= 1;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        hi[j] = nhi[j];
+        mid[j] = nmid[j];
+      }
     }
   }
 
