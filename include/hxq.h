@@ -88,10 +88,17 @@ enum {
  * indices out into 128-row tiles for coalesced loads (same information, rows
  * padded to whole 16- or 64-weight chunks), sorts the sidecar into per-row
  * patch lists, and synchronises the device before returning: the caller may
- * free its buffers afterwards. The handle is immutable and owns a split-K
- * workspace, so forwards on ONE handle must not overlap in time on the GPU
- * (different streams racing on it give wrong results); different handles are
- * independent.
+ * free its buffers afterwards. Device memory of a handle: the re-laid-out
+ * indices, 12 bytes per sidecar entry plus the per-row and per-stage patch
+ * offsets, the codebook, and a small split-K workspace of the CUDA-core
+ * GEMV (2 x 8 x 128 floats per SM). The tensor-core kernels (M > 4) use a
+ * workspace per device and stream instead (2 x 256 x 128 floats per SM,
+ * 39 MB on a 148-SM B200), allocated by the first such forward issued on that
+ * stream and kept until the process exits: make that first forward before
+ * capturing the stream into a CUDA graph. The handle is immutable; forwards
+ * on ONE handle must not overlap in time on the GPU (different streams
+ * racing on it give wrong results); forwards of different handles may run
+ * concurrently on different streams.
  *
  * Returns HXQ_EINVAL for: NULL codebook/indices/out, NULL sidecar arrays with
  * n_sidecar > 0, n_sidecar < 0, > N*K or >= 2^31, N < 1, K < 8, K % 8 != 0, unknown
@@ -109,7 +116,9 @@ int hxq_linear_create(const float* codebook, const uint8_t* indices, int mode,
  * aligned. Asynchronous: returns after the launch. M >= 1. The handle's
  * device must be the current one (as for every call that takes a handle).
  * Returns HXQ_EINVAL for a NULL handle/x/y, M < 1, a misaligned x or
- * another device current; HXQ_ECUDA if a launch fails.
+ * another device current; HXQ_ENOMEM if the stream's tensor-core workspace
+ * cannot be allocated (first forward with M > 4 on a stream); HXQ_ECUDA if a
+ * launch fails.
  */
 int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M,
                        void* stream);

@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <numeric>
 #include <vector>
@@ -63,6 +64,46 @@ __global__ void sidecar_delta_kernel(Layer L, const int64_t* __restrict__ pos, i
   }
   delta[i] = L.pv[i] - c;
 }
+
+}  // namespace
+
+namespace hxq {
+namespace {
+struct StreamWorkspace {
+  int device;
+  cudaStream_t stream;
+  float* work;
+  size_t floats;
+};
+std::mutex g_ws_mu;
+std::vector<StreamWorkspace> g_ws;  // lives until the process exits
+}  // namespace
+
+cudaError_t tc_workspace(int device, cudaStream_t s, int num_sms, float** work, size_t* floats) {
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  for (const StreamWorkspace& w : g_ws)
+    if (w.device == device && w.stream == s) {
+      *work = w.work;
+      *floats = w.floats;
+      return cudaSuccess;
+    }
+  const size_t n = tc_workspace_floats(num_sms);
+  float* p = nullptr;
+  const cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&p), n * sizeof(float));
+  if (e != cudaSuccess) return e;
+  try {
+    g_ws.push_back({device, s, p, n});
+  } catch (const std::bad_alloc&) {
+    cudaFree(p);
+    return cudaErrorMemoryAllocation;
+  }
+  *work = p;
+  *floats = n;
+  return cudaSuccess;
+}
+}  // namespace hxq
+
+namespace {
 
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return HXQ_OK;
@@ -190,10 +231,9 @@ static int create_impl(const float* codebook, const uint8_t* indices, int mode, 
   const size_t cb_floats = mode == HXQ_MODE_SCALAR8 ? 256 : 8192;
   const size_t idx_bytes = (size_t)N * L.KC * 16 * L.P;
   const size_t src_bytes = mode == HXQ_MODE_SCALAR8 ? (size_t)NK : (size_t)(3 * NK / 4);
-  // stream-K workspace: two partial tiles per CTA (GEMV: per 128-thread
-  // virtual CTA, up to 32 tokens; tensor-core kernel: per CTA, up to 256 tokens)
-  h->work_floats = std::max<size_t>((size_t)h->num_sms * 4 * 2 * 32 * hxq::kTileRows,
-                                    hxq::tc_workspace_floats(h->num_sms));
+  // GEMV stream-K workspace: two partial tiles of up to 8 tokens per CTA (the
+  // tensor-core kernels use a workspace per device and stream, tc_workspace)
+  h->work_floats = (size_t)h->num_sms * 2 * hxq::kGemvMaxTokens * hxq::kTileRows;
   h->n_counters = L.n_tiles * 64 * hxq::kQuads;  // (token block, tile, quadrant)
 
   cudaError_t e = cudaSuccess;
@@ -307,7 +347,7 @@ int forward_impl(hxq_linear_t h, const void* x_bf16, const hxq::Out& out, int M,
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return e == cudaErrorInvalidValue ? HXQ_EINVAL : HXQ_ECUDA;
+    return e == cudaErrorInvalidValue ? HXQ_EINVAL : e == cudaErrorMemoryAllocation ? HXQ_ENOMEM : HXQ_ECUDA;
   }
   return HXQ_OK;
 }

@@ -121,6 +121,14 @@ cudaError_t launch_gemv_group(const hxq_group& g, const uint16_t* x, const Out* 
 bool gemv_supports(const hxq_linear& h, int M);
 int gemv_grid(const hxq_linear& h, int split);
 size_t tc_workspace_floats(int num_sms);
+// The tensor-core kernels' split-partial workspace for (device, stream):
+// allocated by the first tensor-core forward on that stream of that device
+// and kept until the process exits, so that forwards on different streams
+// never share one. cudaErrorMemoryAllocation if it cannot be allocated.
+cudaError_t tc_workspace(int device, cudaStream_t s, int num_sms, float** work, size_t* floats);
+// GEMV split partials per handle: two partial tiles of up to kGemvMaxTokens x
+// 128 floats per CTA.
+constexpr int kGemvMaxTokens = 8;
 
 // Launch `kern` with programmatic stream serialization: it may start while
 // the previous kernel in the stream drains, and waits for it (griddepcontrol

@@ -601,7 +601,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int BN, int TERMS, int MODE>
-cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid_req, cudaStream_t st) {
+cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid_req, float* work,
+                       size_t work_floats, cudaStream_t st) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tm;
@@ -630,8 +631,8 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
     int64_t grid = grid_req > 0 ? grid_req : std::min<int64_t>(h.num_sms, U * kMaxContrib);
     grid = std::max<int64_t>(1, std::min<int64_t>({grid, (int64_t)h.num_sms, W}));
     if (W * grid >= INT_MAX) return cudaErrorInvalidValue;  // item arithmetic is 32-bit
-    if ((size_t)grid * 2 * BN * kTileRows > h.work_floats) return cudaErrorInvalidValue;
-    e = launch_pdl(kern, (unsigned)grid, kTcThreads, smem, st, tm, h.L, out, M, tb0 * BN, n_tb, h.d_work,
+    if ((size_t)grid * 2 * BN * kTileRows > work_floats) return cudaErrorInvalidValue;
+    e = launch_pdl(kern, (unsigned)grid, kTcThreads, smem, st, tm, h.L, out, M, tb0 * BN, n_tb, work,
                    h.d_counters, h.d_status);
     if (e != cudaSuccess) return e;
   }
@@ -639,16 +640,19 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
 }
 
 template <int MODE>
-cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, cudaStream_t st) {
-  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, out, M, grid, st);
-  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, out, M, grid, st);
-  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, out, M, grid, st);
-  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, out, M, grid, st);
-  return launch_cfg<256, 1, MODE>(h, x, out, M, grid, st);
+cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, float* work,
+                        size_t work_floats, cudaStream_t st) {
+  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, out, M, grid, work, work_floats, st);
+  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, out, M, grid, work, work_floats, st);
+  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, out, M, grid, work, work_floats, st);
+  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, out, M, grid, work, work_floats, st);
+  return launch_cfg<256, 1, MODE>(h, x, out, M, grid, work, work_floats, st);
 }
 
 }  // namespace
 
+// Split partials of the tensor-core kernel: two slots of up to 256 tokens x
+// 128 rows per CTA.
 size_t tc_workspace_floats(int num_sms) { return (size_t)num_sms * 2 * 256 * kTileRows; }
 
 // `split` (when non-zero) sets the persistent grid so that each tile's K is
@@ -661,8 +665,12 @@ cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, in
     grid = std::max(1, n_tb * h.L.n_tiles * split);
     grid = std::min(grid, n_tb * h.L.n_tiles * kMaxContrib * 4);
   }
-  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, out, M, grid, st);
-  return launch_mode<HXQ_MODE_VQ2D12>(h, x, out, M, grid, st);
+  float* work = nullptr;
+  size_t work_floats = 0;
+  const cudaError_t e = tc_workspace(h.device, st, h.num_sms, &work, &work_floats);
+  if (e != cudaSuccess) return e;
+  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, out, M, grid, work, work_floats, st);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, out, M, grid, work, work_floats, st);
 }
 
 }  // namespace hxq
