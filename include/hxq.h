@@ -239,14 +239,14 @@ int hxq_assign(const float* points, int64_t n, int dim, const float* centroids, 
  * with the result). The pages name no initialisation and no stopping rule:
  * the caller supplies the start (for instance a seeded random sample of the
  * points) and the number of rounds. Each round assigns every point as
- * hxq_assign does and moves every centroid with points to their mean,
- * rounded to fp32; a centroid without points stays. The means are formed
- * from 64-bit fixed-point sums: each coordinate is scaled by 2^S and rounded
- * once, with 2^S = 2^(61 - lg - e) for n <= 2^lg points and every
- * |coordinate| < 2^e. Integer sums do not depend on order, so the result is
- * bitwise repeatable. A mean is within 2^(lg + e - 62) of the exact mean
- * before its fp32 rounding: for |w| < 0.125 and 2^24 points that is 2^-41,
- * about 4.5e-13. labels (NULL allowed)
+ * hxq_assign does and moves every centroid with points to their mean: the
+ * exact sum of their fp32 coordinates over their count, rounded once to fp32
+ * (nearest even); a centroid without points stays. The sums are exact
+ * integers on a fixed-point grid as fine as the smallest nonzero |coordinate|
+ * of the points, so every mean is correctly rounded whenever the nonzero
+ * magnitudes span at most 2^38 (e.g. 1e-12 .. 0.1); beyond that span the
+ * smallest coordinates are first rounded to that grid. Integer sums do not
+ * depend on order: results are bitwise repeatable. labels (NULL allowed)
  * receives the assignment to the final centroids. iters >= 0; other limits
  * and errors as hxq_assign, plus HXQ_ENOMEM if scratch cannot be allocated.
  */

@@ -28,8 +28,10 @@ Readings where the pages are silent (each is listed in the design notes):
   kernels: for one dimension d = |p - c| (one rounded subtraction); for
   pairs d = dx*dx + dy*dy, each product and the sum rounded to fp32 in that
   order, with no fused multiply-add. Equal distances go to the lowest index.
-* A centroid moves to the mean of its points, formed in float64 and rounded
-  to fp32 (nearest even); a centroid with no points stays where it is.
+* A centroid moves to the mean of its points: the exact mean of the points'
+  fp32 coordinates (their exact sum over their count, a rational number),
+  rounded once to fp32, nearest even; a centroid with no points stays where
+  it is. The sums are formed exactly, in integers.
 * The sidecar threshold is on |w - w_hat| per weight, in fp32, and strict
   (an error equal to the threshold is not stored). An entry stores the
   weight itself, the replacement form the decoder takes (the whitepaper's
@@ -81,19 +83,81 @@ def assign(points, centroids) -> np.ndarray:
     return out
 
 
+def round_rational_f32(num: int, den: int) -> np.float32:
+    """The fp32 value nearest to the rational num / den (den > 0), ties to
+    the even significand (IEEE 754 round to nearest even), subnormals
+    included; exact integer arithmetic throughout."""
+    num, den = int(num), int(den)
+    if den <= 0:
+        raise ValueError("den must be positive")
+    if num == 0:
+        return np.float32(0.0)
+    a = abs(num)
+    # 2^E <= a / den < 2^(E + 1)
+    E = a.bit_length() - den.bit_length()
+    if (a << max(0, -E)) < (den << max(0, E)):
+        E -= 1
+    lsb = max(E - 23, -149)  # weight of the significand's last bit
+    if lsb >= 0:
+        d = den << lsb
+        q, r = divmod(a, d)
+    else:
+        d = den
+        q, r = divmod(a << -lsb, den)
+    if 2 * r > d or (2 * r == d and q & 1):
+        q += 1
+    v = float(q) * 2.0 ** lsb  # exact: q <= 2^24 and 2^lsb >= 2^-149
+    return np.float32(-v if num < 0 else v)
+
+
+def f32_integer_parts(v):
+    """(m, e) with v = m * 2^e exactly, m a signed int64 (|m| < 2^24) and e
+    the exponent of the last significand bit (-149 for subnormals)."""
+    bits = np.ascontiguousarray(v, dtype=np.float32).view(np.uint32).astype(np.int64)
+    ef = (bits >> 23) & 0xFF
+    frac = bits & 0x7FFFFF
+    m = np.where(ef == 0, frac, frac | 0x800000)
+    m = np.where(bits >> 31 != 0, -m, m)
+    e = np.where(ef == 0, -149, ef - 150)
+    return m, e
+
+
+def exact_sums(values, labels, k):
+    """Exact sum of the fp32 values of each label 0..k-1, as Python integers
+    in units of 2^-149 (every fp32 value is an integer multiple of 2^-149).
+    The signed mantissas are split into 12-bit halves and added per (label,
+    exponent) bin with float64 weights: a bin of at most 2^31 values sums
+    to under 2^43 in magnitude, so float64 adds those integers exactly; each
+    bin's sum is then shifted into place as a Python integer."""
+    m, e = f32_integer_parts(values)
+    lab = np.asarray(labels, dtype=np.int64)
+    if lab.size >= 1 << 31:
+        raise ValueError("too many points for exact float64 bins")
+    key = lab * 256 + (e + 149)
+    sgn = np.sign(m)
+    a = np.abs(m)
+    lo = np.bincount(key, weights=(sgn * (a & 0xFFF)).astype(np.float64), minlength=k * 256)
+    hi = np.bincount(key, weights=(sgn * (a >> 12)).astype(np.float64), minlength=k * 256)
+    out = [0] * k
+    for b in np.flatnonzero((lo != 0) | (hi != 0)).tolist():
+        out[b >> 8] += ((int(hi[b]) << 12) + int(lo[b])) << (b & 255)
+    return out
+
+
 def kmeans_update(points, labels, centroids) -> np.ndarray:
-    """Each centroid moves to the mean of its points (float64 sum / count,
-    rounded to fp32); one without points keeps its position."""
-    p = _as_points(points).astype(np.float64)
+    """Each centroid moves to the mean of its points: their exact sum over
+    their count, rounded once to fp32 (nearest even); one without points
+    keeps its position."""
+    p = _as_points(points)
     c = _as_points(centroids)
     k, dim = c.shape
     labels = np.asarray(labels, dtype=np.int64)
     count = np.bincount(labels, minlength=k)
     new = c.copy()
     for d in range(dim):
-        s = np.bincount(labels, weights=p[:, d], minlength=k)
-        has = count > 0
-        new[has, d] = (s[has] / count[has]).astype(np.float32)
+        sums = exact_sums(p[:, d], labels, k)
+        for j in np.flatnonzero(count > 0).tolist():
+            new[j, d] = round_rational_f32(sums[j], int(count[j]) << 149)
     return new
 
 

@@ -43,6 +43,8 @@ def _load():
         lib.oracle_forward.restype = None
         lib.oracle_assign.argtypes = [vp, i64, i, vp, i, vp]
         lib.oracle_assign.restype = None
+        lib.oracle_assign_threads.argtypes = [vp, i64, i, vp, i, vp, i]
+        lib.oracle_assign_threads.restype = None
         lib.oracle_kmeans_update.argtypes = [vp, i64, i, vp, i, vp]
         lib.oracle_kmeans_update.restype = None
         lib.oracle_sidecar_select.argtypes = [vp, vp, i64, ctypes.c_float, vp, vp, i64]
@@ -106,10 +108,14 @@ def _pts(a):
     return p.reshape(-1, 1) if p.ndim == 1 else p
 
 
-def assign(points, centroids) -> np.ndarray:
+def assign(points, centroids, threads=1) -> np.ndarray:
     p, c = _pts(points), _pts(centroids)
     lab = np.empty(p.shape[0], np.int32)
-    _load().oracle_assign(_p(p), int(p.shape[0]), int(p.shape[1]), _p(c), int(c.shape[0]), _p(lab))
+    if threads > 1:
+        _load().oracle_assign_threads(_p(p), int(p.shape[0]), int(p.shape[1]), _p(c), int(c.shape[0]), _p(lab),
+                                      int(threads))
+    else:
+        _load().oracle_assign(_p(p), int(p.shape[0]), int(p.shape[1]), _p(c), int(c.shape[0]), _p(lab))
     return lab.astype(np.int64)
 
 

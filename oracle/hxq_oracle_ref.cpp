@@ -20,10 +20,12 @@
 //    x widened exactly from its bf16 bits; s[m][n] the same sum of absolute
 //    values (the tolerance scale).
 // The encoder functions below follow the same readings as the numpy encoder
-// oracle: fp32 distance decisions with ties to the lowest index, float64
-// means rounded to fp32 with empty clusters kept, a strict threshold on
-// |w - w_hat| that stores the weight itself.
+// oracle: fp32 distance decisions with ties to the lowest index, the exact
+// mean of a cluster's fp32 coordinates rounded once to fp32 (nearest even)
+// with empty clusters kept, a strict threshold on |w - w_hat| that stores the
+// weight itself.
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <numeric>
@@ -142,8 +144,9 @@ int oracle_forward_rows(int mode, const float* codebook, const uint8_t* indices,
 // distance |p - c| (dim 1) or dx*dx + dy*dy (dim 2), every operation rounded
 // to fp32 as written (compiled without contraction); a strictly smaller
 // distance wins, so ties keep the lowest index.
-void oracle_assign(const float* points, int64_t n, int dim, const float* centroids, int k, int32_t* labels) {
-  for (int64_t i = 0; i < n; ++i) {
+static void oracle_assign_range(const float* points, int64_t i0, int64_t i1, int dim, const float* centroids, int k,
+                         int32_t* labels) {
+  for (int64_t i = i0; i < i1; ++i) {
     float best = 0.f;
     int bi = -1;
     for (int e = 0; e < k; ++e) {
@@ -167,21 +170,130 @@ void oracle_assign(const float* points, int64_t n, int dim, const float* centroi
   }
 }
 
-// One Lloyd update: each centroid with points moves to their mean (float64
-// sum in point order, divided by the count, rounded to fp32); the others stay.
+void oracle_assign(const float* points, int64_t n, int dim, const float* centroids, int k, int32_t* labels) {
+  oracle_assign_range(points, 0, n, dim, centroids, k, labels);
+}
+
+// oracle_assign on `threads` host threads, each on a contiguous block of
+// points (the same decisions; only the work is split).
+void oracle_assign_threads(const float* points, int64_t n, int dim, const float* centroids, int k,
+                           int32_t* labels, int threads) {
+  const int T = (int)std::max<int64_t>(1, std::min<int64_t>(threads, n));
+  std::vector<std::thread> pool;
+  for (int t = 1; t < T; ++t)
+    pool.emplace_back(oracle_assign_range, points, n * t / T, n * (t + 1) / T, dim, centroids, k, labels);
+  oracle_assign_range(points, 0, n / T, dim, centroids, k, labels);
+  for (auto& th : pool) th.join();
+}
+
+}  // extern "C"
+
+namespace {
+
+// The exact sum of fp32 values as a signed integer in units of 2^-149
+// (every fp32 value is a multiple of 2^-149; the largest is below 2^128, so
+// 277 bits plus the count's bits), kept as base-2^32 digits in int64 words
+// that absorb carries until the end.
+struct ExactSum {
+  static constexpr int kDigits = 11;  // 352 bits
+  int64_t d[kDigits] = {};
+  void add(float v) {
+    uint32_t bits;
+    std::memcpy(&bits, &v, sizeof bits);
+    const int ef = (int)((bits >> 23) & 0xFF);
+    uint64_t m = bits & 0x7FFFFFu;
+    int shift = 0;  // position of m's last bit above 2^-149
+    if (ef != 0) {
+      m |= 0x800000u;
+      shift = ef - 1;
+    }
+    if (m == 0) return;
+    const int neg = (int)(bits >> 31);
+    const unsigned __int128 wide = (unsigned __int128)m << (shift % 32);  // under 2^56
+    const int i = shift / 32;
+    const int64_t lo = (int64_t)(uint64_t)(wide & 0xFFFFFFFFu);
+    const int64_t hi = (int64_t)(uint64_t)(wide >> 32);
+    d[i] += neg ? -lo : lo;
+    d[i + 1] += neg ? -hi : hi;
+  }
+};
+
+// The fp32 value nearest to (sum x 2^-149) / count, ties to even: carries
+// resolved, magnitude divided by count digit by digit from the top, then
+// 24 significant bits kept with the rest deciding the rounding.
+float exact_mean_f32(const ExactSum& s, int64_t count) {
+  int64_t w[ExactSum::kDigits];
+  for (int i = 0; i < ExactSum::kDigits; ++i) w[i] = s.d[i];
+  for (int i = 0; i + 1 < ExactSum::kDigits; ++i) {  // carries: every digit into [0, 2^32)
+    const int64_t carry = w[i] >> 32;                  // floor division (arithmetic shift)
+    w[i] -= carry * ((int64_t)1 << 32);
+    w[i + 1] += carry;
+  }
+  const bool neg = w[ExactSum::kDigits - 1] < 0;
+  uint32_t mag[ExactSum::kDigits];
+  if (neg) {  // two's complement negation of the digit string
+    uint64_t borrow = 1;
+    for (int i = 0; i < ExactSum::kDigits; ++i) {
+      const uint64_t inv = (~(uint64_t)w[i]) & 0xFFFFFFFFu;
+      const uint64_t t = inv + borrow;
+      mag[i] = (uint32_t)t;
+      borrow = t >> 32;
+    }
+  } else {
+    for (int i = 0; i < ExactSum::kDigits; ++i) mag[i] = (uint32_t)w[i];
+  }
+  uint32_t q[ExactSum::kDigits];
+  uint64_t rem = 0;
+  for (int i = ExactSum::kDigits - 1; i >= 0; --i) {
+    const uint64_t cur = (rem << 32) | mag[i];
+    q[i] = (uint32_t)(cur / (uint64_t)count);
+    rem = cur % (uint64_t)count;
+  }
+  int top = -1;  // highest set bit of q
+  for (int i = ExactSum::kDigits - 1; i >= 0 && top < 0; --i)
+    if (q[i])
+      for (int b = 31; b >= 0; --b)
+        if ((q[i] >> b) & 1u) {
+          top = 32 * i + b;
+          break;
+        }
+  auto bit = [&](int j) -> uint32_t { return j < 0 ? 0u : (q[j / 32] >> (j % 32)) & 1u; };
+  const int p = top >= 24 ? top - 23 : 0;  // weight 2^(p - 149) of the kept last bit
+  uint64_t sig = 0;
+  for (int j = top; j >= p; --j) sig = (sig << 1) | bit(j);
+  bool up;
+  if (p == 0) {
+    up = 2 * rem > (uint64_t)count || (2 * rem == (uint64_t)count && (sig & 1));
+  } else {
+    bool rest = rem != 0;
+    for (int j = p - 2; j >= 0 && !rest; --j) rest = bit(j) != 0;
+    up = bit(p - 1) && (rest || (sig & 1));
+  }
+  sig += up ? 1 : 0;
+  const double v = std::ldexp((double)sig, p - 149);
+  return (float)(neg ? -v : v);
+}
+
+}  // namespace
+
+extern "C" {
+
+// One Lloyd update: each centroid with points moves to their mean -- the
+// exact sum of their fp32 coordinates over their count, rounded once to fp32
+// (nearest even); the others stay.
 void oracle_kmeans_update(const float* points, int64_t n, int dim, const int32_t* labels, int k,
                           float* centroids) {
-  std::vector<double> sum((size_t)k * dim, 0.0);
+  std::vector<ExactSum> sum((size_t)k * dim);
   std::vector<int64_t> count((size_t)k, 0);
   for (int64_t i = 0; i < n; ++i) {
     const int e = labels[i];
     ++count[(size_t)e];
-    for (int d = 0; d < dim; ++d) sum[(size_t)e * dim + d] += (double)points[i * dim + d];
+    for (int d = 0; d < dim; ++d) sum[(size_t)e * dim + d].add(points[i * dim + d]);
   }
   for (int e = 0; e < k; ++e)
     if (count[(size_t)e] > 0)
       for (int d = 0; d < dim; ++d)
-        centroids[(size_t)e * dim + d] = (float)(sum[(size_t)e * dim + d] / (double)count[(size_t)e]);
+        centroids[(size_t)e * dim + d] = exact_mean_f32(sum[(size_t)e * dim + d], count[(size_t)e]);
 }
 
 // Flat positions (ascending) where |w - w_hat| > t in fp32, and the weights

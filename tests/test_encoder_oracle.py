@@ -285,3 +285,85 @@ def test_hand_worked_encoder_cases():
             pos, val = enc.sidecar_select(w, cb[lab], t)
             assert np.array_equal(pos, [int(v) for v in f[5]]), name
             assert np.array_equal(val, _arr(f[6])), name
+
+
+# ---- the exact mean rounded once to fp32 (reading: exact sum / count, one
+# rounding to nearest even)
+
+def _nearest_f32_brute(fr):
+    """Round the Fraction fr to fp32 by comparing it exactly with its two fp32
+    neighbours (ties to the even significand)."""
+    from fractions import Fraction
+    if fr == 0:
+        return np.float32(0.0)
+    lo = np.float32(float(fr))  # near fr; step to the two neighbours around fr
+    while Fraction(float(lo)) > fr:
+        lo = np.nextafter(lo, np.float32(-np.inf))
+    while Fraction(float(np.nextafter(lo, np.float32(np.inf)))) <= fr:
+        lo = np.nextafter(lo, np.float32(np.inf))
+    hi = np.nextafter(lo, np.float32(np.inf))
+    if Fraction(float(lo)) == fr:
+        return lo
+    dl, dh = fr - Fraction(float(lo)), Fraction(float(hi)) - fr
+    if dl != dh:
+        return lo if dl < dh else hi
+    return lo if (int(np.float32(lo).view(np.uint32)) & 1) == 0 else hi
+
+
+def test_round_rational_matches_brute_force():
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    cases = [(1, 3), (-1, 3), (2, 3), (7, 10), (1, 1 << 150), (3, 1 << 150), (5, 1 << 150), (1, 1 << 151),
+             (-(1 << 24) - 1, 2), ((1 << 24) + 1, 2), ((1 << 25) + 2, 4), ((1 << 25) + 6, 4)]
+    for _ in range(3000):
+        den = int(rng.integers(1, 1 << 40))
+        num = int(rng.integers(-(1 << 62), 1 << 62)) >> int(rng.integers(0, 60))
+        cases.append((num, den << int(rng.integers(0, 140))))
+    for num, den in cases:
+        got = enc.round_rational_f32(num, den)
+        want = _nearest_f32_brute(Fraction(num, den))
+        assert got.view(np.uint32) == want.view(np.uint32), (num, den, got, want)
+
+
+def test_round_rational_equals_float32_of_exact_float64():
+    """Where the rational is exactly a float64, one rounding of that float64
+    to fp32 (numpy's cast) is the right answer."""
+    rng = np.random.default_rng(12)
+    x = rng.normal(0, 1, 20000) * np.exp2(rng.integers(-140, 100, 20000))
+    for v in x.tolist():
+        n, d = float(v).as_integer_ratio()
+        assert enc.round_rational_f32(n, d).view(np.uint32) == np.float32(v).view(np.uint32)
+
+
+def test_kmeans_update_is_exact_mean_rounded_once():
+    """Against Fraction arithmetic, on sets built so that a float64 running
+    sum is inexact: a huge value and many tiny ones in one cluster, exact
+    ties at fp32 midpoints."""
+    from fractions import Fraction
+    rng = np.random.default_rng(13)
+    pts = np.concatenate([rng.normal(0, 0.02, 4000), [3.0e4], rng.normal(0, 1e-9, 3000),
+                          [np.float32(1.0), np.float32(1.0) + np.float32(2.0 ** -23)]]).astype(np.float32)
+    lab = np.concatenate([rng.integers(0, 5, 4000), [5], np.full(3000, 5), [6, 6]])
+    c = np.zeros(7, np.float32)
+    new = enc.kmeans_update(pts, lab, c)
+    for j in range(7):
+        sel = pts[lab == j]
+        want = _nearest_f32_brute(sum((Fraction(float(v)) for v in sel), Fraction(0)) / len(sel))
+        assert new[j].view(np.uint32) == want.view(np.uint32), j
+    # 1 and 1 + 2^-23 average to a midpoint: ties to the even significand (1.0)
+    assert new[6] == np.float32(1.0)
+
+
+def test_kmeans_update_float64_running_sum_is_caught():
+    """A planted mistake: the mean as a float64 running sum over the count,
+    then one cast to fp32. For {10, 2^-22, 7 * 2^-60, 2^-22} the exact mean
+    is 2.5 + 2^-23 + 7 * 2^-62, just above the midpoint between 2.5 and the
+    next fp32 value, so it rounds up; the float64 sum drops the 7 * 2^-60,
+    lands on the midpoint and ties down to 2.5."""
+    pts = np.array([10.0, 2.0 ** -22, 7 * 2.0 ** -60, 2.0 ** -22], dtype=np.float32)
+    exact = enc.kmeans_update(pts, np.zeros(4, np.int64), np.zeros(1, np.float32))[0]
+    assert exact == np.nextafter(np.float32(2.5), np.float32(3.0))
+    running = np.float64(0.0)
+    for v in pts.tolist():
+        running += np.float64(v)
+    assert np.float32(running / 4) == np.float32(2.5)

@@ -131,3 +131,29 @@ def test_cpp_forward_rows_equals_forward(mode, N, K, ns, threads):
         assert np.array_equal(got, y[:, r0:r1])
     with pytest.raises(ValueError):
         cpp.forward_rows(layer, x, 3, 2)
+
+
+def test_cpp_exact_mean_matches_numpy_over_wide_magnitudes():
+    """The two oracles form the exact mean independently (C++: base-2^32
+    digit sums and long division; numpy: Python integers and a rational
+    rounding) and must agree bit for bit, on clusters spanning about 80
+    binades and on the planted midpoint case."""
+    rng = np.random.default_rng(3)
+    for trial in range(20):
+        n, k, dim = int(rng.integers(1, 20000)), int(rng.integers(1, 50)), int(rng.integers(1, 3))
+        pts = (rng.normal(0, 0.02, size=(n, dim)) * np.exp2(rng.integers(-40, 40, size=(n, dim)))).astype(np.float32)
+        lab = rng.integers(0, k, size=n)
+        c = rng.normal(size=(k, dim)).astype(np.float32)
+        a, b = enc.kmeans_update(pts, lab, c), cpp.kmeans_update(pts, lab, c)
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32)), trial
+    pts = np.array([10.0, 2.0 ** -22, 7 * 2.0 ** -60, 2.0 ** -22], np.float32)
+    got = cpp.kmeans_update(pts, np.zeros(4, np.int64), np.zeros(1, np.float32))[0, 0]
+    assert got == np.nextafter(np.float32(2.5), np.float32(3.0))
+
+
+def test_cpp_threaded_assign_equals_plain():
+    rng = np.random.default_rng(4)
+    for dim in (1, 2):
+        pts = rng.normal(0, 0.02, size=(30001, dim)).astype(np.float32)
+        cents = rng.normal(0, 0.02, size=(77, dim)).astype(np.float32)
+        assert np.array_equal(cpp.assign(pts, cents, threads=5), cpp.assign(pts, cents))

@@ -12,12 +12,20 @@
 // as any other fp32 evaluation of the same expressions.
 //
 // k-means rounds (Lloyd): the assignment kernel also adds every point into
-// its centroid's sum and count. The sums are 64-bit integers in fixed point
-// (each coordinate scaled by 2^S and rounded once, S chosen from the largest
-// magnitude and the point count so that no sum can overflow), added first in
-// shared memory and then once per CTA in global memory. Integer addition does
-// not depend on order, so the new centroids -- sum / count, rounded to fp32
-// -- are bitwise repeatable. A centroid without points stays where it is.
+// its centroid's sum and count. A centroid moves to the exact mean of its
+// points' fp32 coordinates, rounded once to fp32 (nearest even). The sums
+// are exact integers: each coordinate becomes q = p * 2^F, with F chosen
+// from the tensor's smallest nonzero magnitude so that every q is an integer
+// (and from the largest, so that |q| < 2^62), split as q = hi * 2^32 + lo
+// (lo in [0, 2^32)), and the two parts are added in separate 64-bit sums --
+// first in shared memory, then once per CTA in global memory -- which no
+// count of points below 2^31 can overflow. The finalizing kernel joins them
+// into a 128-bit integer, divides by the count and rounds the quotient to
+// fp32 from its bits and the remainder. Integer sums do not depend on order,
+// so the result is bitwise repeatable and equals the correctly rounded mean
+// whenever the nonzero magnitudes span at most 2^38 (beyond that the
+// smallest values are first rounded to the 2^-F grid). A centroid without
+// points stays where it is.
 //
 // Sidecar selection: a weight goes to the sidecar when |w - w_hat| > t in
 // fp32. The entries are written in ascending position without atomics: one
@@ -38,14 +46,15 @@ constexpr int kSideChunk = 8192;                                // weights per c
 constexpr int kSideThreads = 256;
 constexpr int kScanThreads = 1024;
 
-// Fixed-point shift S: every |p| < 2^e (e from the largest magnitude's
-// exponent field) and n <= 2^lg points keep |sum of p 2^S| < 2^61.
-__device__ __forceinline__ int fixed_shift(unsigned maxabs_bits, int64_t n) {
-  const int ef = (int)((maxabs_bits >> 23) & 0xFF);
-  const int e = ef == 0 ? -126 : ef - 126;
-  int lg = 0;
-  while (((int64_t)1 << lg) < n) ++lg;
-  return 61 - lg - e;
+// Fixed-point shift F of the k-means sums, from the largest magnitude's and
+// the smallest nonzero magnitude's fp32 bits (range[0], range[1]): a value
+// of exponent field ef >= 1 has its last bit at 2^(ef - 150) (subnormals at
+// 2^-149, as ef = 1), so F = 150 - ef_min makes every value an integer
+// multiple of 2^-F; it is lowered if needed so that every |q| < 2^62.
+__device__ __forceinline__ int fixed_shift(const unsigned* range) {
+  const int ef_max = max(1, (int)((range[0] >> 23) & 0xFF));
+  const int ef_min = range[1] == 0xFFFFFFFFu ? ef_max : max(1, (int)((range[1] >> 23) & 0xFF));
+  return min(150 - ef_min, 62 + 126 - ef_max);
 }
 
 template <int DIM>
@@ -59,22 +68,24 @@ __device__ __forceinline__ float dist(const float (&p)[2], const float* c) {
 // Nearest centroid of each of the n points [n][DIM]; optionally writes the
 // index (labels) and, with ACCUM, adds each point into its centroid's
 // fixed-point sum and count.
+// gsum: [2][k][DIM] (the hi sums, then the lo sums); range: the largest
+// and smallest nonzero magnitudes' bits.
 template <int DIM, typename OutT, bool ACCUM>
 __global__ void __launch_bounds__(kAssignThreads)
 assign_kernel(const float* __restrict__ pts, int64_t n, const float* __restrict__ cent, int k,
               OutT* __restrict__ labels, unsigned long long* __restrict__ gsum, unsigned* __restrict__ gcount,
-              const unsigned* __restrict__ maxabs_bits) {
+              const unsigned* __restrict__ range) {
   extern __shared__ __align__(16) unsigned char sm[];
   float* c = reinterpret_cast<float*>(sm);  // [k][DIM]
-  unsigned long long* ssum =
+  unsigned long long* ssum =               // [2][k][DIM]: hi, lo
       reinterpret_cast<unsigned long long*>(sm + (((size_t)k * DIM * sizeof(float) + 15) & ~(size_t)15));
-  unsigned* scount = reinterpret_cast<unsigned*>(ssum + (size_t)k * DIM);
+  unsigned* scount = reinterpret_cast<unsigned*>(ssum + 2 * (size_t)k * DIM);
   for (int i = threadIdx.x; i < k * DIM; i += blockDim.x) c[i] = cent[i];
-  int S = 0;
+  int F = 0;
   if (ACCUM) {
-    for (int i = threadIdx.x; i < k * DIM; i += blockDim.x) ssum[i] = 0ull;
+    for (int i = threadIdx.x; i < 2 * k * DIM; i += blockDim.x) ssum[i] = 0ull;
     for (int i = threadIdx.x; i < k; i += blockDim.x) scount[i] = 0u;
-    S = fixed_shift(*maxabs_bits, n);
+    F = fixed_shift(range);
   }
   __syncthreads();
 
@@ -110,8 +121,10 @@ assign_kernel(const float* __restrict__ pts, int64_t n, const float* __restrict_
         atomicAdd(scount + bi[j], 1u);
 #pragma unroll
         for (int d = 0; d < DIM; ++d) {
-          const long long q = llrint(ldexp((double)p[j][d], S));
-          atomicAdd(ssum + (size_t)bi[j] * DIM + d, (unsigned long long)q);
+          // exact: q has at most 24 significant bits
+          const long long q = llrint(ldexp((double)p[j][d], F));
+          atomicAdd(ssum + (size_t)bi[j] * DIM + d, (unsigned long long)(q >> 32));
+          atomicAdd(ssum + (size_t)(k + bi[j]) * DIM + d, (unsigned long long)(q & 0xFFFFFFFFll));
         }
       }
     }
@@ -122,32 +135,75 @@ assign_kernel(const float* __restrict__ pts, int64_t n, const float* __restrict_
       if (scount[i] == 0) continue;
       atomicAdd(gcount + i, scount[i]);
 #pragma unroll
-      for (int d = 0; d < DIM; ++d) atomicAdd(gsum + (size_t)i * DIM + d, ssum[(size_t)i * DIM + d]);
+      for (int d = 0; d < DIM; ++d) {
+        atomicAdd(gsum + (size_t)i * DIM + d, ssum[(size_t)i * DIM + d]);
+        atomicAdd(gsum + (size_t)(k + i) * DIM + d, ssum[(size_t)(k + i) * DIM + d]);
+      }
     }
   }
 }
 
-// Largest |p| as fp32 bits (non-negative floats order like their bits).
-__global__ void maxabs_kernel(const float* __restrict__ p, int64_t n, unsigned* __restrict__ out) {
-  unsigned m = 0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-    m = max(m, __float_as_uint(p[i]) & 0x7FFFFFFFu);
-  m = __reduce_max_sync(0xffffffffu, m);
-  if ((threadIdx.x & 31) == 0) atomicMax(out, m);
+// Largest |p| and smallest nonzero |p| as fp32 bits (non-negative floats
+// order like their bits): out[0] starts at 0, out[1] at 0xFFFFFFFF.
+__global__ void range_kernel(const float* __restrict__ p, int64_t n, unsigned* __restrict__ out) {
+  unsigned mx = 0, mn = 0xFFFFFFFFu;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const unsigned a = __float_as_uint(p[i]) & 0x7FFFFFFFu;
+    mx = max(mx, a);
+    if (a != 0) mn = min(mn, a);
+  }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  if ((threadIdx.x & 31) == 0) {
+    atomicMax(out, mx);
+    atomicMin(out + 1, mn);
+  }
 }
 
-// New centroid = sum / count (float64, rounded to fp32); no points: unchanged.
+__device__ __forceinline__ int bitlen128(unsigned __int128 v) {
+  const unsigned long long hi = (unsigned long long)(v >> 64), lo = (unsigned long long)v;
+  return hi ? 128 - __clzll((long long)hi) : (lo ? 64 - __clzll((long long)lo) : 0);
+}
+
+// The fp32 value nearest to T / (cnt * 2^F), ties to the even significand.
+// The numerator is scaled by 2^sh so that Q = |T| 2^sh / cnt has at least
+// 25 bits; the kept last bit is at max(2^(E - 23), 2^-149) for the value's
+// exponent E, i.e. at Q's bit p = max(len(Q) - 24, F + sh - 149); the bit
+// below it and everything further down, the remainder included, decide the
+// rounding.
+__device__ __forceinline__ float round_mean_f32(__int128 T, unsigned cnt, int F) {
+  if (T == 0) return 0.f;
+  const bool neg = T < 0;
+  const unsigned __int128 a = neg ? (unsigned __int128)(-T) : (unsigned __int128)T;  // below 2^94
+  const int cl = 32 - __clz((int)cnt);
+  const int sh = max(0, 26 - (bitlen128(a) - cl));  // then |T| 2^sh stays below 2^(26 + 32)
+  const unsigned __int128 num = a << sh;
+  const unsigned __int128 Q = num / cnt;
+  const unsigned long long R = (unsigned long long)(num % cnt);
+  const int Fe = F + sh;
+  const int p = max(bitlen128(Q) - 24, Fe - 149);  // at least 1: Q has at least 25 bits
+  const unsigned long long sig = p < 128 ? (unsigned long long)(Q >> p) : 0ull;
+  const bool half = p - 1 < 128 && ((unsigned)(Q >> (p - 1)) & 1u);
+  const unsigned __int128 below = p - 1 < 128 ? Q & ((((unsigned __int128)1) << (p - 1)) - 1) : Q;
+  const bool up = half && (below != 0 || R != 0 || (sig & 1));
+  const double v = ldexp((double)(sig + (up ? 1 : 0)), p - Fe);  // exact
+  return (float)(neg ? -v : v);
+}
+
+// New centroid = the exact sum over the count, rounded once to fp32; no
+// points: unchanged.
 __global__ void kmeans_finalize(float* __restrict__ cent, int k, int dim, const unsigned long long* __restrict__ gsum,
-                                const unsigned* __restrict__ gcount, const unsigned* __restrict__ maxabs_bits,
-                                int64_t n) {
+                                const unsigned* __restrict__ gcount, const unsigned* __restrict__ range) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= k) return;
   const unsigned cnt = gcount[i];
   if (cnt == 0) return;
-  const int S = fixed_shift(*maxabs_bits, n);
+  const int F = fixed_shift(range);
   for (int d = 0; d < dim; ++d) {
-    const double s = (double)(long long)gsum[(size_t)i * dim + d];
-    cent[(size_t)i * dim + d] = __double2float_rn(ldexp(s, -S) / (double)cnt);
+    const long long hi = (long long)gsum[(size_t)i * dim + d];
+    const long long lo = (long long)gsum[(size_t)(k + i) * dim + d];  // a sum of values below 2^32
+    const __int128 T = (__int128)hi * ((__int128)1 << 32) + (__int128)lo;
+    cent[(size_t)i * dim + d] = round_mean_f32(T, cnt, F);
   }
 }
 
@@ -283,19 +339,19 @@ int device_sms() {
 
 size_t assign_smem(int dim, int k, bool accum) {
   size_t s = ((size_t)k * dim * sizeof(float) + 15) & ~(size_t)15;
-  if (accum) s += (size_t)k * dim * sizeof(unsigned long long) + (size_t)k * sizeof(unsigned);
+  if (accum) s += 2 * (size_t)k * dim * sizeof(unsigned long long) + (size_t)k * sizeof(unsigned);
   return s;
 }
 
 template <int DIM, typename OutT, bool ACCUM>
 cudaError_t launch_assign(const float* pts, int64_t n, const float* cent, int k, OutT* labels,
-                          unsigned long long* gsum, unsigned* gcount, const unsigned* maxabs, cudaStream_t s) {
+                          unsigned long long* gsum, unsigned* gcount, const unsigned* range, cudaStream_t s) {
   auto kern = assign_kernel<DIM, OutT, ACCUM>;
   const size_t smem = assign_smem(DIM, k, ACCUM);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = grid_for(n, kAssignTile, device_sms(), 2);
-  kern<<<grid, kAssignThreads, smem, s>>>(pts, n, cent, k, labels, gsum, gcount, maxabs);
+  kern<<<grid, kAssignThreads, smem, s>>>(pts, n, cent, k, labels, gsum, gcount, range);
   return cudaGetLastError();
 }
 
@@ -304,25 +360,27 @@ cudaError_t kmeans_rounds(const float* pts, int64_t n, int k, int iters, float* 
                           cudaStream_t s) {
   cudaError_t e = cudaSuccess;
   if (iters > 0) {
-    // scratch: sums [k][DIM] int64, counts [k], the largest magnitude
-    const size_t bytes = (size_t)k * DIM * 8 + (size_t)k * 4 + 16;
+    // scratch: sums [2][k][DIM] int64, counts [k], the magnitude range
+    const size_t sums = 2 * (size_t)k * DIM * 8 + (size_t)k * 4;
+    const size_t bytes = sums + 16;
     void* scratch = nullptr;
     if ((e = cudaMallocAsync(&scratch, bytes, s)) != cudaSuccess) return e;
     auto* gsum = static_cast<unsigned long long*>(scratch);
-    auto* gcount = reinterpret_cast<unsigned*>(gsum + (size_t)k * DIM);
-    auto* maxabs = gcount + k;
+    auto* gcount = reinterpret_cast<unsigned*>(gsum + 2 * (size_t)k * DIM);
+    auto* range = gcount + k;
     const int sms = device_sms();
-    e = cudaMemsetAsync(maxabs, 0, sizeof(unsigned), s);
+    e = cudaMemsetAsync(range, 0, sizeof(unsigned), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(range + 1, 0xFF, sizeof(unsigned), s);
     if (e == cudaSuccess) {
-      maxabs_kernel<<<grid_for(n * DIM, 256, sms, 4), 256, 0, s>>>(pts, n * DIM, maxabs);
+      range_kernel<<<grid_for(n * DIM, 256, sms, 4), 256, 0, s>>>(pts, n * DIM, range);
       e = cudaGetLastError();
     }
     for (int it = 0; it < iters && e == cudaSuccess; ++it) {
-      e = cudaMemsetAsync(scratch, 0, (size_t)k * DIM * 8 + (size_t)k * 4, s);
+      e = cudaMemsetAsync(scratch, 0, sums, s);
       if (e == cudaSuccess)
-        e = launch_assign<DIM, uint16_t, true>(pts, n, cent, k, nullptr, gsum, gcount, maxabs, s);
+        e = launch_assign<DIM, uint16_t, true>(pts, n, cent, k, nullptr, gsum, gcount, range, s);
       if (e == cudaSuccess) {
-        kmeans_finalize<<<(k + 255) / 256, 256, 0, s>>>(cent, k, DIM, gsum, gcount, maxabs, n);
+        kmeans_finalize<<<(k + 255) / 256, 256, 0, s>>>(cent, k, DIM, gsum, gcount, range);
         e = cudaGetLastError();
       }
     }
