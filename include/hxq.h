@@ -283,11 +283,25 @@ int hxq_decode(hxq_linear_t h, float* W_out, void* stream);
 /*
  * Synchronise the device and report whether any kernel of this handle gave up
  * a bounded device-side wait since the last check (HXQ_ETIMEOUT, then the
- * flag is cleared) -- the tensor-core kernel bounds every pipeline wait at 2 s
- * and returns early instead of hanging. HXQ_OK otherwise, HXQ_EINVAL for a
- * NULL handle, HXQ_ECUDA if the device reports an error.
+ * flag and the handle's split-tile arrival counters are cleared, so that
+ * the next forward starts clean) -- the kernels bound every pipeline wait
+ * at 2 s and return early instead of hanging. HXQ_OK otherwise, HXQ_EINVAL
+ * for a NULL handle, HXQ_ECUDA if the device reports an error.
  */
 int hxq_linear_check(hxq_linear_t h);
+
+/*
+ * Test hook, not for production use: the tensor-core forward (M >= 5) with
+ * every pipeline wait bounded at wait_limit_us microseconds (1 .. 2e6) and
+ * the activations of item `withhold_item` (>= 0) of each CTA's range never
+ * requested, so that the MMA's wait for them runs out: the CTAs drain the
+ * copies they issued, free their tensor memory and return, and the next
+ * hxq_linear_check reports HXQ_ETIMEOUT. y is not written meaningfully.
+ * Nothing faults or hangs: every wait is bounded and nothing is left in
+ * flight. Returns HXQ_EINVAL for bad arguments, HXQ_ECUDA if a launch fails.
+ */
+int hxq_test_forward_withheld(hxq_linear_t h, const void* x_bf16, float* y, int M,
+                              int withhold_item, unsigned wait_limit_us, void* stream);
 
 /*
  * The CUDA-core GEMV (M <= 4) for callers that cannot call cudaMalloc at the
@@ -301,10 +315,15 @@ int hxq_linear_check(hxq_linear_t h);
  * kernel, but its scratch (per-tile arrival counters and the fp32 partial
  * sums of tiles split between CTAs) lives in one fixed array of 1 MiB + 16 KiB
  * compiled into this library, resident on every GPU that loads it until the
- * process exits; the call itself allocates nothing. The first call on a
- * device looks up that array's device address (cudaGetSymbolAddress) and
- * should come before any stream capture. Each call clears the counters on
- * `stream` before the kernel runs. All calls share the one array, which keeps
+ * process exits; the call itself allocates nothing. hxq_linear_create looks
+ * up that array's device address (cudaGetSymbolAddress) on its device, so
+ * the no-alloc call only reads a cached pointer; the pointer is kept for the
+ * life of the process and is not valid across cudaDeviceReset (create the
+ * handles again after a reset). The CUDA runtime may still load the
+ * kernel's code at its first launch in the process (lazy module loading);
+ * callers that must not allocate at all can set CUDA_MODULE_LOADING=EAGER
+ * or make one call during set-up. Each call clears the counters on `stream`
+ * before the kernel runs. All calls share the one array, which keeps
  * the last call's contents: calls that overlap in time on the GPU (other
  * streams, other threads) race and give wrong results -- serialise them.
  *

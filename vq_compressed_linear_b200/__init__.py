@@ -53,6 +53,8 @@ lib.hxq_decode.argtypes = [_vp, _vp, _vp]
 lib.hxq_decode.restype = _i
 lib.hxq_linear_check.argtypes = [_vp]
 lib.hxq_linear_check.restype = _i
+lib.hxq_test_forward_withheld.argtypes = [_vp, _vp, _vp, _i, _i, ctypes.c_uint, _vp]
+lib.hxq_test_forward_withheld.restype = _i
 lib.hxq_linear_info.argtypes = [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i),
                                 ctypes.POINTER(_i64)]
 lib.hxq_linear_info.restype = _i
@@ -75,7 +77,8 @@ lib.hxq_strerror.restype = ctypes.c_char_p
 
 EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_linear_forward_out",
             "hxq_linear_forward_noalloc", "hxq_group_create", "hxq_group_forward", "hxq_group_destroy", "hxq_assign", "hxq_kmeans", "hxq_encode", "hxq_decode",
-            "hxq_linear_check", "hxq_linear_info", "hxq_linear_destroy", "hxq_strerror")
+            "hxq_linear_check", "hxq_test_forward_withheld", "hxq_linear_info", "hxq_linear_destroy",
+            "hxq_strerror")
 
 
 class HXQError(RuntimeError):
@@ -186,6 +189,14 @@ def hxq_decode(h, W_out, stream=None) -> None:
 
 def hxq_linear_check(h) -> None:
     _check(lib.hxq_linear_check(h), "hxq_linear_check")
+
+
+def hxq_test_forward_withheld(h, x, y, M, withhold_item, wait_limit_us, stream=None) -> None:
+    """Test hook: the tensor-core forward with one item's activations withheld
+    and every pipeline wait bounded at wait_limit_us (the next
+    hxq_linear_check reports HXQ_ETIMEOUT)."""
+    _check(lib.hxq_test_forward_withheld(h, _ptr(x), _ptr(y), int(M), int(withhold_item), int(wait_limit_us),
+                                         _stream(stream)), "hxq_test_forward_withheld")
 
 
 def hxq_linear_info(h) -> tuple[int, int, int, int]:

@@ -300,6 +300,9 @@ static int create_impl(const float* codebook, const uint8_t* indices, int mode, 
     cudaGetLastError();
     return cuda_status(e);
   }
+  // the no-alloc forward's scratch address is looked up here, where
+  // allocating is allowed (a failure here is reported by that entry point)
+  if (hxq::noalloc_prepare(dev) != cudaSuccess) cudaGetLastError();
   *out = h;
   return HXQ_OK;
 }
@@ -450,9 +453,27 @@ int hxq_linear_check(hxq_linear_t h) {
     return HXQ_ECUDA;
   }
   if (status != 0) {
+    // an aborted launch may have left split-tile arrivals half counted
     cudaMemset(h->d_status, 0, sizeof(int));
+    cudaMemset(h->d_counters, 0, (size_t)h->n_counters * sizeof(int));
     cudaDeviceSynchronize();
     return HXQ_ETIMEOUT;
+  }
+  return HXQ_OK;
+}
+
+int hxq_test_forward_withheld(hxq_linear_t h, const void* x_bf16, float* y, int M, int withhold_item,
+                              unsigned wait_limit_us, void* stream) {
+  if (!h || !x_bf16 || !y || M < 5 || withhold_item < 0 || wait_limit_us < 1 || wait_limit_us > 2000000u)
+    return HXQ_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) != 0) return HXQ_EINVAL;
+  if (const int rc = check_device(h->device)) return rc;
+  const cudaError_t e = hxq::launch_tc(*h, static_cast<const uint16_t*>(x_bf16), hxq::Out{y, nullptr, 0}, M, 0,
+                                       static_cast<cudaStream_t>(stream), (uint64_t)wait_limit_us * 1000ull,
+                                       withhold_item);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e == cudaErrorInvalidValue ? HXQ_EINVAL : HXQ_ECUDA;
   }
   return HXQ_OK;
 }

@@ -987,6 +987,16 @@ cudaError_t noalloc_scratch(int dev, void** out) {
 }
 }  // namespace
 
+namespace hxq {
+// Looks up the scratch array's device address on device `dev` (current) and
+// caches it; called when a handle is created, so that the no-alloc entry
+// point itself only reads the cache.
+cudaError_t noalloc_prepare(int dev) {
+  void* p = nullptr;
+  return noalloc_scratch(dev, &p);
+}
+}  // namespace hxq
+
 extern "C" int hxq_linear_forward_noalloc(hxq_linear_t h, const void* x_bf16, float* y, int M, void* stream) {
   using namespace hxq;
   if (!h || !x_bf16 || !y || M < 1 || M > 4) return HXQ_EINVAL;

@@ -114,11 +114,16 @@ namespace hxq {
 cudaError_t launch_decode(const hxq_linear& h, float* W, cudaStream_t s);
 cudaError_t launch_gemv(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split,
                         cudaStream_t s);
+// wait_limit_ns bounds every pipeline wait; withhold_item >= 0 is a test
+// hook (that item of each CTA never gets its activations).
 cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split,
-                      cudaStream_t s);
+                      cudaStream_t s, uint64_t wait_limit_ns = 2000000000ull, int withhold_item = -1);
 // One launch of the GEMV over every layer of g (outs[i] for layer i).
 cudaError_t launch_gemv_group(const hxq_group& g, const uint16_t* x, const Out* outs, int M, cudaStream_t s);
 bool gemv_supports(const hxq_linear& h, int M);
+// Resolves (and caches) the device address of the no-alloc entry point's
+// scratch array on the current device `dev`.
+cudaError_t noalloc_prepare(int dev);
 int gemv_grid(const hxq_linear& h, int split);
 size_t tc_workspace_floats(int num_sms);
 // The tensor-core kernels' split-partial workspace for (device, stream):
@@ -229,7 +234,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t sleep_ns = 0) {
+                                          uint32_t sleep_ns = 0, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
@@ -237,7 +242,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 0) {  // the abort flag and the clock are read now and then, not on every poll
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         return false;
       }

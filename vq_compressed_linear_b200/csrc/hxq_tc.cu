@@ -172,10 +172,18 @@ __device__ __forceinline__ void quarter_words_2d(const uint8_t* p0, int rows, in
   }
 }
 
+// Test hook of the tensor-core kernel: the limit of every pipeline wait, and
+// an item of each CTA's range whose activations are never requested (-1 =
+// none), so that a test can make a wait run out without a GPU fault.
+struct TestHook {
+  uint64_t wait_limit_ns;
+  int withhold_item;
+};
+
 template <int BN, int TERMS, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int tok0, int n_tb,
-          float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status) {
+          float* __restrict__ work, int* __restrict__ counters, int* __restrict__ status, TestHook hook) {
   constexpr int XSLOT = BN * 128;
   constexpr int kSlots = num_slots<BN, TERMS>();
   constexpr int kIS = idx_slots<BN, TERMS, MODE>();
@@ -199,6 +207,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
   __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = hook.wait_limit_ns;
   const int n_st = n_stages(L);
   const int W = n_tb * L.n_tiles * n_st;
   const int G = gridDim.x;
@@ -292,9 +301,18 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
         const int T = w / n_st, st = w - T * n_st;
         const int tb = T / L.n_tiles;
         if (i + kIS + kPrefetchItems < n_items) prefetch_item(i + kIS + kPrefetchItems);
+        if (i == hook.withhold_item) {
+          // test hook: this item's activations are never requested; wait for
+          // the copies already issued and stop (the MMA thread's wait for
+          // them runs out and the CTA aborts)
+          volatile int never = 0;
+          for (int j = max(0, issued - kSlots); j < issued; ++j)
+            mbar_wait(&bar_x[j % kSlots], (j / kSlots) & 1, &never);
+          break;
+        }
         // (the producers run slots ahead: they poll with short sleeps, so that
         // their warps leave issue slots to the decoders)
-        if (!mbar_wait(&bar_empty[b], ph ^ 1, abrt, 64)) break;
+        if (!mbar_wait(&bar_empty[b], ph ^ 1, abrt, 64, lim)) break;
         mbar_arrive_expect_tx(&bar_x[b], XSLOT);
         tma_load_2d(xs + b * XSLOT, &tmx, &bar_x[b], st * kStageK, tok0 + tb * BN);
         ++issued;
@@ -319,9 +337,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
         if (first) {
           ++seg;
           const int u = seg / NACC;
-          if (u >= 1 && !mbar_wait(&bar_dfree[seg % NACC], (u - 1) & 1, abrt)) break;
+          if (u >= 1 && !mbar_wait(&bar_dfree[seg % NACC], (u - 1) & 1, abrt, 0, lim)) break;
         }
-        if (!mbar_wait(&bar_x[b], par, abrt) || !mbar_wait(&bar_a[b], par, abrt)) break;
+        if (!mbar_wait(&bar_x[b], par, abrt, 0, lim) || !mbar_wait(&bar_a[b], par, abrt, 0, lim)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(xs + b * XSLOT);
         const uint32_t dcol = tmem + (seg % NACC) * BN;
@@ -351,7 +369,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
       int issued = 0, s = 0;
       uint32_t ph = 0;
       for (int i = 0; i < n_items; ++i) {
-        if (!mbar_wait(&bar_ifree[s], ph ^ 1, abrt, 64)) break;
+        if (!mbar_wait(&bar_ifree[s], ph ^ 1, abrt, 64, lim)) break;
         const int w = w0 + i, T = w / n_st, st = w - T * n_st, t = T % L.n_tiles;
         const int rows = min(kTileRows, L.N - t * kTileRows);
         const uint32_t bytes = (uint32_t)(NPC * rows * 16);
@@ -384,7 +402,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
       const int tok_b = tok0 + tb * BN;           // first token of this block
       const int ntok = min(BN, M - tok_b);
       // a whole segment of MMAs away: sleep between polls
-      if (!mbar_wait(&bar_acc[seg % NACC], (seg / NACC) & 1, abrt, 200)) break;
+      if (!mbar_wait(&bar_acc[seg % NACC], (seg / NACC) & 1, abrt, 200, lim)) break;
       tc_fence_after();
       const int slot = (T == w0 / n_st) ? 0 : 1;
       float* part = work + ((size_t)(blockIdx.x * 2 + slot) * BN) * kTileRows + r;
@@ -477,7 +495,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
     auto fetch_decode = [&](int i, uint32_t (&hi)[8], uint32_t (&mid)[8]) -> bool {
       const int w = w0 + i, T = w / n_st, st = w - T * n_st, t = T % L.n_tiles;
       const int rows = min(kTileRows, L.N - t * kTileRows);
-      if (!mbar_wait(&bar_ifull[is], iph, abrt)) return false;
+      if (!mbar_wait(&bar_ifull[is], iph, abrt, 0, lim)) return false;
       const uint8_t* src = ring + (size_t)is * ISLOT + r * 16;
       uint32_t wd[4] = {0, 0, 0, 0};
       if (r < rows) {
@@ -559,7 +577,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
     uint32_t hi[8], mid[8], nhi[8], nmid[8];
     bool ok = n_items > 0 && fetch_decode(0, hi, mid);
     for (int i = 0; ok && i < n_items; ++i) {
-      if (!mbar_wait(&bar_empty[b], bph ^ 1, abrt)) break;
+      if (!mbar_wait(&bar_empty[b], bph ^ 1, abrt, 0, lim)) break;
       tc_fence_after();
       const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS + g * 8;
       tmem_st8(acol, hi);
@@ -602,7 +620,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int BN, int TERMS, int MODE>
 cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid_req, float* work,
-                       size_t work_floats, cudaStream_t st) {
+                       size_t work_floats, TestHook hook, cudaStream_t st) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tm;
@@ -633,7 +651,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
     if (W * grid >= INT_MAX) return cudaErrorInvalidValue;  // item arithmetic is 32-bit
     if ((size_t)grid * 2 * BN * kTileRows > work_floats) return cudaErrorInvalidValue;
     e = launch_pdl(kern, (unsigned)grid, kTcThreads, smem, st, tm, h.L, out, M, tb0 * BN, n_tb, work,
-                   h.d_counters, h.d_status);
+                   h.d_counters, h.d_status, hook);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -641,12 +659,12 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
 
 template <int MODE>
 cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, float* work,
-                        size_t work_floats, cudaStream_t st) {
-  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, out, M, grid, work, work_floats, st);
-  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, out, M, grid, work, work_floats, st);
-  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, out, M, grid, work, work_floats, st);
-  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, out, M, grid, work, work_floats, st);
-  return launch_cfg<256, 1, MODE>(h, x, out, M, grid, work, work_floats, st);
+                        size_t work_floats, TestHook hook, cudaStream_t st) {
+  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
+  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
+  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
+  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
+  return launch_cfg<256, 1, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
 }
 
 }  // namespace
@@ -657,7 +675,9 @@ size_t tc_workspace_floats(int num_sms) { return (size_t)num_sms * 2 * 256 * kTi
 
 // `split` (when non-zero) sets the persistent grid so that each tile's K is
 // shared by about `split` CTAs; 0 = one CTA per SM.
-cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split, cudaStream_t st) {
+cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int split, cudaStream_t st,
+                      uint64_t wait_limit_ns, int withhold_item) {
+  const TestHook hook{wait_limit_ns, withhold_item};
   int grid = 0;
   if (split > 0) {
     const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
@@ -669,8 +689,9 @@ cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, in
   size_t work_floats = 0;
   const cudaError_t e = tc_workspace(h.device, st, h.num_sms, &work, &work_floats);
   if (e != cudaSuccess) return e;
-  if (h.L.mode == HXQ_MODE_SCALAR8) return launch_mode<HXQ_MODE_SCALAR8>(h, x, out, M, grid, work, work_floats, st);
-  return launch_mode<HXQ_MODE_VQ2D12>(h, x, out, M, grid, work, work_floats, st);
+  if (h.L.mode == HXQ_MODE_SCALAR8)
+    return launch_mode<HXQ_MODE_SCALAR8>(h, x, out, M, grid, work, work_floats, hook, st);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, out, M, grid, work, work_floats, hook, st);
 }
 
 }  // namespace hxq
