@@ -79,8 +79,8 @@ enum {
  *  mode         HXQ_MODE_SCALAR8 or HXQ_MODE_VQ2D12
  *  sidecar_pos  n_sidecar int64 flat positions n*K + k (may be NULL if 0)
  *  sidecar_val  n_sidecar float replacement values (may be NULL if 0)
- *  N, K         output and input features, N >= 1, K >= 8, K % 8 == 0;
- *               2D mode additionally needs K % 4 == 0 (implied)
+ *  N, K         output and input features, N >= 1, K >= 1; 2D mode needs
+ *               K % 4 == 0 (each row's 12-bit index stream is whole bytes)
  *  out          receives the handle
  *
  * Pointers may be device or host memory (copies use cudaMemcpyDefault).
@@ -95,14 +95,19 @@ enum {
  * workspace per device and stream instead (2 x 256 x 128 floats per SM,
  * 39 MB on a 148-SM B200), allocated by the first such forward issued on that
  * stream and kept until the process exits: make that first forward before
- * capturing the stream into a CUDA graph. The handle is immutable; forwards
+ * capturing the stream into a CUDA graph. When K % 8 != 0 the rows of x are
+ * not 16-byte aligned for the tensor-core kernels' activation loads: such a
+ * forward first copies x into rows of K rounded up to 8 in a buffer of that
+ * stream (one more kernel launch; the buffer grows, after a synchronize of
+ * the stream, when a forward needs more than it holds, so run the largest M
+ * once before capturing). The handle is immutable; forwards
  * on ONE handle must not overlap in time on the GPU (different streams
  * racing on it give wrong results); forwards of different handles may run
  * concurrently on different streams.
  *
  * Returns HXQ_EINVAL for: NULL codebook/indices/out, NULL sidecar arrays with
- * n_sidecar > 0, n_sidecar < 0, > N*K or >= 2^31, N < 1, K < 8, K % 8 != 0, unknown
- * mode, a sidecar position outside [0, N*K) or repeated. HXQ_EUNSUPPORTED if
+ * n_sidecar > 0, n_sidecar < 0, > N*K or >= 2^31, N < 1, K < 1, 2D mode with
+ * K % 4 != 0, unknown mode, a sidecar position outside [0, N*K) or repeated. HXQ_EUNSUPPORTED if
  * the current device is not compute capability 10.0. HXQ_ENOMEM / HXQ_ECUDA
  * on allocation / copy failures (nothing is leaked).
  */
@@ -263,7 +268,7 @@ int hxq_kmeans(const float* points, int64_t n, int dim, int k, int iters, float*
  * fp32 pairs (2D). *n_sidecar (device int64) receives the number of such
  * weights; only the first min(*n_sidecar, max_sidecar) are written, so a
  * caller that finds *n_sidecar > max_sidecar can retry with more room.
- * Shape limits as hxq_linear_create (K >= 8, K % 8 == 0), N*K < 2^31.
+ * Shape limits as hxq_linear_create (K >= 1; 2D: K % 4 == 0), N*K < 2^31.
  * Returns HXQ_EINVAL for NULL W/codebook/indices/n_sidecar, NULL sidecar
  * arrays with max_sidecar > 0, max_sidecar < 0, a negative or NaN
  * threshold, an unknown mode or a bad shape; HXQ_ENOMEM / HXQ_ECUDA on

@@ -31,7 +31,8 @@ int main(void) {
     EXPECT(hxq_linear_create(cb, idx, HXQ_MODE_SCALAR8, &pos, &val, 1, 8, 8, NULL) == HXQ_EINVAL);
     EXPECT(hxq_linear_create(NULL, idx, HXQ_MODE_SCALAR8, NULL, NULL, 0, 8, 8, &h) == HXQ_EINVAL);
     EXPECT(hxq_linear_create(cb, idx, 7, NULL, NULL, 0, 8, 8, &h) == HXQ_EINVAL);
-    EXPECT(hxq_linear_create(cb, idx, HXQ_MODE_SCALAR8, NULL, NULL, 0, 8, 12, &h) == HXQ_EINVAL);
+    EXPECT(hxq_linear_create(cb, idx, HXQ_MODE_VQ2D12, NULL, NULL, 0, 8, 10, &h) == HXQ_EINVAL);
+    EXPECT(hxq_linear_create(cb, idx, HXQ_MODE_SCALAR8, NULL, NULL, 0, 8, 0, &h) == HXQ_EINVAL);
     EXPECT(h == NULL);
     EXPECT(hxq_linear_forward(NULL, x, y, 1, NULL) == HXQ_EINVAL);
     EXPECT(hxq_linear_forward_ex(NULL, x, y, 1, HXQ_KERNEL_AUTO, 0, NULL) == HXQ_EINVAL);

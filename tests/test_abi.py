@@ -52,7 +52,7 @@ def _create(m, cb, idx, mode, pos, val, ns, N, K, out=True):
 
 
 @pytest.mark.parametrize("case", ["null_out", "null_cb", "null_idx", "bad_mode", "N0", "K0", "Kneg",
-                                  "K_not_mult8", "neg_sidecar", "too_many_sidecar", "null_sidecar"])
+                                  "vq2d_K_not_mult4", "neg_sidecar", "too_many_sidecar", "null_sidecar"])
 def test_create_rejects_bad_arguments(case):
     import vq_compressed_linear_b200 as m
     N, K = 16, 32
@@ -68,7 +68,8 @@ def test_create_rejects_bad_arguments(case):
     if case == "N0": args["N"] = 0
     if case == "K0": args["K"] = 0
     if case == "Kneg": args["K"] = -8
-    if case == "K_not_mult8": args["K"] = 36
+    if case == "vq2d_K_not_mult4":
+        args.update(mode=1, K=34, cb=np.zeros(8192, np.float32))
     if case == "neg_sidecar": args["ns"] = -1
     if case == "too_many_sidecar": args["ns"] = N * K + 1
     if case == "null_sidecar": args["pos"] = None
@@ -158,8 +159,8 @@ def test_create_argument_rules_fuzzed():
            ns=st.one_of(st.integers(-3, 8), st.sampled_from([(1 << 31) - 1, 1 << 31, 1 << 40])),
            null_cb=st.booleans(), null_idx=st.booleans(), null_side=st.booleans(), null_out=st.booleans())
     def check(mode, N, K, ns, null_cb, null_idx, null_side, null_out):
-        invalid = (null_cb or null_idx or null_out or mode not in (0, 1) or N < 1 or K < 8 or K % 8
-                   or ns < 0 or ns > N * K or (ns > 0 and null_side) or ns >= (1 << 31))
+        invalid = (null_cb or null_idx or null_out or mode not in (0, 1) or N < 1 or K < 1
+                   or (mode == 1 and K % 4) or ns < 0 or ns > N * K or (ns > 0 and null_side) or ns >= (1 << 31))
         h = ctypes.c_void_p()
         rc = m.lib.hxq_linear_create(None if null_cb else m._ptr(cb), None if null_idx else m._ptr(idx), mode,
                                      None if null_side else m._ptr(pos), None if null_side else m._ptr(val),
@@ -206,8 +207,8 @@ def test_encoder_argument_rules_fuzzed():
            t=st.sampled_from([0.0, 0.5, -1e-9, float("nan"), float("inf")]), cap=st.integers(-2, 5),
            nulls=st.lists(st.booleans(), min_size=5, max_size=5))
     def check_encode(mode, N, K, t, cap, nulls):
-        bad = (nulls[0] or nulls[1] or nulls[2] or nulls[3] or mode not in (0, 1) or N < 1 or K < 8 or K % 8
-               or N * K >= (1 << 31) or not (t >= 0) or cap < 0 or (cap > 0 and nulls[4]))
+        bad = (nulls[0] or nulls[1] or nulls[2] or nulls[3] or mode not in (0, 1) or N < 1 or K < 1
+               or (mode == 1 and K % 4) or N * K >= (1 << 31) or not (t >= 0) or cap < 0 or (cap > 0 and nulls[4]))
         side = None if nulls[4] else m._ptr(buf)
         rc = m.lib.hxq_encode(P(nulls[0]), mode, N, K, P(nulls[1]), t, P(nulls[2]), side, side, cap,
                               None if nulls[3] else m._ptr(cnt), None)

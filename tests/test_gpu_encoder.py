@@ -174,7 +174,8 @@ def _encode_gpu(hxq, W, mode, cb, tau, cap):
 
 
 @pytest.mark.parametrize("mode,N,K,tau", [(0, 1000, 1024, 0.0009), (0, 37, 200, 0.0009), (1, 600, 512, 0.012),
-                                        (1, 9, 72, 0.003)])
+                                        (1, 9, 72, 0.003), (0, 41, 13, 0.0003), (0, 7, 1, 0.0),
+                                        (1, 33, 12, 0.003)])
 def test_encode_bit_exact(hxq, mode, N, K, tau):
     rng = np.random.default_rng(400 + mode + N)
     W = rng.normal(0, 0.02, size=(N, K)).astype(np.float32)
@@ -256,5 +257,5 @@ def test_encoder_rejects_bad_arguments(hxq):
                 cnt.data_ptr(), None) == hxq.HXQ_EINVAL
     assert enc_(p.data_ptr(), 2, 8, 8, c.data_ptr(), 0.1, idx.data_ptr(), None, None, 0,
                 cnt.data_ptr(), None) == hxq.HXQ_EINVAL
-    assert enc_(p.data_ptr(), 0, 8, 12, c.data_ptr(), 0.1, idx.data_ptr(), None, None, 0,
+    assert enc_(p.data_ptr(), 1, 4, 10, c.data_ptr(), 0.1, idx.data_ptr(), None, None, 0,
                 cnt.data_ptr(), None) == hxq.HXQ_EINVAL

@@ -90,6 +90,37 @@ def test_forward_matches_oracle(hxq, mode, N, K, M):
             assert_within(y, y_ref, s, tau_for(M, kernel), f"mode {mode} {N}x{K} M={M} k={kernel} S={split}")
 
 
+# Any nn.Linear width: scalar K with no alignment, 2D K a multiple of 4 but
+# not of 8. Rows of x are then not 16-byte aligned (element-wise staging in
+# the GEMV, a re-strided copy ahead of the tensor-core kernel).
+RAGGED = [(0, 37, 1), (0, 130, 7), (0, 129, 13), (0, 300, 1001), (1, 131, 4), (1, 200, 12), (1, 257, 1004)]
+
+
+@pytest.mark.parametrize("mode,N,K", RAGGED)
+def test_ragged_k_decode_bit_exact(hxq, mode, N, K):
+    layer = synthetic.make_layer(mode, N, K, 13, sidecar_count=max(1, N * K // 300))
+    W = hxq.HelixLinear.from_layer(layer).decode().cpu().numpy()
+    W_ref = oracle.decode(mode, layer["codebook"], layer["indices"], layer["sidecar_pos"],
+                          layer["sidecar_val"], N, K)
+    assert np.array_equal(W.view(np.uint32), W_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("mode,N,K", RAGGED)
+def test_ragged_k_forward_matches_oracle(hxq, mode, N, K):
+    layer = synthetic.make_layer(mode, N, K, 13, sidecar_count=max(1, N * K // 300))
+    lin = hxq.HelixLinear.from_layer(layer)
+    # M rising then falling: the tensor-core path's re-strided copy grows,
+    # then is reused by smaller forwards
+    for M in (1, 3, 4, 5, 8, 16, 32, 33, 300, 6):
+        x = synthetic.activations(M, K, 13 + M)
+        _, y_ref, s = oracle.forward_layer(layer, x)
+        kernels = [AUTO, TC] + ([GEMV] if M <= 8 else [])
+        for kernel in kernels:
+            for split in (0, 3):
+                y = run(hxq, lin, x, kernel, split)
+                assert_within(y, y_ref, s, tau_for(M, kernel), f"mode {mode} {N}x{K} M={M} k={kernel} S={split}")
+
+
 @pytest.mark.parametrize("M", [33, 256, 300])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_prefill_equals_bf16_weight_oracle(hxq, mode, M):

@@ -24,14 +24,14 @@ def _xdev(x_bits):
     return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).cuda()
 
 
-# The last three shapes cannot take the thread-block-cluster split (their
+# The last five shapes cannot take the thread-block-cluster split (their
 # tiles x 16, the largest cluster, stay under 70 % of the SMs), so they run
 # the stream-K decomposition whose counters and partial sums live in the
 # fixed array; the first shapes take the cluster split where the device
-# allows it.
+# allows it. The last two have rows of x that are not 16-byte aligned.
 @pytest.mark.parametrize("mode,N,K,M", [(0, 8512, 2048, 1), (0, 2048, 4096, 4), (1, 1100, 4096, 2),
                                         (0, 300, 200, 3), (0, 640, 8192, 4), (0, 200, 4096, 1),
-                                        (1, 384, 8192, 2)])
+                                        (1, 384, 8192, 2), (0, 300, 1001, 3), (1, 260, 1004, 1)])
 def test_noalloc_matches_forward_twice(hxq, mode, N, K, M):
     import torch
     num_sms = torch.cuda.get_device_properties(0).multi_processor_count

@@ -74,6 +74,8 @@ struct StreamWorkspace {
   cudaStream_t stream;
   float* work;
   size_t floats;
+  uint16_t* xpad;  // activations re-strided to 16-byte rows (K % 8 != 0)
+  size_t xpad_bytes;
 };
 std::mutex g_ws_mu;
 std::vector<StreamWorkspace> g_ws;  // lives until the process exits
@@ -92,7 +94,7 @@ cudaError_t tc_workspace(int device, cudaStream_t s, int num_sms, float** work, 
   const cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&p), n * sizeof(float));
   if (e != cudaSuccess) return e;
   try {
-    g_ws.push_back({device, s, p, n});
+    g_ws.push_back({device, s, p, n, nullptr, 0});
   } catch (const std::bad_alloc&) {
     cudaFree(p);
     return cudaErrorMemoryAllocation;
@@ -100,6 +102,33 @@ cudaError_t tc_workspace(int device, cudaStream_t s, int num_sms, float** work, 
   *work = p;
   *floats = n;
   return cudaSuccess;
+}
+
+cudaError_t tc_xpad(int device, cudaStream_t s, size_t bytes, uint16_t** xpad) {
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  for (StreamWorkspace& w : g_ws) {
+    if (w.device != device || w.stream != s) continue;
+    if (w.xpad_bytes < bytes) {
+      if (w.xpad) {
+        // kernels queued on this stream may still read the old buffer
+        cudaError_t e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return e;
+        cudaFree(w.xpad);
+        w.xpad = nullptr;
+        w.xpad_bytes = 0;
+      }
+      const size_t grown = std::max(bytes, (size_t)1 << 20);
+      cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&w.xpad), grown);
+      if (e != cudaSuccess) {
+        w.xpad = nullptr;
+        return e;
+      }
+      w.xpad_bytes = grown;
+    }
+    *xpad = w.xpad;
+    return cudaSuccess;
+  }
+  return cudaErrorInvalidResourceHandle;  // tc_workspace creates the entry first
 }
 }  // namespace hxq
 
@@ -156,7 +185,7 @@ static int create_impl(const float* codebook, const uint8_t* indices, int mode, 
   *out = nullptr;
   if (!codebook || !indices) return HXQ_EINVAL;
   if (mode != HXQ_MODE_SCALAR8 && mode != HXQ_MODE_VQ2D12) return HXQ_EINVAL;
-  if (N < 1 || K < 8 || (K % 8) != 0) return HXQ_EINVAL;
+  if (N < 1 || K < 1 || (mode == HXQ_MODE_VQ2D12 && (K % 4) != 0)) return HXQ_EINVAL;
   if (n_sidecar < 0 || n_sidecar > (int64_t)N * K) return HXQ_EINVAL;
   if (n_sidecar > 0 && (!sidecar_pos || !sidecar_val)) return HXQ_EINVAL;
   if (n_sidecar >= (int64_t)1 << 31) return HXQ_EINVAL;  // patch offsets are int32

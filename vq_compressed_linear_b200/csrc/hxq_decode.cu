@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(256) decode_scalar_kernel(Layer L, float* __re
   }
   float* out = W + (int64_t)n * L.K + k0;
   const int cnt = min(16, L.K - k0);
-  if (cnt == 16) {
+  if (cnt == 16 && (reinterpret_cast<uintptr_t>(out) & 15) == 0) {
 #pragma unroll
     for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(out + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
   } else {
@@ -60,6 +60,7 @@ __global__ void __launch_bounds__(256) decode_vq2d_kernel(Layer L, float* __rest
   const int k0 = c * 64;
   float* out = W + (int64_t)n * L.K + k0;
   const int cnt = min(64, L.K - k0);
+  const bool v2 = (reinterpret_cast<uintptr_t>(out) & 7) == 0;
   int p = row_lower_bound(L, n, k0);
   const int pe = L.row_ptr[n + 1];
 #pragma unroll
@@ -70,8 +71,11 @@ __global__ void __launch_bounds__(256) decode_vq2d_kernel(Layer L, float* __rest
     for (; p < pe && L.pk[p] < k0 + 2 * j + 2; ++p) {
       if (L.pk[p] == k0 + 2 * j) v.x = L.pv[p]; else v.y = L.pv[p];
     }
-    if (2 * j + 1 < cnt) {
+    if (2 * j + 1 < cnt && v2) {
       *reinterpret_cast<float2*>(out + 2 * j) = v;
+    } else if (2 * j + 1 < cnt) {
+      out[2 * j] = v.x;
+      out[2 * j + 1] = v.y;
     } else if (2 * j < cnt) {
       out[2 * j] = v.x;
     }

@@ -460,7 +460,8 @@ int hxq_encode(const float* W, int mode, int N, int K, const float* codebook, fl
   using namespace hxq;
   if (!W || !codebook || !indices || !n_sidecar) return HXQ_EINVAL;
   if (mode != HXQ_MODE_SCALAR8 && mode != HXQ_MODE_VQ2D12) return HXQ_EINVAL;
-  if (N < 1 || K < 8 || (K % 8) != 0 || (int64_t)N * K >= kMaxPoints) return HXQ_EINVAL;
+  if (N < 1 || K < 1 || (mode == HXQ_MODE_VQ2D12 && (K % 4) != 0) || (int64_t)N * K >= kMaxPoints)
+    return HXQ_EINVAL;
   if (!(threshold >= 0.f) || max_sidecar < 0 || (max_sidecar > 0 && (!sidecar_pos || !sidecar_val)))
     return HXQ_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

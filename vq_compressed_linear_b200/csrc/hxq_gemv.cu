@@ -498,7 +498,18 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
   }
   // activations (zero-padded to Kp) once the previous kernel is done
   pdl_wait();
-  {
+  if (L.K & 7) {
+    // rows of x are not 16-byte aligned: one element per load
+    const int n = MT * L.Kp;
+    for (int i = threadIdx.x; i < n; i += kGemvThreads) {
+      const int m = i / L.Kp, k = i % L.Kp;
+      const uint16_t v = (m < M && k < L.K) ? __ldg(x + (size_t)m * L.K + k) : (uint16_t)0;
+      if (XF32)
+        *reinterpret_cast<float*>(sc.at((uint32_t)i * 4)) = bf16lo(v);
+      else
+        *reinterpret_cast<uint16_t*>(sc.at((uint32_t)i * 2)) = v;
+    }
+  } else {
     constexpr int XU = 4;  // activation loads in flight per thread
     const int n8 = MT * (L.Kp / 8);
     for (int i0 = threadIdx.x; i0 < n8; i0 += XU * kGemvThreads) {

@@ -131,6 +131,10 @@ size_t tc_workspace_floats(int num_sms);
 // and kept until the process exits, so that forwards on different streams
 // never share one. cudaErrorMemoryAllocation if it cannot be allocated.
 cudaError_t tc_workspace(int device, cudaStream_t s, int num_sms, float** work, size_t* floats);
+// A buffer of at least `bytes` for activations re-strided to 16-byte rows on
+// (device, stream), which tc_workspace must have created; grown (after a
+// synchronize of `s`) when a larger one is asked for.
+cudaError_t tc_xpad(int device, cudaStream_t s, size_t bytes, uint16_t** xpad);
 // GEMV split partials per handle: two partial tiles of up to kGemvMaxTokens x
 // 128 floats per CTA.
 constexpr int kGemvMaxTokens = 8;

@@ -618,14 +618,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// x [M][K] into rows of ld elements (ld = K rounded up to 8), so that every
+// row starts on the 16-byte boundary the activation tensor map needs.
+__global__ void __launch_bounds__(256) restride_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xp,
+                                                      int M, int K, int ld) {
+  const int64_t n = (int64_t)M * K;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = i / K;
+    xp[m * ld + (i - m * K)] = x[i];
+  }
+}
+
 template <int BN, int TERMS, int MODE>
-cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid_req, float* work,
-                       size_t work_floats, TestHook hook, cudaStream_t st) {
+cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, int ld, const Out& out, int M, int grid_req,
+                       float* work, size_t work_floats, TestHook hook, cudaStream_t st) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tm;
   cuuint64_t dims[2] = {(cuuint64_t)h.L.K, (cuuint64_t)M};
-  cuuint64_t strides[1] = {(cuuint64_t)h.L.K * 2};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   cuuint32_t box[2] = {(cuuint32_t)kStageK, (cuuint32_t)BN};
   cuuint32_t estr[2] = {1, 1};
   CUresult cr = fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
@@ -658,13 +669,13 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
 }
 
 template <int MODE>
-cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, const Out& out, int M, int grid, float* work,
-                        size_t work_floats, TestHook hook, cudaStream_t st) {
-  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
-  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
-  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
-  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
-  return launch_cfg<256, 1, MODE>(h, x, out, M, grid, work, work_floats, hook, st);
+cudaError_t launch_mode(const hxq_linear& h, const uint16_t* x, int ld, const Out& out, int M, int grid,
+                        float* work, size_t work_floats, TestHook hook, cudaStream_t st) {
+  if (M <= 16) return launch_cfg<16, 2, MODE>(h, x, ld, out, M, grid, work, work_floats, hook, st);
+  if (M <= 32) return launch_cfg<32, 2, MODE>(h, x, ld, out, M, grid, work, work_floats, hook, st);
+  if (M <= 64) return launch_cfg<64, 1, MODE>(h, x, ld, out, M, grid, work, work_floats, hook, st);
+  if (M <= 128) return launch_cfg<128, 1, MODE>(h, x, ld, out, M, grid, work, work_floats, hook, st);
+  return launch_cfg<256, 1, MODE>(h, x, ld, out, M, grid, work, work_floats, hook, st);
 }
 
 }  // namespace
@@ -687,11 +698,24 @@ cudaError_t launch_tc(const hxq_linear& h, const uint16_t* x, const Out& out, in
   }
   float* work = nullptr;
   size_t work_floats = 0;
-  const cudaError_t e = tc_workspace(h.device, st, h.num_sms, &work, &work_floats);
+  cudaError_t e = tc_workspace(h.device, st, h.num_sms, &work, &work_floats);
   if (e != cudaSuccess) return e;
+  int ld = h.L.K;
+  if (h.L.K % 8 != 0) {
+    // the tensor map's row stride must be a multiple of 16 bytes
+    ld = (h.L.K + 7) / 8 * 8;
+    uint16_t* xp = nullptr;
+    e = tc_xpad(h.device, st, (size_t)M * ld * sizeof(uint16_t), &xp);
+    if (e != cudaSuccess) return e;
+    const int64_t n = (int64_t)M * h.L.K;
+    const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, (int64_t)h.num_sms * 8);
+    restride_kernel<<<blocks, 256, 0, st>>>(x, xp, M, h.L.K, ld);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    x = xp;
+  }
   if (h.L.mode == HXQ_MODE_SCALAR8)
-    return launch_mode<HXQ_MODE_SCALAR8>(h, x, out, M, grid, work, work_floats, hook, st);
-  return launch_mode<HXQ_MODE_VQ2D12>(h, x, out, M, grid, work, work_floats, hook, st);
+    return launch_mode<HXQ_MODE_SCALAR8>(h, x, ld, out, M, grid, work, work_floats, hook, st);
+  return launch_mode<HXQ_MODE_VQ2D12>(h, x, ld, out, M, grid, work, work_floats, hook, st);
 }
 
 }  // namespace hxq
