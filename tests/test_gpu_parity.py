@@ -275,6 +275,42 @@ def test_full_size_prefill_sampled_rows(hxq, name, M):
     assert_within(y[:, rows], y_ref, s, TAU_PREFILL, f"prefill {name} M={M}")
 
 
+def _abs_layer(layer):
+    """The layer with |codebook| and |sidecar values|: its decode is |W|
+    elementwise (decode only selects values), so its forward on |x| is
+    s = sum_k |x||w|."""
+    a = dict(layer)
+    a["codebook"] = np.abs(layer["codebook"])
+    a["sidecar_val"] = np.abs(layer["sidecar_val"])
+    return a
+
+
+CPP_FULL = ([(cfg, name, M) for cfg in ("mamba2", "qwen25_3b", "vq2d")
+             for name, _, _, _, Ms, _ in synthetic.CONFIGS[cfg] for M in Ms]
+            + [("prefill", name, M) for name in ("mlp_up", "mlp_down") for M in (512, 2048)])
+
+
+@pytest.mark.parametrize("cfg,name,M", CPP_FULL)
+def test_full_size_against_plain_cpp_oracle(hxq, cfg, name, M):
+    """The benchmark's layers at full size, checked by the plain C++ loop
+    oracle (decode with the sidecar, float64 dot products, no library
+    routine): every output feature for M <= 32, four 128-row blocks
+    (first, last, two inside) for the prefill sizes."""
+    import os
+    from oracle import hxq_oracle_cpp as cpp
+    layer = dict((n, l) for n, l, _ in synthetic.config_layers(cfg))[name]
+    N = layer["N"]
+    x = synthetic.activations(M, layer["K"], 0)
+    y = run(hxq, hxq.HelixLinear.from_layer(layer), x)
+    blocks = [(0, N)] if M <= 32 else [(0, 128), (N // 3, N // 3 + 128), (N // 2 + 64, N // 2 + 192),
+                                       (N - 128, N)]
+    threads = os.cpu_count() or 1
+    for r0, r1 in blocks:
+        y_ref = cpp.forward_rows(layer, x, r0, r1, threads)
+        s = cpp.forward_rows(_abs_layer(layer), x & 0x7FFF, r0, r1, threads)
+        assert_within(y[:, r0:r1], y_ref, s, tau_for(M, AUTO), f"{cfg}/{name} M={M} rows {r0}:{r1}")
+
+
 def _cluster_shapes(num_sms):
     """Layer heights whose tile counts select each cluster size (2, 4, 8, and
     the non-portable 12 and 16 where the device allows them): tiles x size
