@@ -753,6 +753,52 @@ gemv_group_kernel(const __grid_constant__ GemvGroup g, const uint16_t* __restric
                             (int)blockIdx.x - g.first[li], g.first[li + 1] - g.first[li]);
 }
 
+// Launch shapes and SM sharing. Every launch may share an SM with the next
+// one (both at most kSmemShared bytes), so that the next layer's prologue
+// overlaps this one's tail. The block scheduler may then also put two CTAs of
+// ONE launch on an SM (when a CTA slot frees up next to a CTA of the same
+// launch): those two run at half speed and the whole launch waits for them.
+// Launches in clusters of 2 therefore take `exclusive_smem` bytes: two CTAs
+// of that size do not fit on one SM, one still fits next to a CTA of the
+// neighbouring launch. (Measured on the Mamba2 in_proj / out_proj pair: 15 %
+// less time per pair. Given the exclusive size, launches in larger clusters
+// got slower -- their clusters wait for whole groups of SMs to clear -- and
+// stream-K launches gained nothing, so they keep the shared size.)
+inline bool want_exclusive(int cs) { return cs == 2; }
+
+template <int MT, bool XF32, int MODE, bool GROUP>
+size_t exclusive_smem() {
+  static const size_t bytes = [] {
+    const void* kern = GROUP ? reinterpret_cast<const void*>(gemv_group_kernel<MT, XF32, MODE>)
+                             : reinterpret_cast<const void*>(gemv_kernel<MT, XF32, MODE>);
+    int dev = 0, per_sm = 0, reserved = 0;
+    cudaFuncAttributes fa;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+      cudaGetLastError();
+      return (size_t)0;
+    }
+    const size_t st = (fa.sharedSizeBytes + 127) / 128 * 128;
+    // smallest multiple of 128 with 2 x (dynamic + static + reserved) > per_sm
+    const size_t half = (size_t)per_sm / 2;
+    if (half < (size_t)reserved + st) return (size_t)0;
+    const size_t dyn = ((half - reserved - st) / 128 + 1) * 128;
+    // room left beside it for a CTA of kSmemShared dynamic bytes
+    if (dyn > kSmemLimit || 2 * (st + (size_t)reserved) + dyn + kSmemShared > (size_t)per_sm) return (size_t)0;
+    // the occupancy calculator agrees: one CTA per SM
+    int nb = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kGemvBlock, dyn) != cudaSuccess || nb != 1) {
+      cudaGetLastError();
+      return (size_t)0;
+    }
+    return dyn;
+  }();
+  return bytes;
+}
+
 // Sets the kernel's dynamic shared memory size and asks for the largest
 // shared-memory carveout, so that two CTAs of up to kSmemShared bytes each
 // (this launch's and the next one's) can be resident on one SM.
@@ -769,7 +815,7 @@ cudaError_t set_smem(Kern kern, size_t smem) {
 // the SMs without exceeding them and whose clusters all fit on the GPU at
 // once. 0 = the stream-K decomposition. `cached` keeps the answer for the
 // next launch of the same shape.
-template <int MT, bool XF32, int MODE, typename Kern>
+template <int MT, bool XF32, int MODE, bool GROUP, typename Kern>
 int pick_cluster_for(Kern kern, int n_tiles, int Kp, int num_sms, int& cached) {
   if (cached >= 0) return cached;
   cached = 0;
@@ -779,7 +825,8 @@ int pick_cluster_for(Kern kern, int n_tiles, int Kp, int num_sms, int& cached) {
     const int g = n_tiles * cs;
     if (g > num_sms || 100 * g < 70 * num_sms || n_st < cs) continue;
     if (ring_slots(MODE, MT, Kp, XF32, cs) < kMinRing) continue;
-    const size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
+    size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
+    if (want_exclusive(cs)) smem = std::max(smem, exclusive_smem<MT, XF32, MODE, GROUP>());
     if (set_smem(kern, smem) != cudaSuccess ||
         (cs > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
       cudaGetLastError();
@@ -813,7 +860,7 @@ constexpr int cluster_slot() { return (XF32 ? 4 : 0) + (MT <= 1 ? 0 : MT <= 2 ? 
 
 template <int MT, bool XF32, int MODE>
 int pick_cluster(const hxq_linear& h) {
-  return pick_cluster_for<MT, XF32, MODE>(gemv_kernel<MT, XF32, MODE>, h.L.n_tiles, h.L.Kp, h.num_sms,
+  return pick_cluster_for<MT, XF32, MODE, false>(gemv_kernel<MT, XF32, MODE>, h.L.n_tiles, h.L.Kp, h.num_sms,
                                           h.gemv_cluster[cluster_slot<MT, XF32>()]);
 }
 
@@ -825,7 +872,8 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, const Out& out, i
   const int cs = allow_cluster ? pick_cluster<MT, XF32, MODE>(h) : 0;
   if (cs > 0) {
     const int Rc = ring_slots(MODE, MT, h.L.Kp, XF32, cs);
-    const size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32, cs);
+    size_t smem = gemv_smem(MODE, MT, h.L.Kp, XF32, cs);
+    if (want_exclusive(cs)) smem = std::max(smem, exclusive_smem<MT, XF32, MODE, false>());
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl_cluster(kern, h.L.n_tiles * cs, kGemvBlock, smem, cs, s, h.L, x, out, M, W, Rc, cs, work, counters,
@@ -877,7 +925,7 @@ cudaError_t launch_group_cfg(const hxq_group& g, const uint16_t* x, const Out* o
     p.W[i] = (int)W[i];
     n_tiles += h.L.n_tiles;
   }
-  const int cs = pick_cluster_for<MT, XF32, MODE>(kern, n_tiles, Kp, g.num_sms,
+  const int cs = pick_cluster_for<MT, XF32, MODE, true>(kern, n_tiles, Kp, g.num_sms,
                                                   g.gemv_cluster[cluster_slot<MT, XF32>()]);
   p.first[0] = 0;
   if (cs > 0) {
@@ -899,7 +947,8 @@ cudaError_t launch_group_cfg(const hxq_group& g, const uint16_t* x, const Out* o
   const int grid = p.first[g.n];
   const int R = ring_slots(MODE, MT, Kp, XF32, cs);
   if (R < kMinRing) return cudaErrorInvalidValue;
-  const size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
+  size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
+  if (want_exclusive(cs)) smem = std::max(smem, exclusive_smem<MT, XF32, MODE, true>());
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   if (cs > 0) return launch_pdl_cluster(kern, grid, kGemvBlock, smem, cs, s, p, x, M, R, cs);
