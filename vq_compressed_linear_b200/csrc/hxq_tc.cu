@@ -443,14 +443,26 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
         if (last) {
           __threadfence();
           if (r < rows) {
-            for (int j0 = 0; j0 < ntok; j0 += 4) {  // 4 tokens' loads in flight per contributor
+            // 4 tokens x 8 contributors of loads in flight, then added in
+            // contributor order
+            for (int j0 = 0; j0 < ntok; j0 += 4) {
               float s4[4] = {0.f, 0.f, 0.f, 0.f};
-              for (int c = c_first; c <= c_last; ++c) {
-                const int cs = (T == ((c * W) / G) / n_st) ? 0 : 1;
-                const float* src = work + ((size_t)(c * 2 + cs) * BN + j0) * kTileRows + r;
+              for (int c0 = c_first; c0 <= c_last; c0 += 8) {
+                float pv[8][4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  if (j0 + u < ntok) s4[u] += __ldcg(src + u * kTileRows);
+                for (int e = 0; e < 8; ++e) {
+                  const int c = min(c0 + e, c_last);
+                  const int cs = (T == ((c * W) / G) / n_st) ? 0 : 1;
+                  const float* src = work + ((size_t)(c * 2 + cs) * BN + j0) * kTileRows + r;
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) pv[e][u] = j0 + u < ntok ? __ldcg(src + u * kTileRows) : 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  if (c0 + e <= c_last) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) s4[u] += pv[e][u];
+                  }
               }
 #pragma unroll
               for (int u = 0; u < 4; ++u)
