@@ -64,7 +64,7 @@ constexpr int kEpiWarp0 = 4;                            // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;                            // warps 8..: decoders
 constexpr int kTmemCols = 512;
 constexpr int kMaxTokBlocks = 64;                       // token blocks per launch (counter space)
-constexpr int kMaxContrib = 16;                         // CTAs sharing one tile's K at most
+constexpr int kMaxContrib = 8;                          // CTAs sharing one tile's K at most
 constexpr int kPrefetchItems = 16;                      // index bytes streamed into L2 this far ahead
 
 // Decoding warps: 4 groups of 4 (one warp per TMEM lane quadrant). Every
