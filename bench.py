@@ -253,9 +253,10 @@ def time_workload(hxq, torch, items, steps, warmup, l2_bytes, stream, soak_s=0.0
 
 
 def e2e_workload(hxq, torch, items, steps, warmup, stream, groups=()):
-    """Same metric through HelixLinear.forward_host semantics: pinned host x
-    in, y out, every step (one x per group for `groups`). Returns (ms, h2d
-    bytes/step, d2h bytes/step)."""
+    """Same metric through the host-buffer call (HelixLinear.forward_host,
+    i.e. hxq_linear_forward_host: pinned host x in, y out, on the stream) for
+    every layer of every step (grouped layers: one x copy per group and
+    HelixGroup.forward). Returns (ms, h2d bytes/step, d2h bytes/step)."""
     lins = [hxq.HelixLinear.from_layer(l) for _, l, _ in items]
     grps = [hxq.HelixGroup([lins[j] for j in g]) for g in groups]
     grouped = {j for g in groups for j in g}
@@ -274,9 +275,7 @@ def e2e_workload(hxq, torch, items, steps, warmup, stream, groups=()):
         for j, lin in enumerate(lins):
             if j in grouped:
                 continue
-            xd[j].copy_(xh[j], non_blocking=True)
-            lin.forward(xd[j], yd[j], stream=stream)
-            yh[j].copy_(yd[j], non_blocking=True)
+            lin.forward_host(xh[j], yh[j], xd[j], yd[j], stream=stream, sync=False)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):

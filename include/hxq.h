@@ -129,6 +129,23 @@ int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M,
                        void* stream);
 
 /*
+ * hxq_linear_forward on host buffers, as one call on `stream`: x from host
+ * memory x_host (bf16 bits [M][K]) into the caller's device buffer x_dev
+ * (M*K bf16, 16-byte aligned), the forward, and y into host memory y_host
+ * (M*N floats). Pinned host buffers are read and written by the kernels
+ * themselves (a small copy kernel for x; the forward stores y straight into
+ * y_host), which costs far less than copy-engine transfers of a few
+ * kilobytes; pageable buffers go through cudaMemcpyAsync, y by way of the
+ * caller's device buffer y_dev (M*N floats, unused otherwise). Asynchronous:
+ * synchronise the stream before reading y_host. Nothing is allocated beyond
+ * what hxq_linear_forward allocates. Returns HXQ_EINVAL for a NULL argument,
+ * M < 1, a misaligned x_dev or another device current; otherwise as
+ * hxq_linear_forward (HXQ_ECUDA also for a failed copy).
+ */
+int hxq_linear_forward_host(hxq_linear_t h, const void* x_host, void* x_dev, float* y_dev,
+                            float* y_host, int M, void* stream);
+
+/*
  * hxq_linear_forward with an explicit kernel choice (HXQ_KERNEL_*) and split
  * count along K (0 = automatic, else 1..64), for tests and benchmarks. The
  * numerics of each kernel are those stated above for its M range.

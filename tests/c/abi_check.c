@@ -38,6 +38,7 @@ int main(void) {
     EXPECT(hxq_linear_forward_ex(NULL, x, y, 1, HXQ_KERNEL_AUTO, 0, NULL) == HXQ_EINVAL);
     EXPECT(hxq_linear_forward_out(NULL, x, NULL, y, HXQ_OUT_F32, 1, NULL) == HXQ_EINVAL);
     EXPECT(hxq_linear_forward_noalloc(NULL, x, y, 1, NULL) == HXQ_EINVAL);
+    EXPECT(hxq_linear_forward_host(NULL, x, x, y, y, 1, NULL) == HXQ_EINVAL);
     EXPECT(hxq_decode(NULL, y, NULL) == HXQ_EINVAL);
     EXPECT(hxq_linear_check(NULL) == HXQ_EINVAL);
     EXPECT(hxq_linear_info(NULL, NULL, NULL, NULL, NULL) == HXQ_EINVAL);

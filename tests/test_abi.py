@@ -84,6 +84,7 @@ def test_forward_and_decode_reject_null_handle():
     assert m.lib.hxq_linear_forward_ex(None, m._ptr(x), m._ptr(y), 1, 0, 0, None) == m.HXQ_EINVAL
     assert m.lib.hxq_linear_forward_out(None, m._ptr(x), None, m._ptr(y), m.HXQ_OUT_F32, 1, None) == m.HXQ_EINVAL
     assert m.lib.hxq_linear_forward_noalloc(None, m._ptr(x), m._ptr(y), 1, None) == m.HXQ_EINVAL
+    assert m.lib.hxq_linear_forward_host(None, m._ptr(x), m._ptr(x), m._ptr(y), m._ptr(y), 1, None) == m.HXQ_EINVAL
     assert m.lib.hxq_decode(None, m._ptr(y), None) == m.HXQ_EINVAL
     assert m.lib.hxq_linear_check(None) == m.HXQ_EINVAL
     assert m.lib.hxq_linear_info(None, None, None, None, None) == m.HXQ_EINVAL

@@ -121,6 +121,37 @@ def test_ragged_k_forward_matches_oracle(hxq, mode, N, K):
                 assert_within(y, y_ref, s, tau_for(M, kernel), f"mode {mode} {N}x{K} M={M} k={kernel} S={split}")
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+@pytest.mark.parametrize("mode,N,K,M", [(0, 300, 200, 1), (0, 129, 13, 3), (1, 200, 136, 8), (0, 256, 512, 40),
+                                        (0, 8512, 2048, 1)])
+def test_forward_host_buffers(hxq, mode, N, K, M, pinned):
+    """hxq_linear_forward_host: x in, y out on one stream, with no
+    synchronisation between calls until the end; every call's y against
+    the oracle, and a bad call (misaligned x_dev) rejected before any copy.
+    Pinned buffers are read and written by the kernels, pageable ones go
+    through copies."""
+    import torch
+    layer = synthetic.make_layer(mode, N, K, 21, sidecar_count=max(1, N * K // 400))
+    lin = hxq.HelixLinear.from_layer(layer)
+    st = torch.cuda.Stream()
+    xs = [synthetic.activations(M, K, 21 + i) for i in range(3)]
+    pin = (lambda t: t.pin_memory()) if pinned else (lambda t: t)
+    xh = [pin(torch.from_numpy(x.view(np.int16))) for x in xs]
+    yh = [pin(torch.full((M, N), float("nan"), dtype=torch.float32)) for _ in xs]
+    xd = torch.empty((M, K), dtype=torch.int16, device="cuda")
+    yd = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    for i in range(3):
+        lin.forward_host(xh[i], yh[i], xd, yd, stream=st, sync=False)
+    st.synchronize()
+    lin.check()
+    for i in range(3):
+        _, y_ref, s = oracle.forward_layer(layer, xs[i])
+        assert_within(yh[i].numpy(), y_ref, s, tau_for(M, AUTO), f"host buffers call {i}")
+    xbad = torch.empty(M * K + 8, dtype=torch.int16, device="cuda")[1:]
+    assert hxq.lib.hxq_linear_forward_host(lin.handle, hxq._ptr(xh[0]), hxq._ptr(xbad), hxq._ptr(yd),
+                                           hxq._ptr(yh[0]), M, hxq._stream(st)) == hxq.HXQ_EINVAL
+
+
 @pytest.mark.parametrize("M", [33, 256, 300])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_prefill_equals_bf16_weight_oracle(hxq, mode, M):

@@ -47,6 +47,8 @@ lib.hxq_linear_forward_ex.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp]
 lib.hxq_linear_forward_ex.restype = _i
 lib.hxq_linear_forward_out.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _vp]
 lib.hxq_linear_forward_out.restype = _i
+lib.hxq_linear_forward_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _vp]
+lib.hxq_linear_forward_host.restype = _i
 lib.hxq_linear_forward_noalloc.argtypes = [_vp, _vp, _vp, _i, _vp]
 lib.hxq_linear_forward_noalloc.restype = _i
 lib.hxq_decode.argtypes = [_vp, _vp, _vp]
@@ -76,7 +78,7 @@ lib.hxq_strerror.argtypes = [_i]
 lib.hxq_strerror.restype = ctypes.c_char_p
 
 EXPORTED = ("hxq_linear_create", "hxq_linear_forward", "hxq_linear_forward_ex", "hxq_linear_forward_out",
-            "hxq_linear_forward_noalloc", "hxq_group_create", "hxq_group_forward", "hxq_group_destroy", "hxq_assign", "hxq_kmeans", "hxq_encode", "hxq_decode",
+            "hxq_linear_forward_host", "hxq_linear_forward_noalloc", "hxq_group_create", "hxq_group_forward", "hxq_group_destroy", "hxq_assign", "hxq_kmeans", "hxq_encode", "hxq_decode",
             "hxq_linear_check", "hxq_test_forward_withheld", "hxq_linear_info", "hxq_linear_destroy",
             "hxq_strerror")
 
@@ -135,6 +137,11 @@ def hxq_linear_forward_ex(h, x, y, M, kernel, split_k, stream=None) -> None:
 def hxq_linear_forward_out(h, x, bias, y, out_dtype, M, stream=None) -> None:
     _check(lib.hxq_linear_forward_out(h, _ptr(x), _ptr(bias), _ptr(y), int(out_dtype), int(M), _stream(stream)),
            "hxq_linear_forward_out")
+
+
+def hxq_linear_forward_host(h, x_host, x_dev, y_dev, y_host, M, stream=None) -> None:
+    _check(lib.hxq_linear_forward_host(h, _ptr(x_host), _ptr(x_dev), _ptr(y_dev), _ptr(y_host), int(M),
+                                       _stream(stream)), "hxq_linear_forward_host")
 
 
 def hxq_linear_forward_noalloc(h, x, y, M, stream=None) -> None:
@@ -254,17 +261,16 @@ class HelixLinear:
         hxq_linear_forward_out(self.handle, x, bias, y, out_dtype, M, stream)
         return y
 
-    def forward_host(self, x_host, y_host, x_dev, y_dev, stream=None):
-        """End-to-end call on host buffers: copy x (pinned) in, run, copy y out.
-        The caller owns the four buffers; the copies and the kernel share the
-        stream, which is synchronised before returning."""
+    def forward_host(self, x_host, y_host, x_dev, y_dev, stream=None, sync=True):
+        """End-to-end call on host buffers (hxq_linear_forward_host): copy x
+        (pinned) in, run, copy y (pinned) out, all on `stream`. The caller
+        owns the four buffers. With sync=False the call returns after
+        enqueuing; synchronise the stream before reading y_host."""
         import torch
         s = stream or torch.cuda.current_stream()
-        with torch.cuda.stream(s):
-            x_dev.copy_(x_host, non_blocking=True)
-            hxq_linear_forward_ex(self.handle, x_dev, y_dev, int(x_dev.shape[0]), HXQ_KERNEL_AUTO, 0, s)
-            y_host.copy_(y_dev, non_blocking=True)
-        s.synchronize()
+        hxq_linear_forward_host(self.handle, x_host, x_dev, y_dev, y_host, int(x_dev.shape[0]), s)
+        if sync:
+            s.synchronize()
         return y_host
 
     def decode(self, stream=None):

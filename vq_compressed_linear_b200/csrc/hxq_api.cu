@@ -65,6 +65,34 @@ __global__ void sidecar_delta_kernel(Layer L, const int64_t* __restrict__ pos, i
   delta[i] = L.pv[i] - c;
 }
 
+// x (bf16 bits) from host memory the GPU reads directly (pinned and mapped)
+// into a device buffer: a kernel instead of a copy-engine transfer, whose
+// fixed cost is several times that of a launch for a few kilobytes. Launched
+// with programmatic serialization: the host reads (the first kFetchVec
+// 16-byte words of each thread) are in flight while the previous kernel,
+// which may still read dst, finishes.
+constexpr int kFetchVec = 4;
+__global__ void __launch_bounds__(256) fetch_x_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst,
+                                                      int64_t n) {
+  hxq::pdl_launch_dependents();
+  const bool vec = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0;
+  const int64_t n8 = vec ? n / 8 : 0;  // 16-byte words
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  uint4 v[kFetchVec];
+#pragma unroll
+  for (int u = 0; u < kFetchVec; ++u)
+    if (t + u * stride < n8) v[u] = s4[t + u * stride];
+  hxq::pdl_wait();
+#pragma unroll
+  for (int u = 0; u < kFetchVec; ++u)
+    if (t + u * stride < n8) d4[t + u * stride] = v[u];
+  for (int64_t i = t + kFetchVec * stride; i < n8; i += stride) d4[i] = s4[i];
+  for (int64_t i = n8 * 8 + t; i < n; i += stride) dst[i] = src[i];
+}
+
 }  // namespace
 
 namespace hxq {
@@ -101,6 +129,36 @@ cudaError_t tc_workspace(int device, cudaStream_t s, int num_sms, float** work, 
   }
   *work = p;
   *floats = n;
+  return cudaSuccess;
+}
+
+namespace {
+std::mutex g_attr_mu;
+std::vector<std::pair<int, const void*>> g_attr_done;  // (device, kernel) pairs already set up
+}  // namespace
+
+cudaError_t allow_max_smem(const void* kern) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (const auto& d : g_attr_done)
+    if (d.first == dev && d.second == kern) return cudaSuccess;
+  int optin = 0;
+  cudaFuncAttributes fa;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess ||
+      (e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess)
+    return e;
+  // the opt-in maximum covers static and dynamic shared memory together
+  const int dyn_max = optin - (int)fa.sharedSizeBytes;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+    return e;
+  try {
+    g_attr_done.emplace_back(dev, kern);
+  } catch (const std::bad_alloc&) {
+  }
   return cudaSuccess;
 }
 
@@ -392,6 +450,53 @@ int hxq_linear_forward_ex(hxq_linear_t h, const void* x_bf16, float* y, int M, i
 
 int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M, void* stream) {
   return forward_impl(h, x_bf16, hxq::Out{y, nullptr, 0}, M, HXQ_KERNEL_AUTO, 0, stream);
+}
+
+namespace {
+// The address under which the GPU reads or writes host memory `p` directly
+// (pinned memory, mapped into the device's address space), or nullptr
+// (pageable memory, or not host memory at all).
+void* mapped_host(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+}  // namespace
+
+int hxq_linear_forward_host(hxq_linear_t h, const void* x_host, void* x_dev, float* y_dev, float* y_host, int M,
+                            void* stream) {
+  if (!h || !x_host || !x_dev || !y_dev || !y_host || M < 1) return HXQ_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x_dev) & 15) != 0) return HXQ_EINVAL;
+  if (const int rc = check_device(h->device)) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nx = (int64_t)M * h->L.K;
+  cudaError_t e = cudaSuccess;
+  if (const void* xm = mapped_host(x_host)) {
+    const int64_t per_block = 256LL * kFetchVec * 8;  // elements a block holds across the wait
+    const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>((nx + per_block - 1) / per_block,
+                                                                           (int64_t)h->num_sms));
+    e = hxq::launch_pdl(fetch_x_kernel, blocks, 256, 0, s, static_cast<const uint16_t*>(xm),
+                        static_cast<uint16_t*>(x_dev), nx);
+  } else {
+    e = cudaMemcpyAsync(x_dev, x_host, (size_t)nx * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_ECUDA;
+  }
+  // y straight into mapped host memory: every output is written once
+  float* ym = static_cast<float*>(mapped_host(y_host));
+  const int rc = forward_impl(h, x_dev, hxq::Out{ym ? ym : y_dev, nullptr, 0}, M, HXQ_KERNEL_AUTO, 0, stream);
+  if (rc != HXQ_OK || ym) return rc;
+  if (cudaMemcpyAsync(y_host, y_dev, (size_t)M * h->L.N * sizeof(float), cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return HXQ_ECUDA;
+  }
+  return HXQ_OK;
 }
 
 int hxq_linear_forward_out(hxq_linear_t h, const void* x_bf16, const float* bias, void* y, int out_dtype, int M,

@@ -348,7 +348,7 @@ cudaError_t launch_assign(const float* pts, int64_t n, const float* cent, int k,
                           unsigned long long* gsum, unsigned* gcount, const unsigned* range, cudaStream_t s) {
   auto kern = assign_kernel<DIM, OutT, ACCUM>;
   const size_t smem = assign_smem(DIM, k, ACCUM);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kern));
   if (e != cudaSuccess) return e;
   const int grid = grid_for(n, kAssignTile, device_sms(), 2);
   kern<<<grid, kAssignThreads, smem, s>>>(pts, n, cent, k, labels, gsum, gcount, range);

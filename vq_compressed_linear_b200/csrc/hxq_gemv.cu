@@ -789,7 +789,7 @@ size_t exclusive_smem() {
     if (dyn > kSmemLimit || 2 * (st + (size_t)reserved) + dyn + kSmemShared > (size_t)per_sm) return (size_t)0;
     // the occupancy calculator agrees: one CTA per SM
     int nb = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess ||
+    if (allow_max_smem(kern) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kGemvBlock, dyn) != cudaSuccess || nb != 1) {
       cudaGetLastError();
       return (size_t)0;
@@ -799,14 +799,13 @@ size_t exclusive_smem() {
   return bytes;
 }
 
-// Sets the kernel's dynamic shared memory size and asks for the largest
-// shared-memory carveout, so that two CTAs of up to kSmemShared bytes each
-// (this launch's and the next one's) can be resident on one SM.
+// Lets the kernel take `smem` bytes of dynamic shared memory, with the
+// largest shared-memory carveout, so that two CTAs of up to kSmemShared bytes
+// each (this launch's and the next one's) can be resident on one SM.
 template <typename Kern>
 cudaError_t set_smem(Kern kern, size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  (void)smem;  // the limit is the device's maximum; the launch passes its own size
+  return allow_max_smem(reinterpret_cast<const void*>(kern));
 }
 
 // Cluster split (no global-memory reduction): each tile gets a cluster of

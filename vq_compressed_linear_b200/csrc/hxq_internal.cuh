@@ -131,6 +131,11 @@ size_t tc_workspace_floats(int num_sms);
 // and kept until the process exits, so that forwards on different streams
 // never share one. cudaErrorMemoryAllocation if it cannot be allocated.
 cudaError_t tc_workspace(int device, cudaStream_t s, int num_sms, float** work, size_t* floats);
+// Lets `kern` launch with up to the device's opt-in maximum of dynamic shared
+// memory and asks for the largest shared-memory carveout, once per (device,
+// kernel): the launch's own size then sets its occupancy, and launches do not
+// repeat the driver calls.
+cudaError_t allow_max_smem(const void* kern);
 // A buffer of at least `bytes` for activations re-strided to 16-byte rows on
 // (device, stream), which tc_workspace must have created; grown (after a
 // synchronize of `s`) when a larger one is asked for.

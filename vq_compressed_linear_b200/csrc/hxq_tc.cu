@@ -660,7 +660,7 @@ cudaError_t launch_cfg(const hxq_linear& h, const uint16_t* x, int ld, const Out
   static_assert(tc_smem_bytes<BN, TERMS, MODE>() <= kTcSmemLimit, "shared memory budget");
   const size_t smem = std::max<size_t>(tc_smem_bytes<BN, TERMS, MODE>(), 116 * 1024);
   auto kern = tc_kernel<BN, TERMS, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kern));
   if (e != cudaSuccess) return e;
   const int n_tb_all = (M + BN - 1) / BN;
   const int n_st = n_stages(h.L);
