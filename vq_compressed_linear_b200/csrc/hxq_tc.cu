@@ -442,7 +442,25 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
         last = __shfl_sync(0xffffffffu, last, 0);
         if (last) {
           __threadfence();
-          if (r < rows) {
+          if (r < rows && BN <= 32) {
+            // all tokens of one contributor in flight at a time, added in
+            // contributor order
+            float acc[BN];
+#pragma unroll
+            for (int j = 0; j < BN; ++j) acc[j] = 0.f;
+            for (int c = c_first; c <= c_last; ++c) {
+              const int cs = (T == ((c * W) / G) / n_st) ? 0 : 1;
+              const float* src = work + ((size_t)(c * 2 + cs) * BN) * kTileRows + r;
+              float pv[BN];
+#pragma unroll
+              for (int j = 0; j < BN; ++j) pv[j] = j < ntok ? __ldcg(src + j * kTileRows) : 0.f;
+#pragma unroll
+              for (int j = 0; j < BN; ++j) acc[j] += pv[j];
+            }
+#pragma unroll
+            for (int j = 0; j < BN; ++j)
+              if (j < ntok) store_out(out, (size_t)(tok_b + j) * L.N + n, n, acc[j]);
+          } else if (r < rows) {
             // 4 tokens x 8 contributors of loads in flight, then added in
             // contributor order
             for (int j0 = 0; j0 < ntok; j0 += 4) {
