@@ -417,20 +417,28 @@ def _oracle_threads():
         return os.cpu_count() or 1
 
 
-def profile_run(hxq, torch, items, steps, warmup):
-    """Small, eager run for ncu: replicas just past 1.25x L2, W + K steps."""
+def profile_run(hxq, torch, items, steps, warmup, groups=()):
+    """Small, eager run for ncu: replicas just past 1.25x L2, W + K steps;
+    `groups` (index tuples into items) run as one grouped forward each."""
     props = torch.cuda.get_device_properties(0)
     l2 = getattr(props, "L2_cache_size", 126 << 20)
     dev_bytes = sum(l["indices"].size for _, l, _ in items)
     R = max(1, math.ceil(1.25 * l2 / dev_bytes))
     reps = [[hxq.HelixLinear.from_layer(l) for _, l, _ in items] for _ in range(R)]
+    grps = [[hxq.HelixGroup([rep[j] for j in g]) for g in groups] for rep in reps]
+    grouped = {j for g in groups for j in g}
     xs = [torch.from_numpy(synthetic.activations(M, l["K"], 1).view(np.int16)).cuda() for _, l, M in items]
     ys = [torch.empty((M, l["N"]), dtype=torch.float32, device="cuda") for _, l, M in items]
     for i in range(warmup + steps):
+        for gi, g in enumerate(groups):
+            grps[i % R][gi].forward(xs[g[0]], ys=[ys[j] for j in g])
         for j, lin in enumerate(reps[i % R]):
-            lin.forward(xs[j], ys[j])
+            if j not in grouped:
+                lin.forward(xs[j], ys[j])
     torch.cuda.synchronize()
-    for rep in reps:
+    for rep, gs in zip(reps, grps):
+        for grp in gs:
+            grp.close()
         for lin in rep:
             lin.check()
             lin.close()
@@ -627,7 +635,8 @@ def main():
     import vq_compressed_linear_b200 as hxq
 
     if args.ncu:
-        return profile_run(hxq, torch, items, args.steps, args.warmup)
+        return profile_run(hxq, torch, items, args.steps, args.warmup,
+                           item_groups(args.workload, items) if args.grouped else ())
     if args.encoder:
         return encoder_run(hxq, torch, args)
 
