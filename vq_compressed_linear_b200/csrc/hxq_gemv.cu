@@ -811,18 +811,23 @@ cudaError_t set_smem(Kern kern, size_t smem) {
 // Cluster split (no global-memory reduction): each tile gets a cluster of
 // cs CTAs (2..16; above 8 where the device allows such clusters) that split
 // its K, for the largest cs whose grid (tiles x cs) fills at least 70 % of
-// the SMs without exceeding them and whose clusters all fit on the GPU at
-// once. 0 = the stream-K decomposition. `cached` keeps the answer for the
-// next launch of the same shape.
+// the SMs without exceeding them (any fill for layers of at most a few
+// tiles) and whose clusters all fit on the GPU at once. 0 = the stream-K
+// decomposition. `cached` keeps the answer for the next launch of the same
+// shape.
 template <int MT, bool XF32, int MODE, bool GROUP, typename Kern>
 int pick_cluster_for(Kern kern, int n_tiles, int Kp, int num_sms, int& cached) {
   if (cached >= 0) return cached;
   cached = 0;
   if (MT > 4) return 0;
   const int n_st = Kp / kStageK;
+  // a layer too small to fill 70 % of the SMs at any cluster size takes the
+  // largest that fits: under stream-K its CTAs would hold a stage or two
+  // each, and the split-tile fixup chain would outlast the decode
+  const bool small = 100 * n_tiles * kMaxCluster < 70 * num_sms;
   for (int cs = kMaxCluster; cs >= 2; --cs) {
     const int g = n_tiles * cs;
-    if (g > num_sms || 100 * g < 70 * num_sms || n_st < cs) continue;
+    if (g > num_sms || (!small && 100 * g < 70 * num_sms) || n_st < cs) continue;
     if (ring_slots(MODE, MT, Kp, XF32, cs) < kMinRing) continue;
     size_t smem = gemv_smem(MODE, MT, Kp, XF32, cs);
     if (want_exclusive(cs)) smem = std::max(smem, exclusive_smem<MT, XF32, MODE, GROUP>());
