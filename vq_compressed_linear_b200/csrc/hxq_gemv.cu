@@ -594,6 +594,22 @@ __device__ __forceinline__ void gemv_body(const Layer& L, const uint16_t* __rest
             decode16<MODE>(smem, base + j * 512, rows, q_quarter, lane4, wv);
             fma16(acc[j][0], wv, xv);
           }
+        } else if (MODE == HXQ_MODE_VQ2D12 && MT >= 4) {
+          // 2D, four or more tokens: one row at a time (the pair unpack
+          // needs more registers than the scalar lookups), each token's
+          // activations loaded per row
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            asm volatile("" ::: "memory");
+            float wv[16];
+            decode16<MODE>(smem, base + j * 512, rows, q_quarter, lane4, wv);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              float xv[16];
+              x16<XF32>(sc, L.Kp, m, k0, xv);
+              fma16(acc[j][m], wv, xv);
+            }
+          }
         } else {
           // several tokens: rows two at a time, so that two rows' weights,
           // one token's activations and all the sums fit in registers
