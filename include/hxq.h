@@ -137,8 +137,12 @@ int hxq_linear_forward(hxq_linear_t h, const void* x_bf16, float* y, int M,
  * y_host), which costs far less than copy-engine transfers of a few
  * kilobytes; pageable buffers go through cudaMemcpyAsync, y by way of the
  * caller's device buffer y_dev (M*N floats, unused otherwise). Asynchronous:
- * synchronise the stream before reading y_host. Nothing is allocated beyond
- * what hxq_linear_forward allocates. Returns HXQ_EINVAL for a NULL argument,
+ * synchronise the stream before reading y_host. The x copy may read x_host
+ * before earlier work on the stream has finished (it overlaps the previous
+ * kernel), so x_host must hold its final contents when this call is made and
+ * must not be a buffer that earlier work on the stream writes; the four
+ * buffers must not overlap. Nothing is allocated beyond what
+ * hxq_linear_forward allocates. Returns HXQ_EINVAL for a NULL argument,
  * M < 1, a misaligned x_dev or another device current; otherwise as
  * hxq_linear_forward (HXQ_ECUDA also for a failed copy).
  */
