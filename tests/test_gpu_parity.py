@@ -147,6 +147,14 @@ def test_forward_host_buffers(hxq, mode, N, K, M, pinned):
     for i in range(3):
         _, y_ref, s = oracle.forward_layer(layer, xs[i])
         assert_within(yh[i].numpy(), y_ref, s, tau_for(M, AUTO), f"host buffers call {i}")
+    if pinned:
+        # x_host not 16-byte aligned: the fetch kernel copies element by element
+        xh_off = torch.empty(M * K + 1, dtype=torch.int16).pin_memory()
+        xh_off[1:].copy_(xh[0].view(-1))
+        yh2 = torch.full((M, N), float("nan"), dtype=torch.float32).pin_memory()
+        lin.forward_host(xh_off[1:].view(M, K), yh2, xd, yd, stream=st)
+        _, y_ref, s = oracle.forward_layer(layer, xs[0])
+        assert_within(yh2.numpy(), y_ref, s, tau_for(M, AUTO), "unaligned host x")
     xbad = torch.empty(M * K + 8, dtype=torch.int16, device="cuda")[1:]
     assert hxq.lib.hxq_linear_forward_host(lin.handle, hxq._ptr(xh[0]), hxq._ptr(xbad), hxq._ptr(yd),
                                            hxq._ptr(yh[0]), M, hxq._stream(st)) == hxq.HXQ_EINVAL
