@@ -67,10 +67,15 @@ constexpr int kMaxTokBlocks = 64;                       // token blocks per laun
 constexpr int kMaxContrib = 8;                          // CTAs sharing one tile's K at most
 constexpr int kPrefetchItems = 16;                      // index bytes streamed into L2 this far ahead
 
-// Decoding warps: 4 groups of 4 (one warp per TMEM lane quadrant). Every
-// decoding warp takes part in every item: group g decodes columns
-// [16 g, 16 g + 16) of the stage for the 32 rows of its quadrant.
-constexpr int kDecWarps = 16;
+// Decoding warps: one per TMEM lane quadrant and pair of 16-column groups.
+// Every decoding warp takes part in every item: warp (h, q) decodes the
+// column groups h and h + 2 ([16 g, 16 g + 16) of the stage) for the 32
+// rows of quadrant q. (Measured: 8 such warps beat 16 warps of one group --
+// fewer warps contend with the MMA thread for issue -- and 4 warps of four
+// groups; Qwen2.5-3B layers at M=32 155 -> 140 us, prefill M=2048 466 -> 490
+// TFLOP/s.)
+constexpr int kDecWarps = 8;
+constexpr int kGroupsPerWarp = 16 / kDecWarps;  // 16-column groups x quadrants per warp
 constexpr int kTcThreads = 32 * (kDecWarp0 + kDecWarps);
 constexpr size_t kTcSmemLimit = 226 * 1024;  // dynamic shared memory (the barriers are static)
 
@@ -492,8 +497,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
       }
     }
   } else if (warp >= kDecWarp0) {
-    // ---------------- decoders: group g, columns [16 g, 16 g + 16) of every stage
-    const int g = (warp - kDecWarp0) >> 2;
+    // ---------------- decoders: groups g0 + u kGStride, columns [16 g, 16 g + 16) of every stage
+    const int g0 = (warp - kDecWarp0) >> 2;  // this warp's groups: g0, g0 + 4 / kGroupsPerWarp, ...
+    constexpr int kGStride = 4 / kGroupsPerWarp;
     const int q = warp & 3;                  // TMEM lane quadrant
     const int r = q * 32 + lane;             // row of the tile
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
@@ -522,25 +528,29 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
     // Item i's index words (the index slot goes back to the producer), the
     // sidecar cursor moved to it, and its decoded words: hi (and mid), two
     // weights per 32-bit TMEM cell. false if a wait gave up.
-    auto fetch_decode = [&](int i, uint32_t (&hi)[8], uint32_t (&mid)[8]) -> bool {
+    auto fetch_decode = [&](int i, uint32_t (&hi)[kGroupsPerWarp][8], uint32_t (&mid)[kGroupsPerWarp][8]) -> bool {
       const int w = w0 + i, T = w / n_st, st = w - T * n_st, t = T % L.n_tiles;
       const int rows = min(kTileRows, L.N - t * kTileRows);
       if (!mbar_wait(&bar_ifull[is], iph, abrt, 0, lim)) return false;
       const uint8_t* src = ring + (size_t)is * ISLOT + r * 16;
-      uint32_t wd[4] = {0, 0, 0, 0};
-      if (r < rows) {
-        if (MODE == HXQ_MODE_SCALAR8) {
-          const uint4 v = *reinterpret_cast<const uint4*>(src + g * rows * 16);
-          wd[0] = v.x; wd[1] = v.y; wd[2] = v.z; wd[3] = v.w;
-        } else {
-          quarter_words_2d(src, rows, g, wd);
+      uint32_t wd[kGroupsPerWarp][4];
+#pragma unroll
+      for (int u = 0; u < kGroupsPerWarp; ++u) {
+        const int g = g0 + u * kGStride;
+        wd[u][0] = wd[u][1] = wd[u][2] = wd[u][3] = 0;
+        if (r < rows) {
+          if (MODE == HXQ_MODE_SCALAR8) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src + g * rows * 16);
+            wd[u][0] = v.x; wd[u][1] = v.y; wd[u][2] = v.z; wd[u][3] = v.w;
+          } else {
+            quarter_words_2d(src, rows, g, wd[u]);
+          }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_ifree[is]);
       if (++is == kIS) is = 0, iph ^= 1;
 
-      const int k0 = st * kStageK + g * 16;
       if (T != cur_T) {  // new tile: position the cursor at this stage (per-stage table)
         cur_T = T;
         const int n = t * kTileRows + r;
@@ -555,47 +565,51 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
           }
         }
       }
-      while (pkn < k0) step();  // entries in other quarters
-      if (MODE == HXQ_MODE_SCALAR8) {
-        uint32_t v[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t a = prmt(wd[j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
-          v[j] = *reinterpret_cast<const uint32_t*>(smem + a);
-        }
-        while (pkn < k0 + 16) {  // sidecar: substitute the stored value
-          patch16(v, pkn - k0, TERMS == 1 ? (bf16_bits(pvn) << 16) : split_word(pvn));
-          step();
-        }
+      for (int u = 0; u < kGroupsPerWarp; ++u) {  // groups in ascending columns
+        const int k0 = st * kStageK + (g0 + u * kGStride) * 16;
+        while (pkn < k0) step();  // entries in other quarters
+        if (MODE == HXQ_MODE_SCALAR8) {
+          uint32_t v[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) hi[j] = prmt(v[2 * j], v[2 * j + 1], 0x7632);
-        if (TERMS == 2) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) mid[j] = prmt(v[2 * j], v[2 * j + 1], 0x5410);
-        }
-      } else {
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {  // 8 pairs = 16 weights
-          const int bit = 12 * jj;
-          const uint32_t e = __funnelshift_r(wd[bit >> 5], wd[(bit >> 5) + 1], bit & 31) & 0xFFF;
-          if (TERMS == 1) {
-            hi[jj] = *reinterpret_cast<const uint32_t*>(smem + e * 4);
-          } else {
-            const uint2 hm = *reinterpret_cast<const uint2*>(smem + e * 8);
-            hi[jj] = hm.x;
-            mid[jj] = hm.y;
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t a = prmt(wd[u][j >> 2], lane4, 0x5504u | ((uint32_t)(j & 3) << 4));
+            v[j] = *reinterpret_cast<const uint32_t*>(smem + a);
           }
-        }
-        while (pkn < k0 + 16) {  // sidecar: substitute the stored value
-          const int o = pkn - k0;
-          if (TERMS == 1) {
-            patch8_half(hi, o >> 1, o & 1, bf16_bits(pvn));
-          } else {
-            const uint32_t sw = split_word(pvn);
-            patch8_half(hi, o >> 1, o & 1, sw >> 16);
-            patch8_half(mid, o >> 1, o & 1, sw & 0xFFFFu);
+          while (pkn < k0 + 16) {  // sidecar: substitute the stored value
+            patch16(v, pkn - k0, TERMS == 1 ? (bf16_bits(pvn) << 16) : split_word(pvn));
+            step();
           }
-          step();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) hi[u][j] = prmt(v[2 * j], v[2 * j + 1], 0x7632);
+          if (TERMS == 2) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mid[u][j] = prmt(v[2 * j], v[2 * j + 1], 0x5410);
+          }
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {  // 8 pairs = 16 weights
+            const int bit = 12 * jj;
+            const uint32_t e = __funnelshift_r(wd[u][bit >> 5], wd[u][(bit >> 5) + 1], bit & 31) & 0xFFF;
+            if (TERMS == 1) {
+              hi[u][jj] = *reinterpret_cast<const uint32_t*>(smem + e * 4);
+            } else {
+              const uint2 hm = *reinterpret_cast<const uint2*>(smem + e * 8);
+              hi[u][jj] = hm.x;
+              mid[u][jj] = hm.y;
+            }
+          }
+          while (pkn < k0 + 16) {  // sidecar: substitute the stored value
+            const int o = pkn - k0;
+            if (TERMS == 1) {
+              patch8_half(hi[u], o >> 1, o & 1, bf16_bits(pvn));
+            } else {
+              const uint32_t sw = split_word(pvn);
+              patch8_half(hi[u], o >> 1, o & 1, sw >> 16);
+              patch8_half(mid[u], o >> 1, o & 1, sw & 0xFFFFu);
+            }
+            step();
+          }
         }
       }
       return true;
@@ -604,14 +618,17 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
     // Software pipeline: item i's TMEM stores drain while item i + 1 is
     // fetched and decoded; then the stores are waited for and the MMA
     // thread is told that slot b holds item i.
-    uint32_t hi[8], mid[8], nhi[8], nmid[8];
+    uint32_t hi[kGroupsPerWarp][8], mid[kGroupsPerWarp][8], nhi[kGroupsPerWarp][8], nmid[kGroupsPerWarp][8];
     bool ok = n_items > 0 && fetch_decode(0, hi, mid);
     for (int i = 0; ok && i < n_items; ++i) {
       if (!mbar_wait(&bar_empty[b], bph ^ 1, abrt, 0, lim)) break;
       tc_fence_after();
-      const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS + g * 8;
-      tmem_st8(acol, hi);
-      if (TERMS == 2) tmem_st8(acol + 32, mid);
+#pragma unroll
+      for (int u = 0; u < kGroupsPerWarp; ++u) {
+        const uint32_t acol = lane_base + ACOL0 + b * 32 * TERMS + (g0 + u * kGStride) * 8;
+        tmem_st8(acol, hi[u]);
+        if (TERMS == 2) tmem_st8(acol + 32, mid[u]);
+      }
       if (i + 1 < n_items) ok = fetch_decode(i + 1, nhi, nmid);
       tmem_wait_st();
       tc_fence_before();
@@ -619,10 +636,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmx, Layer L, Out out, int M, int 
       if (lane == 0) mbar_arrive(&bar_a[b]);
       if (++b == kSlots) b = 0, bph ^= 1;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        hi[j] = nhi[j];
-        mid[j] = nmid[j];
-      }
+      for (int u = 0; u < kGroupsPerWarp; ++u)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          hi[u][j] = nhi[u][j];
+          mid[u][j] = nmid[u][j];
+        }
     }
   }
 
