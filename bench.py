@@ -160,10 +160,23 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def _code_only(text):
+    """C++ source without comments, trailing blanks and empty lines: what
+    the compiler sees of it (the kernel files hold no "//" or "/*" inside
+    string literals)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash():
+    """Hash of the kernels' code (comments excluded), recorded with each
+    ncu capture so that stale traffic figures are not reported."""
     h = hashlib.sha256()
     for f in ("hxq_gemv.cu", "hxq_tc.cu", "hxq_internal.cuh"):
-        h.update(open(os.path.join(ROOT, "vq_compressed_linear_b200", "csrc", f), "rb").read())
+        with open(os.path.join(ROOT, "vq_compressed_linear_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

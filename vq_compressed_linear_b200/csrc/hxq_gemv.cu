@@ -6,9 +6,10 @@
 //
 // Work decomposition. The layer's stages (tile of 128 rows x 64 weights along
 // K) are numbered tile-major. Two ways of cutting them, chosen per handle:
-// - cluster split: when some cluster size cs in 2..8 gives one cluster per
-//   tile that fills at least 70 % of the SMs, all clusters resident, tile t
-//   goes to cluster t and rank r of it takes the r-th of cs equal K ranges;
+// - cluster split: when some cluster size cs in 2..16 gives one cluster per
+//   tile that fills at least 70 % of the SMs (any fill for layers of a few
+//   tiles), all clusters resident, tile t goes to cluster t and rank r of it
+//   takes the r-th of cs equal K ranges;
 // - stream-K otherwise: the stages are cut into contiguous ranges of equal
 //   length, one per CTA of a persistent grid (one CTA per SM), so every CTA
 //   streams the same number of index bytes whatever the layer shape.
@@ -28,9 +29,10 @@
 // 8 consumer warps share every chunk: warp q takes the q-th 16-weight piece
 // of the chunk (stage q / 4, quarter q % 4) for all 128 rows, lane l for rows
 // l, l + 32, l + 64, l + 96. So each activation a warp loads from shared
-// memory serves four rows: the decode is bound by the shared-memory pipe, and
-// per 32 weights it costs one conflict-free table lookup wavefront plus a
-// quarter wavefront of index bytes plus the activations.
+// memory serves four rows: per 32 weights the decode costs one conflict-free
+// table lookup wavefront plus a quarter wavefront of index bytes plus the
+// activations (with 8 warps per CTA it runs below that bound, on the
+// latency of its lookup chain).
 //
 // At each tile boundary of the CTA's range the warps' sums meet in shared
 // memory. Under the cluster split every rank writes its sums into rank 0's

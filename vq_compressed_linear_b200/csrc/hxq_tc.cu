@@ -5,14 +5,15 @@
 // and B = a tile of BN tokens of x, so D = y^T for that tile and lives in
 // tensor memory (TMEM): lane = output feature, column = token.
 //
-//  * A is written by 16 decoding warps straight from registers into TMEM
+//  * A is written by 8 decoding warps straight from registers into TMEM
 //    with tcgen05.st (the "A from tensor memory" form of tcgen05.mma): the
-//    decoded weights never touch shared or global memory. Thread r of
-//    decoding group g (4 warps, one per TMEM lane quadrant) owns TMEM lane
-//    r = row r of the tile and columns [16 g, 16 g + 16) of every stage. A
+//    decoded weights never touch shared or global memory. Thread r of a
+//    decoding warp (one per TMEM lane quadrant and pair of column groups)
+//    owns TMEM lane r = row r of the tile and the columns [16 g, 16 g + 16)
+//    of its two groups g of every stage. A
 //    producer warp streams each item's index block (contiguous in the tiled
 //    layout) with TMA bulk copies into a ring of shared-memory slots; the
-//    thread reads its 16 indices from the slot, looks them up in a
+//    thread reads its 2 x 16 indices from the slot, looks them up in a
 //    shared-memory table, substitutes sidecar values, packs two bf16 per
 //    32-bit TMEM cell and stores them. All decoding warps work on the same
 //    item, so the MMA receives items at an even pace.
@@ -46,8 +47,8 @@
 // the next two entries already requested, and substitutes the stored value
 // (as bf16, or as its hi+mid split) before the store.
 //
-// Every mbarrier wait is bounded (2 s): on timeout the CTA sets a status bit,
-// drains what it issued, frees TMEM and returns.
+// Every mbarrier wait is bounded (2 s unless a test lowers it): on timeout the
+// CTA sets a status bit, drains what it issued, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
