@@ -606,6 +606,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference" and rank != 0:
+        return 0  # the oracle arm runs on rank 0 alone; the other ranks do no work
     items = workload(args.workload, 0, args.M if args.M else DEFAULT_M[args.workload])
     is_prefill = all(M > 32 for _, _, M in items)
     metric = ("HelixLinear prefill GEMM TFLOP/s" if is_prefill else "HelixLinear GEMV achieved HBM GB/s")

@@ -118,7 +118,7 @@ def test_reference_arm_encoder_line():
     one JSON line with the encoder metric and the reference fields."""
     env = dict(os.environ, RANK="0", LOCAL_RANK="0", WORLD_SIZE="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--encoder", "tiny", "--steps", "3", "--warmup", "3"],
+                        "--encoder", "tiny", "--steps", "1", "--warmup", "3"],
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     lines = [l for l in r.stdout.splitlines() if l.strip()]
